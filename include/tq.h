@@ -1,0 +1,193 @@
+/*
+ * tq.h -- TurboQuant KV-cache vector quantisation on NVIDIA B200 (sm_100a): the C ABI of libtq.
+ *
+ * The method (web write-ups of TurboQuant, arXiv 2504.19874):
+ *   Algorithm 1 (MSE): rotate a vector by a random orthogonal Pi, quantise every coordinate with a
+ *     Lloyd-Max scalar codebook precomputed for the coordinate law of a rotated unit vector, and
+ *     invert the rotation on decode (ai-navigate-news page, "how it works (technical)"; aiboss88
+ *     page, "TurboQuant technical principles"; techblog-plum page, "step 1: PolarQuant").
+ *   Algorithm 2 (inner product): Algorithm 1 at b-1 bits, then one sign bit per coordinate of
+ *     S r for the residual r, with |r|; inner products estimated from the codes are unbiased
+ *     (ai-navigate-news page, "how it works"; aiboss88 page, "two-stage residual correction";
+ *     techblog-plum page, "step 2: QJL").
+ *   Packing: indices and signs bit-packed, norms and residual norms in float16 (ai-navigate-news
+ *     page, bit-packing paragraph).
+ *   Attention on the compressed cache and vector search from the codes (aiboss88 page, features
+ *     and applications).
+ *
+ * Conventions shared by every call
+ *   - d (vector length) is a multiple of 32, 32 <= d <= 4096 (UNSUPPORTED otherwise; some calls
+ *     have narrower limits, stated below). bits of a codebook: 1..4.
+ *   - All array arguments are DEVICE pointers owned by the caller, 16-byte aligned, row-major,
+ *     unless a comment says "host". The library keeps no pointer after a call returns.
+ *   - fp16 values (norms, residual norms) are passed as raw IEEE binary16 bit patterns (uint16_t).
+ *   - Calls enqueue work on `stream` (a cudaStream_t; NULL = the legacy default stream) and return
+ *     without synchronising. Argument errors are detected on the host before anything is
+ *     enqueued; the call then returns a non-zero status and enqueues nothing.
+ *   - Kernels never trap. A device-side wait that exceeds its bound records an error that
+ *     tq_sync_check() reports as TQ_ERR_DEVICE_TIMEOUT.
+ *   - tq_last_error() returns a message for the last failing call on the calling thread.
+ *
+ * Packed layout (one vector; G = d/32 groups of 32 coordinates; L = 2^b levels)
+ *   codes  uint32 [G][b]  bit l of codes[g][p] = bit p of idx[32 g + l]      (bit planes)
+ *   signs  uint32 [G]     bit l of signs[g]    = [ (S r)_{32 g + l} >= 0 ]    (Algorithm 2)
+ *   norms  fp16           n = ||x||, round to nearest even
+ *   gammas fp16           gamma = ||r||, r = x/n - Pi^T c[idx]            (Algorithm 2)
+ *   idx_j = #{k : t_k < y_j} for y = Pi x / n (ties to the lower index); the zero vector stores
+ *   n = 0, idx_j = L/2 - 1, and for Algorithm 2 gamma = 0 with all sign bits 1.
+ *   Bytes per vector: b d/8 + 2 (Algorithm 1); (b-1) d/8 + d/8 + 4 (Algorithm 2 at b bits).
+ *   Arrays of vectors are the per-vector records above, back to back: codes [n][G][b],
+ *   signs [n][G], norms [n], gammas [n].
+ *
+ * Decode: x_hat = n (Pi^T c[idx] + alpha gamma S^T (2 z - 1)), alpha = sqrt(pi/2) / d; the last
+ * term for Algorithm 2 only. alpha makes E_S[<q, x_hat>] = <q, x> (the residual-sign estimator's
+ * scale, derived from E[s sign(<s, r>)] = sqrt(2/pi) r/|r| for a Gaussian row s).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t tq_status;
+#define TQ_OK 0
+#define TQ_ERR_INVALID_ARG 1     /* NULL / misaligned pointer, negative size, inconsistent shapes */
+#define TQ_ERR_UNSUPPORTED 2     /* d or bits outside the supported range */
+#define TQ_ERR_CUDA 3            /* a CUDA runtime call failed (message has the CUDA error) */
+#define TQ_ERR_NOT_CONVERGED 4   /* the codebook iteration did not converge */
+#define TQ_ERR_DEVICE_TIMEOUT 5  /* a bounded device-side wait gave up (see tq_sync_check) */
+#define TQ_ERR_WORKSPACE 6       /* workspace missing or smaller than the *_workspace_bytes value */
+
+/* element types of dense inputs / outputs */
+#define TQ_F32 0
+#define TQ_BF16 1
+#define TQ_F16 2
+
+/* Codebook of the Lloyd-Max quantiser for one coordinate of a rotated unit vector in R^d.
+ * Host plain-old-data; pass it by pointer to the device calls (it is copied into the launch).
+ * c: ascending centroids (first `levels` = 2^bits used); t: boundaries, t[k] between c[k] and
+ * c[k+1] (first levels-1 used). c, t are the fp32 values that define the packed format; c64,
+ * t64 the fp64 values they were rounded from. distortion = E|u - Q(u)|^2 for a unit u. */
+typedef struct tq_codebook {
+  int32_t d;
+  int32_t bits;
+  int32_t levels;
+  int32_t iterations;
+  float c[16];
+  float t[16];
+  double c64[16];
+  double t64[16];
+  double distortion;
+} tq_codebook;
+
+/* Message of the last failing call on this thread ("" if none). Never NULL. */
+TQ_API const char* tq_last_error(void);
+
+/* Library version string. */
+TQ_API const char* tq_version(void);
+
+/* Lloyd-Max codebook for the density f_d(x) ~ (1 - x^2)^((d-3)/2) on [-1, 1], the law of one
+ * coordinate of a uniformly random unit vector in R^d (aiboss88 page, technical principles:
+ * Beta-distributed coordinates, Lloyd-Max / continuous 1-D k-means; techblog-plum page: the
+ * buckets are computed once, no inference-time cost). HOST ONLY, fp64, deterministic.
+ * d >= 3 (any d, not only multiples of 32), bits in 1..4; `out` is a host pointer.
+ * Errors: INVALID_ARG (out NULL), UNSUPPORTED (d, bits), NOT_CONVERGED. */
+TQ_API tq_status tq_codebook_init(int32_t d, int32_t bits, tq_codebook* out);
+
+/* Size in bytes of the prepared-rotation buffer for dimension d. */
+TQ_API size_t tq_rotation_bytes(int32_t d);
+
+/* Prepares the rotation operands every device call reads: copies Pi and S (fp32 d x d,
+ * row-major, y = Pi x, s = S r) and derives T = S Pi^T, the transposes and the split-fp16 forms
+ * the tensor-core kernels consume. Pi must be orthogonal (the method's random rotation, drawn
+ * by the caller); S has i.i.d. N(0,1) entries (the JL matrix of the residual sign). Both are
+ * device pointers; `rot` is a caller-owned device buffer of tq_rotation_bytes(d) bytes, valid
+ * until the caller frees it or prepares it again. Asynchronous on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED (d), WORKSPACE (rot_bytes too small), CUDA. */
+TQ_API tq_status tq_rotation_prepare(int32_t d, const float* Pi, const float* S, void* rot, size_t rot_bytes,
+                              void* stream);
+
+/* Algorithm 1 encode of n vectors x [n][d] (x_dtype TQ_F32 or TQ_BF16) with a b-bit codebook
+ * (cb->d must equal d): writes codes [n][d/32][b] and norms [n] (fp16 bits).
+ * (ai-navigate-news page: Algorithm 1 = rotation, Lloyd-Max scalar quantisation, MSE-optimal;
+ * keys use it.) d in {32, 64, 96, 128, ..., 256} on the fused tensor-core path; larger d
+ * (multiples of 128 up to 4096) on the tiled path. n may be 0 (no work). */
+TQ_API tq_status tq_encode_mse(const tq_codebook* cb, int64_t n, int32_t d, const void* x, int32_t x_dtype,
+                        const void* rot, uint32_t* codes, uint16_t* norms, void* stream);
+
+/* Algorithm 2 encode at b bits: Algorithm 1 with the (b-1)-bit codebook `cb_bm1`, then the
+ * residual sign bits and the residual norm (ai-navigate-news page: Algorithm 2 = Algorithm 1 at
+ * b-1 bits plus sign(S r), unbiased inner products; values use it). Writes codes
+ * [n][d/32][b-1], signs [n][d/32], norms [n], gammas [n]. Limits as tq_encode_mse. */
+TQ_API tq_status tq_encode_prod(const tq_codebook* cb_bm1, int64_t n, int32_t d, const void* x, int32_t x_dtype,
+                         const void* rot, uint32_t* codes, uint32_t* signs, uint16_t* norms, uint16_t* gammas,
+                         void* stream);
+
+/* Dequantise n packed vectors: x_hat = n (Pi^T c[idx] (+ alpha gamma S^T (2z-1))) into
+ * out [n][d] of out_dtype (TQ_F32 or TQ_BF16). signs and gammas both NULL for Algorithm 1
+ * codes, both non-NULL for Algorithm 2 (then cb is the (b-1)-bit codebook the codes use).
+ * (ai-navigate-news page: inverse rotation after the scalar codebook.) */
+TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t d, const void* rot, const uint32_t* codes,
+                    const uint32_t* signs, const uint16_t* norms, const uint16_t* gammas, void* out,
+                    int32_t out_dtype, void* stream);
+
+/* Workspace bytes tq_scores needs for these sizes. */
+TQ_API size_t tq_scores_workspace_bytes(int64_t nq, int64_t n, int32_t d, int32_t k);
+
+/* Inner-product estimates <q, x_hat_v> of nq queries q [nq][d] (TQ_F32 / TQ_BF16) against n
+ * packed database vectors (layout as tq_decode; signs/gammas NULL for Algorithm 1 codes),
+ * computed from the codes: the query is rotated (q' = Pi q) and projected (q'' = S q) once and
+ * <q, x_hat> = n (<q', c[idx]> + alpha gamma <q'', 2z-1>) (aiboss88 page: inner-product mode,
+ * unbiased estimates; vector-database nearest-neighbour search).
+ * scores: optional [nq][n] fp32 output (NULL: not written).
+ * k: 0, or 1..16 -- then topk_ids [nq][k] (int32) and topk_scores [nq][k] receive, per query,
+ * the k largest scores in descending order, ties to the lower id (ids < 2^31).
+ * ws: caller device workspace of at least tq_scores_workspace_bytes(nq, n, d, k) bytes. */
+TQ_API tq_status tq_scores(const tq_codebook* cb, int64_t nq, int64_t n, int32_t d, const void* q, int32_t q_dtype,
+                    const void* rot, const uint32_t* codes, const uint32_t* signs, const uint16_t* norms,
+                    const uint16_t* gammas, float* scores, int32_t k, int32_t* topk_ids, float* topk_scores,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes tq_attend_decode needs for these sizes. */
+TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t T, int32_t d);
+
+/* One decode step of attention over a packed KV cache (aiboss88 page: attention computed on the
+ * quantised cache; ai-navigate-news page: keys by Algorithm 1, values by Algorithm 2):
+ *   out[b][h] = sum_t softmax_t(scale <q[b][h], k_hat[b][g][t]>) v_hat[b][g][t],  g = h / (Hq/Hkv)
+ * with k_hat, v_hat the decoded cache, evaluated from the codes: the query is rotated once,
+ * scores come from the key codes, and values are accumulated in the rotated / sign domain with
+ * Pi^T and S^T applied once per query head. No mask: every one of the T tokens is attended.
+ *   q       [B][Hq][d]  TQ_BF16 or TQ_F32
+ *   keys    Algorithm 1 with cb_k (b_k bits): k_codes [B][Hkv][T][d/32][b_k], k_norms [B][Hkv][T]
+ *   values  Algorithm 2 with cb_v the (b_v-1)-bit codebook: v_codes [B][Hkv][T][d/32][b_v-1],
+ *           v_signs [B][Hkv][T][d/32], v_norms, v_gammas [B][Hkv][T];
+ *           or Algorithm 1 (v_signs and v_gammas NULL, cb_v the b_v-bit codebook)
+ *   out     [B][Hq][d] fp32
+ * Supported: d = 128 or 64, Hq a multiple of Hkv with Hq/Hkv <= 8, T >= 1.
+ * ws: caller device workspace of at least tq_attend_workspace_bytes(...) bytes. */
+TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq, int32_t Hkv,
+                           int64_t T, int32_t d, const void* q, int32_t q_dtype, const void* rot,
+                           const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* v_codes,
+                           const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
+                           float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reports a pending CUDA error (TQ_ERR_CUDA) or a device-side
+ * timeout recorded by any libtq kernel since the last check (TQ_ERR_DEVICE_TIMEOUT, which this
+ * call clears). TQ_OK otherwise. */
+TQ_API tq_status tq_sync_check(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

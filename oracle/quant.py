@@ -123,23 +123,28 @@ def encode_mse(x: np.ndarray, Pi: np.ndarray, cb: Codebook) -> dict:
     return dict(codes=pack_planes(idx, cb.bits), norms=n16, n=n, u=u, y=y, idx=idx)
 
 
+def residual_signs(u: np.ndarray, idx: np.ndarray, n: np.ndarray, Pi: np.ndarray, S: np.ndarray,
+                   cb_bm1: Codebook) -> dict:
+    """Second stage of Algorithm 2 for given first-stage indices: r = u - Pi^T c[idx],
+    gamma = |r|, s = S r, z = [s >= 0] (zero vectors: r = 0)."""
+    c = cb_bm1.c32.astype(np.float64)
+    chat = c[idx]                                        # rotated-domain reconstruction
+    Pi64 = np.asarray(Pi, dtype=np.float64)
+    r = u - chat @ Pi64                                  # u - Pi^T c[idx], original domain
+    r[np.asarray(n) == 0] = 0.0
+    gamma = np.sqrt(np.sum(r * r, axis=1))
+    s = r @ np.asarray(S, dtype=np.float64).T            # S r
+    z = s >= 0
+    return dict(signs=pack_signs(z), gammas=gamma.astype(np.float16), gamma=gamma, r=r, s=s, z=z, chat=chat)
+
+
 def encode_prod(x: np.ndarray, Pi: np.ndarray, S: np.ndarray, cb_bm1: Codebook) -> dict:
     """Algorithm 2 at b bits = Algorithm 1 at b-1 bits (``cb_bm1``) + QJL sign of S r.
 
     Returns codes [N, d/32, b-1], signs [N, d/32], norms fp16, gammas fp16 and intermediates.
     """
     e = encode_mse(x, Pi, cb_bm1)
-    c = cb_bm1.c32.astype(np.float64)
-    chat = c[e["idx"]]                                   # rotated-domain reconstruction
-    Pi64 = np.asarray(Pi, dtype=np.float64)
-    r = e["u"] - chat @ Pi64                             # u - Pi^T c[idx], original domain
-    zero = e["n"] == 0
-    r[zero] = 0.0
-    gamma = np.sqrt(np.sum(r * r, axis=1))
-    s = r @ np.asarray(S, dtype=np.float64).T            # S r
-    z = s >= 0
-    e.update(signs=pack_signs(z), gammas=gamma.astype(np.float16), gamma=gamma, r=r, s=s, z=z,
-             chat=chat)
+    e.update(residual_signs(e["u"], e["idx"], e["n"], Pi, S, cb_bm1))
     return e
 
 

@@ -1,0 +1,87 @@
+"""libtq on the host (no GPU needed): the shared library loads, exports every symbol the header
+declares, computes the same codebook as the oracle, and rejects bad arguments before touching a
+device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_vector_encode_b200 as tq
+from oracle.codebook import distortion_per_vector, lloyd_max
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from kv_cache_vector_encode_b200 import build
+    build.build()
+    return tq.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]+?\b(tq_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert tq.tq_version().startswith("libtq")
+
+
+@pytest.mark.parametrize("d,bits", [(64, 1), (64, 2), (64, 3), (128, 1), (128, 2), (128, 3), (128, 4),
+                                    (1536, 3), (1536, 4), (3, 2), (4, 3)])
+def test_codebook_matches_oracle(L, d, bits):
+    cb = tq.tq_codebook_init(d, bits)
+    ora = lloyd_max(d, bits)
+    assert cb.d == d and cb.bits == bits and cb.levels == 1 << bits
+    c64 = np.array(cb.c64[: cb.levels])
+    t64 = np.array(cb.t64[: cb.levels - 1])
+    assert np.max(np.abs(c64 - ora.c)) <= 1e-12 * np.max(np.abs(ora.c))
+    assert np.max(np.abs(t64 - ora.t)) <= 1e-12 * np.max(np.abs(ora.c))
+    # the fp32 values that define the packed format are identical
+    assert np.array_equal(np.array(cb.c[: cb.levels], dtype=np.float32), ora.c32)
+    assert np.array_equal(np.array(cb.t[: cb.levels - 1], dtype=np.float32), ora.t32)
+    assert abs(cb.distortion - distortion_per_vector(ora)) < 1e-11
+
+
+def test_codebook_argument_errors(L):
+    out = tq.Codebook()
+    assert L.tq_codebook_init(128, 0, ctypes.byref(out)) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_codebook_init(128, 5, ctypes.byref(out)) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_codebook_init(2, 2, ctypes.byref(out)) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_codebook_init(128, 2, None) == tq.TQ_ERR_INVALID_ARG
+    assert b"NULL" in L.tq_last_error()
+    assert L.tq_codebook_init(128, 2, ctypes.byref(out)) == tq.TQ_OK
+    assert L.tq_last_error() == b""
+
+
+def test_rotation_bytes(L):
+    assert tq.tq_rotation_bytes(100) == 0          # not a multiple of 32
+    assert tq.tq_rotation_bytes(128) >= 3 * 128 * 128 * 4 + 8 * 128 * 128 * 2
+    assert tq.tq_rotation_bytes(1536) > tq.tq_rotation_bytes(128)
+
+
+def test_device_calls_reject_bad_arguments_on_host(L):
+    # validation happens before any CUDA call, so these run without a GPU
+    cb = tq.tq_codebook_init(128, 3)
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    assert L.tq_encode_mse(ctypes.byref(cb), 10, 128, good, tq.TQ_BF16, good, None, good, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_encode_mse(ctypes.byref(cb), -1, 128, good, tq.TQ_BF16, good, good, good, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_encode_mse(ctypes.byref(cb), 10, 100, good, tq.TQ_BF16, good, good, good, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse(ctypes.byref(cb), 10, 64, good, tq.TQ_BF16, good, good, good, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_encode_mse(ctypes.byref(cb), 10, 128, P((1 << 20) + 4), tq.TQ_BF16, good, good, good, None) \
+        == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_encode_mse(ctypes.byref(cb), 10, 128, good, tq.TQ_F16, good, good, good, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse(ctypes.byref(cb), 0, 128, good, tq.TQ_BF16, good, good, good, None) == tq.TQ_OK
+    assert L.tq_encode_prod(ctypes.byref(cb), 10, 128, good, tq.TQ_BF16, good, good, None, good, good, None) \
+        == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_decode(ctypes.byref(cb), 10, 128, good, good, good, good, None, good, tq.TQ_F32, None) \
+        == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_rotation_prepare(128, good, good, good, 16, None) == tq.TQ_ERR_WORKSPACE
