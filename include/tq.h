@@ -173,7 +173,8 @@ TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int6
  *           v_signs [B][Hkv][T][d/32], v_norms, v_gammas [B][Hkv][T];
  *           or Algorithm 1 (v_signs and v_gammas NULL, cb_v the b_v-bit codebook)
  *   out     [B][Hq][d] fp32
- * Supported: d = 128 or 64, Hq a multiple of Hkv with Hq/Hkv <= 8, T >= 1.
+ * Supported: d = 128, Hq a multiple of Hkv with Hq/Hkv <= 8, T >= 1, key codebooks of 1..3 bits,
+ * value codebooks of 1..2 bits (Algorithm 2 values at 2..3 bits, Algorithm 1 values at 1..2 bits).
  * ws: caller device workspace of at least tq_attend_workspace_bytes(...) bytes. */
 TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq, int32_t Hkv,
                            int64_t T, int32_t d, const void* q, int32_t q_dtype, const void* rot,

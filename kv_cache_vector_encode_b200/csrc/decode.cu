@@ -9,8 +9,9 @@
 // vector, so an epilogue warp writes 32 consecutive floats of a row per store.
 //   D1a = PiT_hi c_hi,  D1b = PiT_lo c_hi + PiT_hi c_lo,  D2a = ST_hi s,  D2b = ST_lo s
 //   x_hat = n ((D1a + 2^-12 D1b) + alpha gamma (D2a + 2^-12 D2b))
-// Roles (10 warps): warp 1 owns TMEM and issues MMAs; warps 2-5 load the packed tile and write the
-// B operands; warps 6-9 are the epilogue. All waits are bounded.
+// Roles (14 warps): warp 0 bulk-copies the resident operands; warp 1 owns TMEM and issues MMAs;
+// warps 2-5 unpack (one thread per (vector, 32-coordinate group), 16-byte swizzled stores);
+// warps 6-13 are the epilogue (two warps per TMEM lane quarter). All waits are bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -23,101 +24,92 @@
 namespace tq {
 namespace {
 
-constexpr int kDecThreads = 320;
+constexpr int kDecThreads = 448;
 
 struct DecodeParams {
   int64_t n;
-  int d, G, bits, KP, ntiles, dp;
-  const __half* pit_hi;
-  const __half* pit_lo;
-  const __half* st_hi;
-  const __half* st_lo;
+  int d, G, KP, ntiles;
+  const uint8_t* img[4];     // PiT_hi, PiT_lo, ST_hi, ST_lo shared-memory images (band 0)
+  uint32_t img_bytes;
   const uint32_t* codes;
   const uint32_t* signs;
   const uint16_t* norms;
   const uint16_t* gammas;
   void* out;
   float alpha;
-  uint16_t c_hi[16], c_lo[16];
+  uint32_t lut_hi[8], lut_lo[8];   // c_hi / c_lo (fp16) of the 16 levels, two per word
   uint32_t* err;
 };
 
 struct DecLayout {
   uint32_t a_bytes, b_bytes;
-  uint32_t off_a[4], off_b[3], off_codes, off_signs, off_info, off_bar, total;
+  uint32_t off_a[4], off_b[3], off_info, off_bar, total;
 };
 
 __host__ __device__ inline uint32_t dround(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <bool ALG2>
-__host__ __device__ inline DecLayout dec_layout(int KP, int NV, int G, int bits) {
+__host__ __device__ inline DecLayout dec_layout(int KP, int NV) {
   DecLayout L{};
   L.a_bytes = 128u * KP * 2;
   L.b_bytes = (uint32_t)NV * KP * 2;
   uint32_t off = 0;
   for (int i = 0; i < (ALG2 ? 4 : 2); ++i) { L.off_a[i] = off; off += L.a_bytes; }
   for (int i = 0; i < (ALG2 ? 3 : 2); ++i) { L.off_b[i] = off; off += L.b_bytes; }
-  L.off_codes = off; off += dround((uint32_t)NV * G * bits * 4, 128);
-  L.off_signs = off; off += dround((uint32_t)NV * G * 4, 128);
   L.off_info = off; off += 2u * 2 * NV * 4;     // [2 buffers][norm, alpha*gamma][NV]
   L.off_bar = dround(off, 8); off = L.off_bar + 16 * 8;
   L.total = off + 1024;
   return L;
 }
 
-enum DBars { B_FULL = 0, B_EMPTY = 1, ACC_FULL = 2, ACC_EMPTY = 4, INFO_EMPTY = 6, UNP = 8, DNBARS = 9 };
+enum DBars { A_FULL = 0, B_FULL = 1, B_EMPTY = 2, ACC_FULL = 3, ACC_EMPTY = 5, INFO_EMPTY = 7, DNBARS = 9 };
 
-template <bool ALG2, int NV, bool OUT_BF16>
+__device__ __forceinline__ uint32_t pack_h2(uint32_t a, uint32_t b) { return (a & 0xFFFFu) | (b << 16); }
+
+template <bool ALG2, int NV, bool OUT_BF16, int BITS>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;
   constexpr uint32_t NCOLS = 2 * COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const DecLayout Lo = dec_layout<ALG2>(p.KP, NV, p.G, p.bits);
+  const DecLayout Lo = dec_layout<ALG2>(p.KP, NV);
   uint64_t* bar = (uint64_t*)(smem + Lo.off_bar);
   uint32_t* tmem_slot = (uint32_t*)(bar + DNBARS);
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + DNBARS) + 1;
   float* info = (float*)(smem + Lo.off_info);
-  uint32_t* scodes = (uint32_t*)(smem + Lo.off_codes);
-  uint32_t* ssigns = (uint32_t*)(smem + Lo.off_signs);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int d = p.d, KP = p.KP, G = p.G, bits = p.bits;
+  const int d = p.d, KP = p.KP, G = p.G;
+  constexpr int na = ALG2 ? 4 : 2;
 
-  {
-    const __half* srcs[4] = {p.pit_hi, p.pit_lo, p.st_hi, p.st_lo};
-    const int chunks = KP / 8;
-#pragma unroll
-    for (int m = 0; m < (ALG2 ? 4 : 2); ++m) {
-      uint8_t* dst = smem + Lo.off_a[m];
-      for (int c = tid; c < 128 * chunks; c += kDecThreads) {
-        int r = c / chunks, kc = c % chunks;
-        *(uint4*)(dst + sw128_offset(r, kc * 16, 128)) = *(const uint4*)(srcs[m] + (size_t)r * p.dp + kc * 8);
-      }
+  if (tid == 0) {
+    mbar_init(&bar[A_FULL], 1);
+    mbar_init(&bar[B_FULL], 4);                // one arrival per unpacker warp
+    mbar_init(&bar[B_EMPTY], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[ACC_FULL + s], 1);
+      mbar_init(&bar[ACC_EMPTY + s], 8);       // one arrival per epilogue warp
+      mbar_init(&bar[INFO_EMPTY + s], 8);
     }
-    if (tid == 0) {
-      mbar_init(&bar[B_FULL], 128);
-      mbar_init(&bar[B_EMPTY], 1);
-      mbar_init(&bar[ACC_FULL], 1); mbar_init(&bar[ACC_FULL + 1], 1);
-      mbar_init(&bar[ACC_EMPTY], 128); mbar_init(&bar[ACC_EMPTY + 1], 128);
-      mbar_init(&bar[INFO_EMPTY], 128); mbar_init(&bar[INFO_EMPTY + 1], 128);
-      mbar_init(&bar[UNP], 128);
-      *abort_flag = 0;
-      fence_mbar_init();
-    }
-    fence_proxy_async_smem();
-    if (warp == 1) {
-      tmem_alloc(tmem_slot, NCOLS);
-      tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, NCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const int my_tiles = p.ntiles > (int)blockIdx.x ? (p.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-  if (warp == 1) {
+  if (warp == 0) {
     if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[A_FULL], na * p.img_bytes);
+      for (int m = 0; m < na; ++m) bulk_g2s(smem + Lo.off_a[m], p.img[m], p.img_bytes, &bar[A_FULL]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && mbar_wait(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
@@ -147,41 +139,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         mma_commit(&bar[ACC_FULL + a]);
       }
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp < 6) {
     // ---------------- unpackers: codes -> fp16 B operands -----------------------------------------
     const int ut = tid - 64;               // 0..127
-    const int q = ut >> 5;                 // group handled by this warp
-    const int i = q * 32 + lane;           // coordinate handled by this thread
-    __shared__ __half lut_hi[16], lut_lo[16];
-    uint32_t unp_uses = 0;
-    // bounded group barrier of the 128 unpacker threads
-    auto unp_sync = [&]() -> bool {
-      mbar_arrive(&bar[UNP]);
-      const bool ok = mbar_wait(&bar[UNP], unp_uses & 1, p.err, kDevTimeoutSync, abort_flag);
-      ++unp_uses;
-      return ok;
-    };
-    if (ut < 16) {
-      lut_hi[ut] = __ushort_as_half(p.c_hi[ut]);
-      lut_lo[ut] = __ushort_as_half(p.c_lo[ut]);
+    uint32_t lhi[8], llo[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      lhi[h] = p.lut_hi[h];
+      llo[h] = p.lut_lo[h];
     }
-    bool ok = unp_sync();
-    for (int k = 0; k < my_tiles && ok; ++k) {
+    // 16-entry fp16 table held as 8 words; entry idx = half (idx & 1) of word idx >> 1
+    auto lut = [](const uint32_t (&t)[8], int idx) -> uint32_t {
+      uint32_t w = t[0];
+#pragma unroll
+      for (int h = 1; h < (1 << BITS) / 2; ++h) w = (idx >> 1) == h ? t[h] : w;
+      return (idx & 1) ? (w >> 16) : (w & 0xFFFFu);
+    };
+    uint8_t* bch = smem + Lo.off_b[0];
+    uint8_t* bcl = smem + Lo.off_b[1];
+    uint8_t* bsg = ALG2 ? smem + Lo.off_b[2] : nullptr;
+    const int gp = KP / 32;                  // groups per operand row (padding groups included)
+    const int units = NV * gp;
+    for (int k = 0; k < my_tiles; ++k) {
       const int a = k & 1;
       const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
-      // stage the packed words of the tile (coalesced loads)
-      {
-        const int nw = rows * G * bits;
-        const uint32_t* src = p.codes + v0 * G * bits;
-        for (int w = ut; w < nw; w += 128) scodes[w] = __ldg(src + w);
-        if (ALG2) {
-          const int ns = rows * G;
-          const uint32_t* ss = p.signs + v0 * G;
-          for (int w = ut; w < ns; w += 128) ssigns[w] = __ldg(ss + w);
-        }
-      }
-      if (!mbar_wait(&bar[INFO_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[INFO_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
       if (ut < NV) {
         float nv = 0.0f, ag = 0.0f;
         if (ut < rows) {
@@ -191,46 +174,60 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         info[(a * 2 + 0) * NV + ut] = nv;
         info[(a * 2 + 1) * NV + ut] = ag;
       }
-      if (!unp_sync()) break;   // staged words visible to all unpackers
-      if (!mbar_wait(&bar[B_EMPTY], (k & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      uint8_t* bch = smem + Lo.off_b[0];
-      uint8_t* bcl = smem + Lo.off_b[1];
-      uint8_t* bsg = ALG2 ? smem + Lo.off_b[2] : nullptr;
-      if (i < KP) {
-        for (int v = 0; v < NV; ++v) {
-          __half ch = __float2half_rn(0.0f), cl = ch, sg = ch;
-          if (v < rows && i < d) {
-            const uint32_t* wv = scodes + (v * G + q) * bits;
-            int idx = 0;
-            for (int pl = 0; pl < bits; ++pl) idx |= ((wv[pl] >> lane) & 1u) << pl;
-            ch = lut_hi[idx];
-            cl = lut_lo[idx];
-            if (ALG2) sg = ((ssigns[v * G + q] >> lane) & 1u) ? __float2half_rn(1.0f) : __float2half_rn(-1.0f);
+      if (!mbar_wait_warp(&bar[B_EMPTY], (k & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      for (int u = ut; u < units; u += 128) {
+        const int v = u / gp, g = u % gp;
+        const bool live = v < rows && g < G;
+        uint32_t w[BITS], sg = 0;
+#pragma unroll
+        for (int pl = 0; pl < BITS; ++pl) w[pl] = live ? __ldg(p.codes + ((v0 + v) * G + g) * BITS + pl) : 0u;
+        if (ALG2) sg = live ? __ldg(p.signs + (v0 + v) * G + g) : 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {           // four 8-coordinate chunks of the group
+          uint32_t hi4[4], lo4[4], s4[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            uint32_t hv[2], lv[2], sv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int bit = 8 * c + 2 * h + e;
+              int idx = 0;
+#pragma unroll
+              for (int pl = 0; pl < BITS; ++pl) idx |= (int)((w[pl] >> bit) & 1u) << pl;
+              hv[e] = live ? lut(lhi, idx) : 0u;
+              lv[e] = live ? lut(llo, idx) : 0u;
+              sv[e] = live ? (((sg >> bit) & 1u) ? 0x3C00u : 0xBC00u) : 0u;
+            }
+            hi4[h] = pack_h2(hv[0], hv[1]);
+            lo4[h] = pack_h2(lv[0], lv[1]);
+            s4[h] = pack_h2(sv[0], sv[1]);
           }
-          const uint32_t off = sw128_offset(v, 2 * i, NV);
-          *(__half*)(bch + off) = ch;
-          *(__half*)(bcl + off) = cl;
-          if (ALG2) *(__half*)(bsg + off) = sg;
+          const uint32_t off = sw128_offset(v, (g * 32 + c * 8) * 2, NV);
+          *(uint4*)(bch + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+          *(uint4*)(bcl + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+          if (ALG2) *(uint4*)(bsg + off) = make_uint4(s4[0], s4[1], s4[2], s4[3]);
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bar[B_FULL]);
-      ok = unp_sync();          // staging reused by the next tile
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_FULL]);
     }
-  } else if (warp >= 6) {
+  } else {
     // ---------------- epilogue ----------------------------------------------------------------------
+    const int e = warp - 6;
     const int q = warp & 3;
     const int j = q * 32 + lane;          // output coordinate
     const bool active = j < d;
+    const int cbeg = (e >> 2) * (NV / 2), cend = cbeg + NV / 2;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     for (int k = 0; k < my_tiles; ++k) {
       const int a = k & 1;
       const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
-      if (!mbar_wait(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
       const uint32_t d1a = tbase + lane_base + a * COLS, d1b = d1a + NV, d2a = d1a + 2 * NV, d2b = d1a + 3 * NV;
-      for (int c0 = 0; c0 < NV; c0 += 16) {
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
         uint32_t ra[16], rb[16], rc[16], rd[16];
         tmem_ld16(d1a + c0, ra);
         tmem_ld16(d1b + c0, rb);
@@ -259,8 +256,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar[ACC_EMPTY + a]);
-      mbar_arrive(&bar[INFO_EMPTY + a]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[ACC_EMPTY + a]);
+        mbar_arrive(&bar[INFO_EMPTY + a]);
+      }
     }
   }
 
@@ -272,10 +272,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   }
 }
 
-template <bool ALG2, int NV, bool BF16>
+template <bool ALG2, int NV, bool BF16, int BITS>
 tq_status launch_decode(DecodeParams& p, cudaStream_t st) {
-  const DecLayout Lo = dec_layout<ALG2>(p.KP, NV, p.G, p.bits);
-  auto kern = decode_kernel<ALG2, NV, BF16>;
+  const DecLayout Lo = dec_layout<ALG2>(p.KP, NV);
+  auto kern = decode_kernel<ALG2, NV, BF16, BITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "tq_decode: shared memory attribute");
   p.ntiles = (int)((p.n + NV - 1) / NV);
@@ -285,14 +285,24 @@ tq_status launch_decode(DecodeParams& p, cudaStream_t st) {
   return TQ_OK;
 }
 
+template <bool ALG2, int NV, bool BF16>
+tq_status decode_bits(DecodeParams& p, int bits, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_decode<ALG2, NV, BF16, 1>(p, st);
+    case 2: return launch_decode<ALG2, NV, BF16, 2>(p, st);
+    case 3: return launch_decode<ALG2, NV, BF16, 3>(p, st);
+    default: return launch_decode<ALG2, NV, BF16, 4>(p, st);
+  }
+}
+
 }  // namespace
 }  // namespace tq
 
 using namespace tq;
 
-extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t d, const void* rot, const uint32_t* codes,
-                               const uint32_t* signs, const uint16_t* norms, const uint16_t* gammas, void* out,
-                               int32_t out_dtype, void* stream) {
+extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t d, const void* rot,
+                                      const uint32_t* codes, const uint32_t* signs, const uint16_t* norms,
+                                      const uint16_t* gammas, void* out, int32_t out_dtype, void* stream) {
   clear_error();
   if (!cb || !rot || !codes || !norms || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode: NULL pointer");
   if ((signs == nullptr) != (gammas == nullptr))
@@ -308,35 +318,39 @@ extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t 
   if (n == 0) return TQ_OK;
   if (d > 128) return fail(TQ_ERR_UNSUPPORTED, "tq_decode: d > 128 is not supported by this build");
   RotLayout RL = rot_layout(d);
-  const char* base = (const char*)rot;
+  const uint8_t* base = (const uint8_t*)rot;
   DecodeParams p{};
   p.n = n;
   p.d = d;
   p.G = d / 32;
-  p.bits = cb->bits;
   p.KP = d <= 64 ? 64 : 128;
-  p.dp = RL.dp;
-  p.pit_hi = (const __half*)(base + RL.pit_hi);
-  p.pit_lo = (const __half*)(base + RL.pit_lo);
-  p.st_hi = (const __half*)(base + RL.st_hi);
-  p.st_lo = (const __half*)(base + RL.st_lo);
+  p.img[0] = base + RL.pit_hi;
+  p.img[1] = base + RL.pit_lo;
+  p.img[2] = base + RL.st_hi;
+  p.img[3] = base + RL.st_lo;
+  p.img_bytes = 128u * p.KP * 2;
   p.codes = codes;
   p.signs = signs;
   p.norms = norms;
   p.gammas = gammas;
   p.out = out;
   p.alpha = (float)(std::sqrt(M_PI / 2.0) / d);
+  uint16_t hi[16], lo[16];
   for (int k = 0; k < 16; ++k) {
     float c = k < cb->levels ? cb->c[k] : 0.0f;
     __half h = __float2half_rn(c);
     __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
-    p.c_hi[k] = __half_as_ushort(h);
-    p.c_lo[k] = __half_as_ushort(l);
+    hi[k] = __half_as_ushort(h);
+    lo[k] = __half_as_ushort(l);
+  }
+  for (int k = 0; k < 8; ++k) {
+    p.lut_hi[k] = (uint32_t)hi[2 * k] | ((uint32_t)hi[2 * k + 1] << 16);
+    p.lut_lo[k] = (uint32_t)lo[2 * k] | ((uint32_t)lo[2 * k + 1] << 16);
   }
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, "tq_decode: no device error word (is a CUDA device present?)");
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf = out_dtype == TQ_BF16;
-  if (signs) return bf ? launch_decode<true, 64, true>(p, st) : launch_decode<true, 64, false>(p, st);
-  return bf ? launch_decode<false, 128, true>(p, st) : launch_decode<false, 128, false>(p, st);
+  if (signs) return bf ? decode_bits<true, 64, true>(p, cb->bits, st) : decode_bits<true, 64, false>(p, cb->bits, st);
+  return bf ? decode_bits<false, 128, true>(p, cb->bits, st) : decode_bits<false, 128, false>(p, cb->bits, st);
 }

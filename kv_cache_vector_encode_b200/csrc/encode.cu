@@ -13,6 +13,10 @@
 // vector of the tile, so the 32 lanes of an epilogue warp are the 32 coordinates of one packing
 // group and each bit plane word is a single __ballot_sync.
 //
+// Quantiser: the Lloyd-Max codebook is exactly symmetric (c_{L-1-k} = -c_k, t_{L/2-1} = 0), so the
+// top index bit is [y > 0] and the lower bits are m XOR [y <= 0], where m counts the positive
+// boundaries below |y| (a binary search of BITS-1 compares); c[idx] = +-C[m].
+//
 // Precision: x is scaled per vector by a power of two so |x| lies in [2^14, 2^15) and converted to
 // fp16 (exact for bf16 input; fp32 input is split hi + 2^-12 lo). Pi = Pi_hi + 2^-12 Pi_lo. The
 // products are exact in the tensor core and accumulate in fp32 in TMEM:
@@ -20,10 +24,16 @@
 // The QJL projection uses rho scaled by 2^14 and split the same way, with three products
 // (T_hi rho_hi, T_lo rho_hi, T_hi rho_lo). Relative error about 2^-22, far inside the 1e-5 band.
 //
-// Roles (10 warps): warp 0 issues bulk copies of raw input tiles (TMA engine); warp 1 owns TMEM
-// and one lane issues every MMA; warps 2-5 convert a raw tile into the fp16 B operand and compute
-// the norms; warps 6-9 are the epilogue (TMEM -> quantise -> ballot -> store). Buffers: raw input
-// x2, B operand x1, TMEM accumulators x2. All waits are bounded (sm100.cuh).
+// Data movement: the resident operands arrive by one bulk copy each (the prepared rotation buffer
+// stores them as shared-memory images); input tiles arrive by 2-D TMA loads with 128-byte swizzle,
+// i.e. already in the tensor-core operand layout, with out-of-range rows / columns zero-filled.
+// bf16 tiles are converted to fp16 in place.
+//
+// Roles (14 warps): warp 0 issues the bulk / TMA copies; warp 1 owns TMEM and one lane issues every
+// MMA; warps 2-5 convert (one thread per vector: norm, power-of-two scale, fp16); warps 6-13 are
+// the epilogue (two warps per TMEM lane quarter, splitting the vectors of a tile). Buffers: input
+// stage x2, TMEM accumulators x2. All waits are bounded (sm100.cuh).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -34,67 +44,70 @@
 namespace tq {
 namespace {
 
-constexpr int kEncThreads = 320;
+constexpr int kEncThreads = 448;
 constexpr float kRhoScale = 16384.0f;   // 2^14: |rho| < 2 keeps rho * 2^14 below the fp16 maximum
 
 struct EncodeParams {
-  const void* x;
   int64_t n;
-  int d, G, bits, L, KP, ntiles;
-  const __half* pi_hi;
-  const __half* pi_lo;
-  const __half* t_hi;
-  const __half* t_lo;
-  int dp;
+  int d, G, KP, ntiles;
+  const uint8_t* img[4];     // Pi_hi, Pi_lo, T_hi, T_lo shared-memory images (band 0)
+  uint32_t img_bytes;        // bytes of one resident operand (128 rows x KP fp16)
   uint32_t* codes;
   uint32_t* signs;
   uint16_t* norms;
   uint16_t* gammas;
-  float thr[16];
-  float cent[16];
+  float P[8];                // positive boundaries t_{L/2} .. t_{L-2}
+  float C[8];                // positive centroids c_{L/2} .. c_{L-1}
   uint32_t* err;
 };
 
 struct EncLayout {
   uint32_t a_bytes, raw_bytes, bx_bytes;
-  uint32_t off_a[4], off_raw[2], off_bx[2], off_rho[2];
-  uint32_t off_codes, off_signs, off_info, off_gpart, off_lut, off_bar;
+  uint32_t off_a[4], off_raw[2], off_bx[2][2], off_rho[2];
+  uint32_t off_codes, off_signs, off_info, off_gpart, off_bar;
   uint32_t total;
 };
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <int ES, bool ALG2, bool SPLITX>
-__host__ __device__ inline EncLayout enc_layout(int d, int KP, int NV, int G, int bits) {
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+
+// raw tile: bf16 -> NV rows x KP columns (KP/64 boxes of 64 columns); fp32 -> NV rows x DF columns
+// (DF = d rounded up to 32, DF/32 boxes of 32 columns).
+template <int XT, bool ALG2, int NV, int BITS>
+__host__ __device__ inline EncLayout enc_layout(int d, int KP, int G) {
+  constexpr bool F32 = XT == TQ_F32;
   EncLayout L{};
   L.a_bytes = 128u * KP * 2;
-  L.raw_bytes = round_up((uint32_t)NV * d * ES, 1024);
+  L.raw_bytes = F32 ? (uint32_t)NV * round_up(d, 32) * 4 : (uint32_t)NV * KP * 2;
   L.bx_bytes = (uint32_t)NV * KP * 2;
   uint32_t off = 0;
-  int na = ALG2 ? 4 : 2;
-  for (int i = 0; i < na; ++i) { L.off_a[i] = off; off += L.a_bytes; }
-  for (int i = 0; i < 2; ++i) { L.off_raw[i] = off; off += L.raw_bytes; }
-  for (int i = 0; i < (SPLITX ? 2 : 1); ++i) { L.off_bx[i] = off; off += L.bx_bytes; }
+  for (int i = 0; i < (ALG2 ? 4 : 2); ++i) { L.off_a[i] = off; off += L.a_bytes; }
+  for (int s = 0; s < 2; ++s) { L.off_raw[s] = off; off += round_up(L.raw_bytes, 1024); }
+  if (F32)
+    for (int s = 0; s < 2; ++s)
+      for (int h = 0; h < 2; ++h) { L.off_bx[s][h] = off; off += L.bx_bytes; }
   if (ALG2)
-    for (int i = 0; i < 2; ++i) { L.off_rho[i] = off; off += L.bx_bytes; }
-  L.off_codes = off; off += round_up((uint32_t)NV * G * bits * 4, 128);
+    for (int h = 0; h < 2; ++h) { L.off_rho[h] = off; off += L.bx_bytes; }
+  L.off_codes = off; off += round_up((uint32_t)NV * G * BITS * 4, 128);
   L.off_signs = off; off += round_up((uint32_t)NV * G * 4, 128);
   L.off_info = off; off += 2u * NV * 4;
   L.off_gpart = off; off += 4u * NV * 4;
-  L.off_lut = off; off += 16 * 4;
   L.off_bar = round_up(off, 8); off = L.off_bar + 32 * 8;
   L.total = off + 1024;  // slack for 1024-byte alignment of the dynamic buffer
   return L;
 }
 
 enum Bars {
-  RAW_FULL = 0, RAW_EMPTY = 2, BX_FULL = 4, BX_EMPTY = 5, ACC_FULL = 6, ACC_EMPTY = 8, INFO_EMPTY = 10,
-  RHO_FULL = 12, T_FULL = 13, EPI = 15, NBARS = 16
+  A_FULL = 0, RAW_FULL = 1, STAGE_EMPTY = 3, STAGE_READY = 5, ACC_FULL = 7, ACC_EMPTY = 9, INFO_EMPTY = 11,
+  RHO_FULL = 13, T_FULL = 14, EPI = 16, NBARS = 17
 };
 
-__device__ __forceinline__ float transpose_reduce32(float (&r)[32], int lane) {
+// Sum over the 32 lanes of r[lane & 15] for 16 values per lane: lane l (and l ^ 16) gets the total
+// for column l & 15.
+__device__ __forceinline__ float transpose_reduce16(float (&r)[16], int lane) {
 #pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
+  for (int s = 8; s >= 1; s >>= 1) {
     const bool upper = (lane & s) != 0;
 #pragma unroll
     for (int j = 0; j < s; ++j) {
@@ -103,99 +116,118 @@ __device__ __forceinline__ float transpose_reduce32(float (&r)[32], int lane) {
       r[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
     }
   }
-  return r[0];
+  return r[0] + __shfl_xor_sync(0xffffffffu, r[0], 16);
 }
 
-__device__ __forceinline__ float load_x(const uint8_t* row, int k, int ES) {
-  if (ES == 2) {
-    uint32_t b = *(const uint16_t*)(row + 2 * k);
-    return __uint_as_float(b << 16);
+// m = #{positive boundaries < a} by binary search over the H-1 positive boundaries.
+template <int BITS>
+__device__ __forceinline__ int sym_m(float a, const float (&P)[8]) {
+  if (BITS == 1) return 0;
+  if (BITS == 2) return a > P[0] ? 1 : 0;
+  if (BITS == 3) {
+    const int m1 = a > P[1] ? 1 : 0;
+    const int m0 = a > (m1 ? P[2] : P[0]) ? 1 : 0;
+    return 2 * m1 + m0;
   }
-  return *(const float*)(row + 4 * k);
+  const int m2 = a > P[3] ? 1 : 0;
+  const int m1 = a > (m2 ? P[5] : P[1]) ? 1 : 0;
+  const float p0 = m2 ? (m1 ? P[6] : P[4]) : (m1 ? P[2] : P[0]);
+  const int m0 = a > p0 ? 1 : 0;
+  return 4 * m2 + 2 * m1 + m0;
 }
 
-template <int XT, bool ALG2, int NV>
-__global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_constant__ EncodeParams p) {
-  constexpr int ES = XT == TQ_BF16 ? 2 : 4;
-  constexpr bool SPLITX = XT == TQ_F32;
+template <int BITS>
+__device__ __forceinline__ float sym_c(int m, const float (&C)[8]) {
+  if (BITS == 1) return C[0];
+  if (BITS == 2) return m ? C[1] : C[0];
+  if (BITS == 3) return (m & 2) ? ((m & 1) ? C[3] : C[2]) : ((m & 1) ? C[1] : C[0]);
+  const float lo = (m & 2) ? ((m & 1) ? C[3] : C[2]) : ((m & 1) ? C[1] : C[0]);
+  const float hi = (m & 2) ? ((m & 1) ? C[7] : C[6]) : ((m & 1) ? C[5] : C[4]);
+  return (m & 4) ? hi : lo;
+}
+
+// two exact power-of-two factors whose product is 2^e (e may exceed the fp32 exponent range)
+__device__ __forceinline__ void pow2_pair(int e, float& f1, float& f2) {
+  const int e1 = max(min(e, 120), -120);
+  f1 = __int_as_float((127 + e1) << 23);
+  f2 = __int_as_float((127 + (e - e1)) << 23);
+}
+
+template <int XT, bool ALG2, int NV, int BITS>
+__global__ void __launch_bounds__(kEncThreads, 1)
+    encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  constexpr bool F32 = XT == TQ_F32;
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;       // TMEM columns per accumulator buffer
   constexpr uint32_t NCOLS = 2 * COLS;
+  constexpr int TPV = 128 / NV;                            // converter threads per vector
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const EncLayout Lo = enc_layout<ES, ALG2, SPLITX>(p.d, p.KP, NV, p.G, p.bits);
+  const int d = p.d, KP = p.KP, G = p.G;
+  const EncLayout Lo = enc_layout<XT, ALG2, NV, BITS>(d, KP, G);
   uint64_t* bar = (uint64_t*)(smem + Lo.off_bar);
   uint32_t* tmem_slot = (uint32_t*)(bar + NBARS);
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + NBARS) + 1;
   float* info = (float*)(smem + Lo.off_info);
   float* gpart = (float*)(smem + Lo.off_gpart);
-  float* lut = (float*)(smem + Lo.off_lut);
   uint32_t* codes_stage = (uint32_t*)(smem + Lo.off_codes);
   uint32_t* signs_stage = (uint32_t*)(smem + Lo.off_signs);
-
+  // stage-indexed buffers by arithmetic (keeps the layout struct out of local memory)
+  const uint32_t raw0 = Lo.off_raw[0], raw_stride = Lo.off_raw[1] - Lo.off_raw[0];
+  const uint32_t bx0 = F32 ? Lo.off_bx[0][0] : 0u, bx_stride = F32 ? Lo.off_bx[1][0] - Lo.off_bx[0][0] : 0u;
+  const uint32_t bx_lo = F32 ? Lo.off_bx[0][1] - Lo.off_bx[0][0] : 0u;
+  auto raw_off = [&](int s) { return raw0 + s * raw_stride; };
+  auto bxh_off = [&](int s) { return bx0 + s * bx_stride; };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int d = p.d, KP = p.KP, G = p.G, bits = p.bits;
 
-  // ---- set-up: resident A operands, barriers, TMEM --------------------------------------------
-  {
-    const __half* srcs[4] = {p.pi_hi, p.pi_lo, p.t_hi, p.t_lo};
-    const int na = ALG2 ? 4 : 2;
-    const int chunks = KP / 8;   // 16-byte chunks per row
-    for (int m = 0; m < na; ++m) {
-      uint8_t* dst = smem + Lo.off_a[m];
-      for (int c = tid; c < 128 * chunks; c += kEncThreads) {
-        int r = c / chunks, kc = c % chunks;
-        uint4 v = *(const uint4*)(srcs[m] + (size_t)r * p.dp + kc * 8);
-        *(uint4*)(dst + sw128_offset(r, kc * 16, 128)) = v;
-      }
+  if (tid == 0) {
+    mbar_init(&bar[A_FULL], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[RAW_FULL + s], 1);
+      mbar_init(&bar[STAGE_EMPTY + s], 1);
+      mbar_init(&bar[STAGE_READY + s], 4);     // one arrival per converter warp
+      mbar_init(&bar[ACC_FULL + s], 1);
+      mbar_init(&bar[ACC_EMPTY + s], 8);       // one arrival per epilogue warp
+      mbar_init(&bar[INFO_EMPTY + s], 8);
+      mbar_init(&bar[T_FULL + s], 1);
     }
-    if (tid < 16) lut[tid] = p.cent[tid];
-    if (tid == 0) {
-      mbar_init(&bar[RAW_FULL], 1); mbar_init(&bar[RAW_FULL + 1], 1);
-      mbar_init(&bar[RAW_EMPTY], 128); mbar_init(&bar[RAW_EMPTY + 1], 128);
-      mbar_init(&bar[BX_FULL], 128); mbar_init(&bar[BX_EMPTY], 1);
-      mbar_init(&bar[ACC_FULL], 1); mbar_init(&bar[ACC_FULL + 1], 1);
-      mbar_init(&bar[ACC_EMPTY], 128); mbar_init(&bar[ACC_EMPTY + 1], 128);
-      mbar_init(&bar[INFO_EMPTY], 128); mbar_init(&bar[INFO_EMPTY + 1], 128);
-      mbar_init(&bar[RHO_FULL], 128);
-      mbar_init(&bar[T_FULL], 1); mbar_init(&bar[T_FULL + 1], 1);
-      mbar_init(&bar[EPI], 128);
-      *abort_flag = 0;
-      fence_mbar_init();
-    }
-    fence_proxy_async_smem();
-    if (warp == 1) {
-      tmem_alloc(tmem_slot, NCOLS);
-      tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    mbar_init(&bar[RHO_FULL], 8);
+    mbar_init(&bar[EPI], 8);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, NCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const int my_tiles = p.ntiles > (int)blockIdx.x ? (p.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  constexpr int na = ALG2 ? 4 : 2;
 
   if (warp == 0) {
-    // ---------------- producer: raw tiles through the bulk-copy engine ---------------------------
+    // ---------------- producer: resident operands (bulk), input tiles (TMA) ----------------------
     if (lane == 0) {
-      const uint8_t* xb = (const uint8_t*)p.x;
+      mbar_arrive_expect_tx(&bar[A_FULL], na * p.img_bytes);
+      for (int m = 0; m < na; ++m) bulk_g2s(smem + Lo.off_a[m], p.img[m], p.img_bytes, &bar[A_FULL]);
+      const int nbox = F32 ? (d + 31) / 32 : KP / 64;
+      const uint32_t box_bytes = NV * 128;
       for (int k = 0; k < my_tiles; ++k) {
         const int s = k & 1;
-        const int64_t t = blockIdx.x + (int64_t)k * gridDim.x;
-        if (!mbar_wait(&bar[RAW_EMPTY + s], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        const int64_t v0 = t * NV;
-        const int rows = (int)min((int64_t)NV, p.n - v0);
-        const uint32_t bytes = (uint32_t)rows * d * ES;
-        mbar_arrive_expect_tx(&bar[RAW_FULL + s], bytes);
-        bulk_g2s(smem + Lo.off_raw[s], xb + v0 * d * ES, bytes, &bar[RAW_FULL + s]);
+        const int t = blockIdx.x + k * gridDim.x;
+        if (!mbar_wait(&bar[STAGE_EMPTY + s], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        mbar_arrive_expect_tx(&bar[RAW_FULL + s], nbox * box_bytes);
+        for (int b = 0; b < nbox; ++b)
+          tma_load_2d(smem + raw_off(s) + b * box_bytes, &tmap, b * (F32 ? 32 : 64), t * NV, &bar[RAW_FULL + s]);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ---------------------------------------------------------------
-    if (lane == 0) {
+    if (lane == 0 && mbar_wait(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
-      const uint32_t bx0 = smem_u32(smem + Lo.off_bx[0]), bx1 = SPLITX ? smem_u32(smem + Lo.off_bx[1]) : 0u;
       const uint32_t r0 = ALG2 ? smem_u32(smem + Lo.off_rho[0]) : 0u, r1 = ALG2 ? smem_u32(smem + Lo.off_rho[1]) : 0u;
       const int ksteps = KP / 16;
       auto issue_T = [&](int j) -> bool {
@@ -215,112 +247,140 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_con
       };
       bool ok = true;
       for (int k = 0; k < my_tiles && ok; ++k) {
-        const int a = k & 1;
+        const int a = k & 1, s = k & 1;
         if (!mbar_wait(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        if (!mbar_wait(&bar[BX_FULL], k & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait(&bar[STAGE_READY + s], (k >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
         tc_fence_after();
+        const uint32_t bh = smem_u32(smem + (F32 ? bxh_off(s) : raw_off(s)));
+        const uint32_t bl = F32 ? smem_u32(smem + bxh_off(s) + bx_lo) : 0u;
         const uint32_t dhi = tbase + a * COLS, dlo = dhi + NV;
         for (int ks = 0; ks < ksteps; ++ks) {
           const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
           const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
-          const uint64_t db = desc_kmajor_sw128(bx0 + bo);
+          const uint64_t db = desc_kmajor_sw128(bh + bo);
           mma_f16_ss(dhi, desc_kmajor_sw128(a0 + ao), db, idesc, ks > 0);
           mma_f16_ss(dlo, desc_kmajor_sw128(a1 + ao), db, idesc, ks > 0);
-          if (SPLITX) mma_f16_ss(dlo, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bx1 + bo), idesc, 1);
+          if (F32) mma_f16_ss(dlo, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bl + bo), idesc, 1);
         }
-        mma_commit(&bar[BX_EMPTY]);
+        mma_commit(&bar[STAGE_EMPTY + s]);
         mma_commit(&bar[ACC_FULL + a]);
         if (ALG2 && k >= 1) ok = issue_T(k - 1);
       }
       if (ALG2 && ok && my_tiles >= 1 && !*abort_flag) issue_T(my_tiles - 1);
     }
   } else if (warp < 6) {
-    // ---------------- converters: norm, power-of-two scale, fp16 B operand ----------------------
-    const int cw = warp - 2;
-    const int EPL = d / 32;
+    // ---------------- converters: one thread per vector (TPV threads when NV < 128) -------------
+    const int ct = tid - 64;
+    const int v = ct / TPV, part = ct % TPV;
     for (int k = 0; k < my_tiles; ++k) {
-      const int s = k & 1, a = k & 1;
-      const int64_t t = blockIdx.x + (int64_t)k * gridDim.x;
-      const int64_t v0 = t * NV;
-      const int rows = (int)min((int64_t)NV, p.n - v0);
-      if (!mbar_wait(&bar[RAW_FULL + s], (k >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
-      if (!mbar_wait(&bar[BX_EMPTY], (k & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      if (!mbar_wait(&bar[INFO_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      uint8_t* bx = smem + Lo.off_bx[0];
-      uint8_t* bxl = smem + Lo.off_bx[SPLITX ? 1 : 0];
-      const uint8_t* raw = smem + Lo.off_raw[s];
-      for (int v = cw; v < NV; v += 4) {
-        if (v < rows) {
-          const uint8_t* row = raw + (size_t)v * d * ES;
-          float xv[4];
-          double ss = 0.0;       // fp64: squares of any bf16 / fp32 value neither overflow nor underflow
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            xv[e] = 0.0f;
-            if (e < EPL) {
-              xv[e] = load_x(row, lane * EPL + e, ES);
-              ss = fma((double)xv[e], (double)xv[e], ss);
-            }
-          }
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const double nrm = sqrt(ss);
-          double scale = 1.0;
-          float inv = 0.0f;
-          if (nrm > 0.0) {
-            int E;
-            frexp(nrm, &E);
-            scale = ldexp(1.0, 15 - E);            // |x| * scale in [2^14, 2^15)
-            inv = (float)(1.0 / (nrm * scale));
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (e < EPL) {
-              const int kk = lane * EPL + e;
-              const float xs = (float)((double)xv[e] * scale);
-              const __half h = __float2half_rn(xs);
-              *(__half*)(bx + sw128_offset(v, 2 * kk, NV)) = h;
-              if (SPLITX) {
-                const __half l = __float2half_rn((xs - __half2float(h)) * kSplitScale);
-                *(__half*)(bxl + sw128_offset(v, 2 * kk, NV)) = l;
-              }
-            }
-          }
-          if (lane == 0) {
-            info[a * NV + v] = inv;
-            p.norms[v0 + v] = __half_as_ushort(__double2half(nrm));
-          }
-        } else {
-          for (int kk = lane; kk < d; kk += 32) {
-            *(__half*)(bx + sw128_offset(v, 2 * kk, NV)) = __float2half_rn(0.0f);
-            if (SPLITX) *(__half*)(bxl + sw128_offset(v, 2 * kk, NV)) = __float2half_rn(0.0f);
-          }
-          if (lane == 0) info[a * NV + v] = 0.0f;
+      const int s = k & 1;
+      const int64_t v0 = (int64_t)(blockIdx.x + k * gridDim.x) * NV;
+      if (!mbar_wait_warp(&bar[RAW_FULL + s], (k >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[INFO_EMPTY + s], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      uint8_t* raw = smem + raw_off(s);
+      double ss = 0.0;
+      if (!F32) {
+        const int cpp = (KP / 8) / TPV;   // 16-byte chunks (8 values) per thread
+        for (int c = part * cpp; c < (part + 1) * cpp; ++c) {
+          const uint4 w = *(const uint4*)(raw + sw128_offset(v, c * 16, NV));
+          auto acc = [&](uint32_t u) {
+            const double lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xFFFF0000u);
+            ss = fma(lo, lo, ss);
+            ss = fma(hi, hi, ss);
+          };
+          acc(w.x);
+          acc(w.y);
+          acc(w.z);
+          acc(w.w);
         }
-        for (int kk = d + lane; kk < KP; kk += 32) {   // K padding
-          *(__half*)(bx + sw128_offset(v, 2 * kk, NV)) = __float2half_rn(0.0f);
-          if (SPLITX) *(__half*)(bxl + sw128_offset(v, 2 * kk, NV)) = __float2half_rn(0.0f);
+      } else {
+        const int nch = (d + 3) / 4;            // 16-byte chunks of 4 floats actually holding data
+        const int cpp = (nch + TPV - 1) / TPV;
+        for (int c = part * cpp; c < min(nch, (part + 1) * cpp); ++c) {
+          const float4 f = *(const float4*)(raw + sw128_offset(v, c * 16, NV));
+          ss = fma((double)f.x, (double)f.x, ss);
+          ss = fma((double)f.y, (double)f.y, ss);
+          ss = fma((double)f.z, (double)f.z, ss);
+          ss = fma((double)f.w, (double)f.w, ss);
         }
       }
+#pragma unroll
+      for (int o = 1; o < TPV; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const double nrm = sqrt(ss);
+      float f1 = 1.0f, f2 = 1.0f, inv = 0.0f;
+      if (nrm > 0.0) {
+        int E;
+        frexp(nrm, &E);
+        pow2_pair(15 - E, f1, f2);                         // |x| * f1 * f2 in [2^14, 2^15)
+        inv = (float)(1.0 / ldexp(nrm, 15 - E));
+      }
+      if (!F32) {
+        const int cpp = (KP / 8) / TPV;
+        for (int c = part * cpp; c < (part + 1) * cpp; ++c) {
+          uint4* ptr = (uint4*)(raw + sw128_offset(v, c * 16, NV));
+          const uint4 w = *ptr;
+          auto cvt = [&](uint32_t u) -> uint32_t {
+            const __half2 hh = __floats2half2_rn(__uint_as_float(u << 16) * f1 * f2,
+                                                 __uint_as_float(u & 0xFFFF0000u) * f1 * f2);
+            return h2_bits(hh);
+          };
+          *ptr = make_uint4(cvt(w.x), cvt(w.y), cvt(w.z), cvt(w.w));
+        }
+      } else {
+        uint8_t* bxh = smem + bxh_off(s);
+        uint8_t* bxl = bxh + bx_lo;
+        const int nout = KP / 8;                 // 16-byte fp16 chunks of the operand row
+        const int cpp = nout / TPV;
+        for (int c = part * cpp; c < (part + 1) * cpp; ++c) {
+          uint4 wh = make_uint4(0, 0, 0, 0), wl = wh;
+          if (c * 8 < d) {
+            const float4 fa = *(const float4*)(raw + sw128_offset(v, (2 * c) * 16, NV));
+            const float4 fb = *(const float4*)(raw + sw128_offset(v, (2 * c + 1) * 16, NV));
+            // hi = fp16(x s), lo = fp16((x s - hi) 2^12) for a pair of values
+            auto split = [&](float a, float b, uint32_t& h, uint32_t& l) {
+              const float x0 = a * f1 * f2, x1 = b * f1 * f2;
+              const __half2 hh = __floats2half2_rn(x0, x1);
+              const float2 back = __half22float2(hh);
+              h = h2_bits(hh);
+              l = h2_bits(__floats2half2_rn((x0 - back.x) * kSplitScale, (x1 - back.y) * kSplitScale));
+            };
+            split(fa.x, fa.y, wh.x, wl.x);
+            split(fa.z, fa.w, wh.y, wl.y);
+            split(fb.x, fb.y, wh.z, wl.z);
+            split(fb.z, fb.w, wh.w, wl.w);
+          }
+          *(uint4*)(bxh + sw128_offset(v, c * 16, NV)) = wh;
+          *(uint4*)(bxl + sw128_offset(v, c * 16, NV)) = wl;
+        }
+      }
+      if (part == 0) {
+        info[s * NV + v] = inv;
+        if (v0 + v < p.n) p.norms[v0 + v] = __half_as_ushort(__double2half(nrm));
+      }
       fence_proxy_async_smem();
-      mbar_arrive(&bar[RAW_EMPTY + s]);
-      mbar_arrive(&bar[BX_FULL]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[STAGE_READY + s]);
     }
   } else {
     // ---------------- epilogue: quantise, ballot-pack, residual, signs -------------------------
-    const int q = warp & 3;             // TMEM lane quarter = packing group
-    const int i = q * 32 + lane;        // coordinate
+    const int e = warp - 6;                 // 0..7
+    const int q = warp & 3;                 // TMEM lane quarter = packing group
+    const int i = q * 32 + lane;            // coordinate
     const bool active = i < d;
-    const int te = tid - 6 * 32;        // 0..127
+    const int te = tid - 6 * 32;            // 0..255
+    const int cbeg = (e >> 2) * (NV / 2), cend = cbeg + NV / 2;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    float thr[15];
+    float P[8], C[8];
 #pragma unroll
-    for (int kq = 0; kq < 15; ++kq) thr[kq] = p.thr[kq];
-    const int nthr = p.L - 1;
+    for (int kq = 0; kq < 8; ++kq) {
+      P[kq] = p.P[kq];
+      C[kq] = p.C[kq];
+    }
     uint32_t epi_uses = 0;
     auto epi_sync = [&]() -> bool {
-      mbar_arrive(&bar[EPI]);
-      bool ok = mbar_wait(&bar[EPI], epi_uses & 1, p.err, kDevTimeoutSync, abort_flag);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[EPI]);
+      bool ok = mbar_wait_warp(&bar[EPI], epi_uses & 1, p.err, kDevTimeoutSync, abort_flag);
       ++epi_uses;
       return ok;
     };
@@ -328,39 +388,37 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_con
     uint8_t* rho_lo = ALG2 ? smem + Lo.off_rho[1] : nullptr;
     for (int k = 0; k < my_tiles; ++k) {
       const int a = k & 1;
-      const int64_t t = blockIdx.x + (int64_t)k * gridDim.x;
-      const int64_t v0 = t * NV;
+      const int64_t v0 = (int64_t)(blockIdx.x + k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
-      if (!mbar_wait(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
       const uint32_t dhi = tbase + lane_base + a * COLS, dlo = dhi + NV;
-      for (int c0 = 0; c0 < NV; c0 += 32) {
-        uint32_t hi[32], lo[32];
-        tmem_ld16(dhi + c0, *(uint32_t(*)[16]) & hi[0]);
-        tmem_ld16(dhi + c0 + 16, *(uint32_t(*)[16]) & hi[16]);
-        tmem_ld16(dlo + c0, *(uint32_t(*)[16]) & lo[0]);
-        tmem_ld16(dlo + c0 + 16, *(uint32_t(*)[16]) & lo[16]);
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
+        uint32_t hi[16], lo[16];
+        tmem_ld16(dhi + c0, hi);
+        tmem_ld16(dlo + c0, lo);
         tmem_ld_wait();
-        uint32_t myw[4] = {0u, 0u, 0u, 0u};
-        float r2[32];
+        uint32_t myw[BITS];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int pl = 0; pl < BITS; ++pl) myw[pl] = 0u;
+        float r2[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
           const int v = c0 + j;
           const float inv = info[a * NV + v];
           const float y = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j])) * inv;
-          int idx = 0;
+          const bool neg = !(y > 0.0f);
+          const int m = sym_m<BITS>(fabsf(y), P);
 #pragma unroll
-          for (int kq = 0; kq < 15; ++kq)
-            if (kq < nthr) idx += (y > thr[kq]) ? 1 : 0;
-#pragma unroll
-          for (int pl = 0; pl < 4; ++pl) {
-            if (pl < bits) {
-              const uint32_t w = __ballot_sync(0xffffffffu, active && ((idx >> pl) & 1));
-              if (lane == j) myw[pl] = w;
-            }
+          for (int pl = 0; pl < BITS; ++pl) {
+            const bool bit = pl == BITS - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
+            const uint32_t w = __ballot_sync(0xffffffffu, active && bit);
+            if (lane == j) myw[pl] = w;
           }
           if (ALG2) {
-            float rho = (active && inv != 0.0f) ? (y - lut[idx]) : 0.0f;
+            const float cm = sym_c<BITS>(m, C);
+            float rho = neg ? y + cm : y - cm;
+            if (!active || inv == 0.0f) rho = 0.0f;
             r2[j] = rho * rho;
             const float rs = rho * kRhoScale;
             const __half rh = __float2half_rn(rs);
@@ -372,25 +430,25 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_con
             }
           }
         }
-        if (q < G) {
+        if (q < G && lane < 16) {
 #pragma unroll
-          for (int pl = 0; pl < 4; ++pl)
-            if (pl < bits) codes_stage[((c0 + lane) * G + q) * bits + pl] = myw[pl];
+          for (int pl = 0; pl < BITS; ++pl) codes_stage[((c0 + lane) * G + q) * BITS + pl] = myw[pl];
         }
         if (ALG2) {
-          const float tot = transpose_reduce32(r2, lane);
-          gpart[q * NV + c0 + lane] = tot;
+          const float tot = transpose_reduce16(r2, lane);
+          if (lane < 16) gpart[q * NV + c0 + lane] = tot;
         }
       }
       if (ALG2) {
         fence_proxy_async_smem();
-        mbar_arrive(&bar[RHO_FULL]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[RHO_FULL]);
       }
       if (!epi_sync()) break;
       {
-        uint32_t* dst = p.codes + v0 * G * bits;
-        const int nw = rows * G * bits;
-        for (int w = te; w < nw; w += 128) dst[w] = codes_stage[w];
+        uint32_t* dst = p.codes + v0 * G * BITS;
+        const int nw = rows * G * BITS;
+        for (int w = te; w < nw; w += 256) dst[w] = codes_stage[w];
       }
       if (ALG2) {
         if (te < rows) {
@@ -398,33 +456,34 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_con
           for (int qq = 0; qq < G; ++qq) g2 += gpart[qq * NV + te];
           p.gammas[v0 + te] = __half_as_ushort(__float2half_rn(sqrtf(g2)));
         }
-        if (!mbar_wait(&bar[T_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[T_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
         tc_fence_after();
         const uint32_t dT1 = tbase + lane_base + a * COLS + 2 * NV, dT2 = dT1 + NV;
-        for (int c0 = 0; c0 < NV; c0 += 32) {
-          uint32_t s1[32], s2[32];
-          tmem_ld16(dT1 + c0, *(uint32_t(*)[16]) & s1[0]);
-          tmem_ld16(dT1 + c0 + 16, *(uint32_t(*)[16]) & s1[16]);
-          tmem_ld16(dT2 + c0, *(uint32_t(*)[16]) & s2[0]);
-          tmem_ld16(dT2 + c0 + 16, *(uint32_t(*)[16]) & s2[16]);
+        for (int c0 = cbeg; c0 < cend; c0 += 16) {
+          uint32_t s1[16], s2[16];
+          tmem_ld16(dT1 + c0, s1);
+          tmem_ld16(dT2 + c0, s2);
           tmem_ld_wait();
           uint32_t mys = 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const float sv = fmaf(__uint_as_float(s2[j]), kSplitScaleInv, __uint_as_float(s1[j]));
             const uint32_t w = __ballot_sync(0xffffffffu, active && sv >= 0.0f);
             if (lane == j) mys = w;
           }
-          if (q < G) signs_stage[(c0 + lane) * G + q] = mys;
+          if (q < G && lane < 16) signs_stage[(c0 + lane) * G + q] = mys;
         }
         if (!epi_sync()) break;
         uint32_t* dst = p.signs + v0 * G;
         const int nw = rows * G;
-        for (int w = te; w < nw; w += 128) dst[w] = signs_stage[w];
+        for (int w = te; w < nw; w += 256) dst[w] = signs_stage[w];
       }
       tc_fence_before();
-      mbar_arrive(&bar[ACC_EMPTY + a]);
-      mbar_arrive(&bar[INFO_EMPTY + a]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[ACC_EMPTY + a]);
+        mbar_arrive(&bar[INFO_EMPTY + a]);
+      }
       if (!epi_sync()) break;   // stage buffers are reused by the next tile
     }
   }
@@ -437,18 +496,31 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(const __grid_con
   }
 }
 
-template <int XT, bool ALG2, int NV>
-tq_status launch_encode(EncodeParams& p, cudaStream_t st) {
+template <int XT, bool ALG2, int NV, int BITS>
+tq_status launch_encode(EncodeParams& p, const void* x, cudaStream_t st) {
   constexpr int ES = XT == TQ_BF16 ? 2 : 4;
-  const EncLayout Lo = enc_layout<ES, ALG2, XT == TQ_F32>(p.d, p.KP, NV, p.G, p.bits);
-  auto kern = encode_kernel<XT, ALG2, NV>;
+  const EncLayout Lo = enc_layout<XT, ALG2, NV, BITS>(p.d, p.KP, p.G);
+  alignas(64) CUtensorMap tmap;
+  if (!make_tmap_2d_sw128(&tmap, x, ES, (uint64_t)p.d, (uint64_t)p.n, 128 / ES, NV))
+    return fail(TQ_ERR_CUDA, "encode: could not create the TMA tensor map of x");
+  auto kern = encode_kernel<XT, ALG2, NV, BITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "encode: shared memory attribute");
   p.ntiles = (int)((p.n + NV - 1) / NV);
   const int grid = std::min(p.ntiles, sm_count());
-  kern<<<grid, kEncThreads, Lo.total, st>>>(p);
+  kern<<<grid, kEncThreads, Lo.total, st>>>(p, tmap);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "encode: launch");
   return TQ_OK;
+}
+
+template <int XT, bool ALG2, int NV>
+tq_status launch_bits(EncodeParams& p, int bits, const void* x, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_encode<XT, ALG2, NV, 1>(p, x, st);
+    case 2: return launch_encode<XT, ALG2, NV, 2>(p, x, st);
+    case 3: return launch_encode<XT, ALG2, NV, 3>(p, x, st);
+    default: return launch_encode<XT, ALG2, NV, 4>(p, x, st);
+  }
 }
 
 tq_status encode_common(const char* fn, const tq_codebook* cb, int64_t n, int32_t d, const void* x, int32_t xt,
@@ -462,42 +534,46 @@ tq_status encode_common(const char* fn, const tq_codebook* cb, int64_t n, int32_
   if (!valid_dim(d)) return fail(TQ_ERR_UNSUPPORTED, f + ": d must be a multiple of 32 in [32, 4096]");
   if (cb->d != d || cb->bits < 1 || cb->bits > 4 || cb->levels != (1 << cb->bits))
     return fail(TQ_ERR_INVALID_ARG, f + ": codebook does not match d / has bad bits");
+  const int L = cb->levels, H = L / 2;
+  for (int k = 0; k < L; ++k)
+    if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, f + ": codebook is not symmetric");
+  for (int k = 0; k + 1 < L; ++k)
+    if (cb->t[L - 2 - k] != -cb->t[k]) return fail(TQ_ERR_INVALID_ARG, f + ": codebook is not symmetric");
   if (xt != TQ_F32 && xt != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, f + ": x_dtype must be TQ_F32 or TQ_BF16");
   if (!aligned16(x) || !aligned16(rot) || !aligned16(codes) || !aligned16(norms) ||
       (alg2 && (!aligned16(signs) || !aligned16(gammas))))
     return fail(TQ_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
   if (n == 0) return TQ_OK;
   if (d > 128) return fail(TQ_ERR_UNSUPPORTED, f + ": d > 128 is not supported by this build");
+  if (n > ((int64_t)1 << 31) - 256) return fail(TQ_ERR_UNSUPPORTED, f + ": n >= 2^31");
   RotLayout RL = rot_layout(d);
-  const char* base = (const char*)rot;
+  const uint8_t* base = (const uint8_t*)rot;
   EncodeParams p{};
-  p.x = x;
   p.n = n;
   p.d = d;
   p.G = d / 32;
-  p.bits = cb->bits;
-  p.L = cb->levels;
   p.KP = d <= 64 ? 64 : 128;
-  p.pi_hi = (const __half*)(base + RL.pi_hi);
-  p.pi_lo = (const __half*)(base + RL.pi_lo);
-  p.t_hi = (const __half*)(base + RL.t_hi);
-  p.t_lo = (const __half*)(base + RL.t_lo);
-  p.dp = RL.dp;
+  p.img[0] = base + RL.pi_hi;
+  p.img[1] = base + RL.pi_lo;
+  p.img[2] = base + RL.t_hi;
+  p.img[3] = base + RL.t_lo;
+  p.img_bytes = 128u * p.KP * 2;
   p.codes = codes;
   p.signs = signs;
   p.norms = norms;
   p.gammas = gammas;
-  for (int k = 0; k < 16; ++k) {
-    p.cent[k] = k < cb->levels ? cb->c[k] : 0.0f;
-    p.thr[k] = k < cb->levels - 1 ? cb->t[k] : 0.0f;
+  for (int k = 0; k < 8; ++k) {
+    p.P[k] = k < H - 1 ? cb->t[H + k] : 0.0f;
+    p.C[k] = k < H ? cb->c[H + k] : 0.0f;
   }
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, f + ": no device error word (is a CUDA device present?)");
   cudaStream_t st = (cudaStream_t)stream;
-  if (!alg2) {
-    return xt == TQ_BF16 ? launch_encode<TQ_BF16, false, 128>(p, st) : launch_encode<TQ_F32, false, 64>(p, st);
-  }
-  return xt == TQ_BF16 ? launch_encode<TQ_BF16, true, 64>(p, st) : launch_encode<TQ_F32, true, 32>(p, st);
+  if (!alg2)
+    return xt == TQ_BF16 ? launch_bits<TQ_BF16, false, 128>(p, cb->bits, x, st)
+                         : launch_bits<TQ_F32, false, 64>(p, cb->bits, x, st);
+  return xt == TQ_BF16 ? launch_bits<TQ_BF16, true, 64>(p, cb->bits, x, st)
+                       : launch_bits<TQ_F32, true, 32>(p, cb->bits, x, st);
 }
 
 }  // namespace

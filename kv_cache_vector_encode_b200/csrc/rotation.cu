@@ -9,6 +9,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "sm100.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -58,7 +59,9 @@ __global__ void t_matrix_kernel(const float* __restrict__ S, const float* __rest
   if (i < d && j < d) T[(size_t)i * d + j] = (float)acc;
 }
 
-// hi/lo fp16 split of M (or of M^T when transpose), zero padded to dp x dp.
+// hi/lo fp16 split of M (or of M^T when transpose), zero padded to dp x dp, written as the
+// shared-memory image the tensor-core kernels use (see RotLayout): element (r, c) goes to
+//   (r / 128) * (128 * dp * 2) + sw128_offset(r % 128, 2 c, 128)   bytes.
 __global__ void split_kernel(const float* __restrict__ M, int d, int dp, bool transpose, __half* __restrict__ hi,
                              __half* __restrict__ lo) {
   size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -68,8 +71,9 @@ __global__ void split_kernel(const float* __restrict__ M, int d, int dp, bool tr
   if (r < d && c < d) v = transpose ? M[(size_t)c * d + r] : M[(size_t)r * d + c];
   __half h = __float2half_rn(v);
   __half l = __float2half_rn((v - __half2float(h)) * kSplitScale);
-  hi[idx] = h;
-  lo[idx] = l;
+  size_t off = (size_t)(r >> 7) * (128u * dp * 2) + sw128_offset(r & 127, 2 * c, 128);
+  hi[off / 2] = h;
+  lo[off / 2] = l;
 }
 
 __global__ void header_kernel(int* hdr, int d) {

@@ -18,9 +18,13 @@ tq_status cuda_fail(int err, const char* what);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- prepared-rotation buffer layout -------------------------------------------------------------
-// All regions 256-byte aligned. fp32 matrices row-major d x d; fp16 matrices row-major, padded to
-// Dp x Dp (Dp = d rounded up to a multiple of 128) with zeros so tensor-core tiles never read past
-// a region.
+// All regions 256-byte aligned. fp32 matrices row-major d x d. fp16 matrices are padded with zeros
+// to Dp x Dp (Dp = d rounded up to a multiple of 128) and stored as shared-memory images of the
+// tensor-core operand layout (K-major, 128-byte swizzle): 128-row bands of rows, each band laid out
+// as Dp/64 column blocks of [128 rows x 128 bytes]; element (r, c) sits at byte
+//   (r / 128) * (128 * Dp * 2) + blk * 16384 + (r % 128 / 8) * 1024 + (r % 8) * 128
+//     + (((2c % 128) / 16) ^ (r % 8)) * 16 + 2c % 16,     blk = 2c / 128.
+// A kernel therefore loads any (band, column-block) piece with one bulk copy.
 //   Pi32, S32, T32 = S Pi^T
 //   Pi_hi, Pi_lo   : fp16 split of Pi       (Pi  = Pi_hi + 2^-12 Pi_lo)
 //   T_hi,  T_lo    : fp16 split of T
@@ -44,5 +48,10 @@ uint32_t* device_error_word();
 
 // Number of SMs of the current device.
 int sm_count();
+
+// 2-D TMA tensor map (128-byte swizzle, zero fill out of range) for a row-major [rows][cols]
+// matrix of esize-byte elements; `tmap` points at a 64-byte-aligned 128-byte CUtensorMap.
+bool make_tmap_2d_sw128(void* tmap, const void* base, int esize, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                        uint32_t box_rows);
 
 }  // namespace tq
