@@ -85,29 +85,51 @@ __host__ __device__ inline int att_rec(int d) { return 4 + 2 * d; }
 __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   const int slice = blockIdx.x;                  // = b * Hkv + hk
   const int b = slice / p.Hkv, hk = slice % p.Hkv;
-  const int d = p.d, i = threadIdx.x;            // coordinate
-  __shared__ float sq[128];
+  const int d = p.d, i = threadIdx.x;            // coordinate (128 threads)
+  const int warp = i >> 5, lane = i & 31;
+  __shared__ float sq[8][128];
+  __shared__ double qr[8][128];
   __shared__ double red[128];
   const int kbytes = p.mk * d;
   uint8_t* img = p.bq_img + (size_t)slice * p.nq * kbytes;
-  // zero the image (padding rows stay zero)
   for (int o = i; o < p.nq * kbytes / 16; o += blockDim.x) ((uint4*)img)[o] = make_uint4(0, 0, 0, 0);
   for (int h = 0; h < p.Hg; ++h) {
-    const int hq = hk * p.Hg + h;
-    const size_t qoff = ((size_t)b * p.Hq + hq) * d;
-    __syncthreads();
-    if (i < d) {
-      sq[i] = p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
-                       : ((const float*)p.q)[qoff + i];
+    const size_t qoff = ((size_t)b * p.Hq + hk * p.Hg + h) * d;
+    sq[h][i] = p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
+                        : ((const float*)p.q)[qoff + i];
+  }
+  __syncthreads();
+  // q'_h = Pi q_h: one warp per output coordinate, lanes across the row of Pi (coalesced)
+  for (int r = warp; r < d; r += 4) {
+    const float* row = p.Pi + (size_t)r * d;
+    double acc[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) acc[h] = 0.0;
+    for (int j = lane; j < d; j += 32) {
+      const double pij = (double)row[j];
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < p.Hg) acc[h] = fma(pij, (double)sq[h][j], acc[h]);
     }
-    __syncthreads();
-    double acc = 0.0;
-    if (i < d)
-      for (int j = 0; j < d; ++j) acc += (double)p.Pi[(size_t)i * d + j] * (double)sq[j];
-    // Q_h and max_S |beta_S q'_i|
-    double bmax = 0.0;
-    for (int s = 0; s < p.mk; ++s) bmax = fmax(bmax, fabs((double)p.beta_k[s]));
-    red[i] = i < d ? acc : 0.0;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < p.Hg) {
+        double v = acc[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) qr[h][r] = v;
+      }
+    }
+  }
+  __syncthreads();
+  double bmax = 0.0, sb = 0.0;
+  for (int S = 0; S < p.mk; ++S) {
+    bmax = fmax(bmax, fabs((double)p.beta_k[S]));
+    sb += (double)p.beta_k[S];
+  }
+  for (int h = 0; h < p.Hg; ++h) {
+    const double qi = qr[h][i];
+    red[i] = qi;
     __syncthreads();
     for (int o = 64; o > 0; o >>= 1) {
       if (i < o) red[i] += red[i + o];
@@ -115,7 +137,7 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
     }
     const double Qh = red[0];
     __syncthreads();
-    red[i] = i < d ? fabs(acc) * bmax : 0.0;
+    red[i] = fabs(qi) * bmax;
     __syncthreads();
     for (int o = 64; o > 0; o >>= 1) {
       if (i < o) red[i] = fmax(red[i], red[i + o]);
@@ -130,23 +152,18 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
       F = 30 - E;                   // vmax * 2^F < 2^30
     }
     if (i == 0) {
-      double sb = 0.0;
-      for (int s = 0; s < p.mk; ++s) sb += (double)p.beta_k[s];
       p.head_c[(slice * 8 + h) * 2 + 0] = (float)ldexp(1.0, -F);
       p.head_c[(slice * 8 + h) * 2 + 1] = (float)(Qh * sb);
     }
-    if (i < d) {
-      const int g = i >> 5, r = i & 31, jj = r >> 3, s = r & 7;   // coordinate 32g + 8jj + s
-      const int kin = 32 * g + 4 * s + jj;                       // its k index inside a plane
-      for (int S = 0; S < p.mk; ++S) {
-        long long v = llrint(ldexp((double)p.beta_k[S] * acc, F - s));
-        const int k = S * d + kin;
-        for (int l = 0; l < 4; ++l) {
-          long long dl = l < 3 ? (((v + 128) & 255) - 128) : v;   // balanced signed digits
-          v = (v - dl) >> 8;
-          const int row = h * 4 + l;
-          img[sw128_offset(row, k, p.nq)] = (uint8_t)(int8_t)dl;
-        }
+    const int g = i >> 5, rr = i & 31, jj = rr >> 3, s = rr & 7;   // coordinate 32g + 8jj + s
+    const int kin = 32 * g + 4 * s + jj;                          // its k index inside a plane
+    for (int S = 0; S < p.mk; ++S) {
+      long long v = llrint(ldexp((double)p.beta_k[S] * qi, F - s));
+      const int k = S * d + kin;
+      for (int l = 0; l < 4; ++l) {
+        const long long dl = l < 3 ? (((v + 128) & 255) - 128) : v;   // balanced signed digits
+        v = (v - dl) >> 8;
+        img[sw128_offset(h * 4 + l, k, p.nq)] = (uint8_t)(int8_t)dl;
       }
     }
   }
@@ -214,6 +231,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(const AttParams& p, int gchunk) {
   return r;
 }
 
+template <int HG>
 __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __grid_constant__ AttParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -373,20 +391,41 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       tc_fence_after();
       const ChunkPos cp = chunk_pos(p, c_begin + c);
       const int tc = (int)min((int64_t)kChunk, T - (int64_t)cp.cis * kChunk);
-      const uint32_t* kw = (const uint32_t*)(smem + Lo.off_stage + st * Lo.stage_bytes) + t * G * p.bk;
       const bool live = t < tc;
-      const uint32_t ak = tbase + lane_base + kAK0 + b * 128;
-      for (int g = 0; g < G; ++g) {
-        uint32_t pw[4] = {0u, 0u, 0u, 0u};
-        for (int pl = 0; pl < p.bk; ++pl) pw[pl] = live ? kw[g * p.bk + pl] : 0u;
-        for (int S = 0; S < p.mk; ++S) {
-          const int m = p.kmask[S];
-          const uint32_t w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u) ^ ((m & 4) ? pw[2] : 0u) ^
-                             ((m & 8) ? pw[3] : 0u);
-          uint32_t r[8];
+      // the token's G * bk plane words (<= 16, contiguous, 16-byte aligned)
+      const uint4* kw4 = (const uint4*)((const uint32_t*)(smem + Lo.off_stage + st * Lo.stage_bytes) + t * 4 * p.bk);
+      uint32_t kw[16];
 #pragma unroll
-          for (int s = 0; s < 8; ++s) r[s] = w & (0x01010101u << s);
-          tmem_st8(ak + S * (d / 4) + g * 8, r);
+      for (int v4 = 0; v4 < 4; ++v4) {
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (v4 < p.bk && live) x = kw4[v4];
+        kw[4 * v4] = x.x;
+        kw[4 * v4 + 1] = x.y;
+        kw[4 * v4 + 2] = x.z;
+        kw[4 * v4 + 3] = x.w;
+      }
+      const uint32_t ak = tbase + lane_base + kAK0 + b * 128;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t pw[4];
+#pragma unroll
+        for (int pl = 0; pl < 4; ++pl) {
+          // word (g, pl) of a bk-plane record sits at g * bk + pl; bk is 1..3 (selects keep kw in registers)
+          const uint32_t w3 = pl < 3 ? kw[3 * g + (pl < 3 ? pl : 0)] : 0u;
+          const uint32_t w2 = pl < 2 ? kw[2 * g + (pl < 2 ? pl : 0)] : 0u;
+          const uint32_t w1 = pl < 1 ? kw[g] : 0u;
+          pw[pl] = p.bk == 3 ? w3 : (p.bk == 2 ? w2 : w1);
+        }
+#pragma unroll
+        for (int S = 0; S < 4; ++S) {
+          if (S < p.mk) {
+            const int m = p.kmask[S];
+            const uint32_t w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u) ^ ((m & 4) ? pw[2] : 0u);
+            uint32_t r[8];
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) r[s8] = w & (0x01010101u << s8);
+            tmem_st8(ak + S * 32 + g * 8, r);
+          }
         }
       }
       tmem_st_wait();
@@ -398,7 +437,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       }
       return true;
     };
-    float m2run[8], lrun[8];   // running max (log2 domain) and softmax sum (kept by every thread)
+    float m2run[HG];   // running max (log2 domain), kept by every thread
     bool ok = nmy > 0 ? expand_k(0) : true;
     for (int c = 0; c < nmy && ok; ++c) {
       const int b = c & 1;
@@ -408,39 +447,45 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       const bool live = t < tc;
       if (seg_first(c)) {
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          m2run[h] = -INFINITY;
-          lrun[h] = 0.0f;
-        }
+        for (int h = 0; h < HG; ++h) m2run[h] = -INFINITY;
       }
-      // per-token inputs (plain loads, issued before the wait)
+      // per-token inputs (plain loads, issued before the waits)
       const int64_t rec = (int64_t)cp.slice * T + t0 + t;
       const float nk = live ? __half2float(__ushort_as_half(__ldg(p.k_norms + rec))) : 0.0f;
       const float nv = live ? __half2float(__ushort_as_half(__ldg(p.v_norms + rec))) : 0.0f;
       const float gm = (live && p.vsign) ? __half2float(__ushort_as_half(__ldg(p.v_gammas + rec))) : 0.0f;
+      const float4* hc4 = (const float4*)(p.head_c + cp.slice * 16);
+      float hcf[2 * HG];
+#pragma unroll
+      for (int h2 = 0; h2 < HG / 2; ++h2) {
+        const float4 x = __ldg(hc4 + h2);
+        hcf[4 * h2] = x.x;
+        hcf[4 * h2 + 1] = x.y;
+        hcf[4 * h2 + 2] = x.z;
+        hcf[4 * h2 + 3] = x.w;
+      }
       if (c + 1 < nmy && !expand_k(c + 1)) break;
       if (!mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
-      uint32_t dsr[32];
+      uint32_t dsr[4 * HG];
       tmem_ld16(tbase + lane_base + kDS0 + b * 32, *(uint32_t(*)[16]) & dsr[0]);
-      if (p.nq > 16) tmem_ld16(tbase + lane_base + kDS0 + b * 32 + 16, *(uint32_t(*)[16]) & dsr[16]);
+      if (HG > 4) tmem_ld16(tbase + lane_base + kDS0 + b * 32 + 16, *(uint32_t(*)[16]) & dsr[HG > 4 ? 16 : 0]);
       tmem_ld_wait();
-      float lg[8];
-      const float* hc = p.head_c + cp.slice * 16;
+      float lg[HG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
         lg[h] = -INFINITY;
         if (h < Hg && live) {
           const long long dot = (long long)(int)dsr[4 * h] + ((long long)(int)dsr[4 * h + 1] << 8) +
                                 ((long long)(int)dsr[4 * h + 2] << 16) + ((long long)(int)dsr[4 * h + 3] << 24);
-          const float score = nk * fmaf(-2.0f * __ldg(hc + 2 * h), (float)dot, __ldg(hc + 2 * h + 1));
+          const float score = nk * fmaf(-2.0f * hcf[2 * h], (float)dot, hcf[2 * h + 1]);
           lg[h] = score * p.scale_log2e;
         }
       }
-      // chunk max per head, across the 128 tokens
-      float mx[8];
+      // chunk max per head, across the 128 tokens; max |v| (and |v| gamma) for the fixed point
+      float mx[HG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
         float v = lg[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -455,14 +500,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       float* rb = red + (c & 1) * 128;
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < 8; ++h) rb[q * 32 + h] = mx[h];
+        for (int h = 0; h < HG; ++h) rb[q * 32 + h] = mx[h];
         rb[q * 32 + 8] = vmx;
         rb[q * 32 + 9] = gmx;
       }
       if (!tok_sync()) break;
-      float m2new[8], corr[8];
+      float m2new[HG], corr[HG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
         const float cm = fmaxf(fmaxf(rb[h], rb[32 + h]), fmaxf(rb[64 + h], rb[96 + h]));
         m2new[h] = fmaxf(m2run[h], cm);
         corr[h] = (m2new[h] == -INFINITY) ? 1.0f : exp2f(m2run[h] - m2new[h]);
@@ -474,10 +519,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       frexpf(fmaxf(U2, 1e-30f), &E2);
       const float sw = ldexpf(1.0f, 32 - E1), sw2 = ldexpf(1.0f, 32 - E2);   // w * sw < 2^32
       // weights, their fixed-point limbs (one 32-bit word per head = its four limbs) and sums
-      uint32_t wv[8], wz[8];
-      float sp[8], sw_[8], sz_[8];
+      uint32_t wv[HG], wz[HG];
+      float sp[HG], sw_[HG], sz_[HG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
         const float pr = (lg[h] == -INFINITY) ? 0.0f : exp2f(lg[h] - m2new[h]);
         const float w = pr * nv, wg = w * gm;
         wv[h] = __float2uint_rn(w * sw);
@@ -490,13 +535,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       if (c >= 2 && !mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       uint8_t* bw = smem + Lo.off_bw + (b * 2 + 0) * Lo.bw_bytes;
       uint8_t* bz = smem + Lo.off_bw + (b * 2 + 1) * Lo.bw_bytes;
-      for (int blk = 0; blk < p.nvc / 16; ++blk) {
+#pragma unroll
+      for (int blk = 0; blk < HG / 4; ++blk) {
         *(uint4*)(bw + blk * kChunk * 16 + t * 16) = make_uint4(wv[4 * blk], wv[4 * blk + 1], wv[4 * blk + 2], wv[4 * blk + 3]);
         *(uint4*)(bz + blk * kChunk * 16 + t * 16) = make_uint4(wz[4 * blk], wz[4 * blk + 1], wz[4 * blk + 2], wz[4 * blk + 3]);
       }
       // chunk sums per head
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           sp[h] += __shfl_xor_sync(0xffffffffu, sp[h], o);
@@ -507,7 +553,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       float* rs = red + 256 + (c & 1) * 128;
       if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
+        for (int h = 0; h < HG; ++h) {
           rs[q * 32 + h] = sp[h];
           rs[q * 32 + 8 + h] = sw_[h];
           rs[q * 32 + 16 + h] = sz_[h];
@@ -517,29 +563,34 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       if (!tok_sync()) break;
       // chunk scalars for the accumulators (4-deep ring)
       float* sc = scal + (c & 3) * 64;
-      if (q == 0 && lane < 8) {
+      if (q == 0 && lane < HG) {
         const int h = lane;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
         for (int w4 = 0; w4 < 4; ++w4) {
           a0 += rs[w4 * 32 + h];
           a1 += rs[w4 * 32 + 8 + h];
           a2 += rs[w4 * 32 + 16 + h];
         }
-        sc[h] = corr[h];            // rescale of the running sums
+        float ch = 1.0f, mh = 0.0f;
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh)
+          if (hh == h) {
+            ch = corr[hh];
+            mh = m2new[hh];
+          }
+        sc[h] = ch;                 // rescale of the running sums
         sc[8 + h] = a0;             // sum of p
         sc[16 + h] = a1;            // sum of w = p * |v|
         sc[24 + h] = a2;            // sum of w' = p * |v| * gamma
-        sc[32 + h] = m2new[h];
+        sc[32 + h] = mh;
         if (h == 0) {
           sc[40] = 1.0f / sw;       // fixed-point scales of the two weight kinds
           sc[41] = 1.0f / sw2;
         }
       }
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        lrun[h] = lrun[h] * corr[h];
-        m2run[h] = m2new[h];
-      }
+      for (int h = 0; h < HG; ++h) m2run[h] = m2new[h];
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[SCAL_FULL + (c & 3)]);
@@ -557,24 +608,46 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       const int tc = (int)min((int64_t)kChunk, T - (int64_t)cp.cis * kChunk);
       const bool live = t < tc;
       const uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
-      const uint32_t* vw = (const uint32_t*)(stg + Lo.kc_bytes) + t * G * p.bv;
-      const uint32_t* sw = (const uint32_t*)(stg + Lo.kc_bytes + kChunk * G * p.bv * 4) + t * G;
-      for (int g = 0; g < G; ++g) {
-        uint32_t pw[4] = {0u, 0u, 0u, 0u};
-        for (int pl = 0; pl < p.bv; ++pl) pw[pl] = live ? vw[g * p.bv + pl] : 0u;
-        for (int P = 0; P < p.np; ++P) {
-          uint32_t w;
-          if (p.vsign && P == p.np - 1) {
-            w = live ? sw[g] : 0u;
-          } else {
-            const int m = p.vmask[P];
-            w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u) ^ ((m & 4) ? pw[2] : 0u) ^ ((m & 8) ? pw[3] : 0u);
+      const uint4* vw4 = (const uint4*)((const uint32_t*)(stg + Lo.kc_bytes) + t * 4 * p.bv);
+      const uint4* sw4 = (const uint4*)((const uint32_t*)(stg + Lo.kc_bytes + kChunk * 16 * p.bv) + t * 4);
+      uint32_t vwr[8];
+#pragma unroll
+      for (int v4 = 0; v4 < 2; ++v4) {
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (v4 < p.bv && live) x = vw4[v4];
+        vwr[4 * v4] = x.x;
+        vwr[4 * v4 + 1] = x.y;
+        vwr[4 * v4 + 2] = x.z;
+        vwr[4 * v4 + 3] = x.w;
+      }
+      uint4 sx = make_uint4(0, 0, 0, 0);
+      if (p.vsign && live) sx = *sw4;
+      const uint32_t swr[4] = {sx.x, sx.y, sx.z, sx.w};
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t pw[2];
+#pragma unroll
+        for (int pl = 0; pl < 2; ++pl) {
+          const uint32_t w2 = vwr[2 * g + pl];
+          const uint32_t w1 = pl < 1 ? vwr[g] : 0u;
+          pw[pl] = p.bv == 2 ? w2 : w1;
+        }
+#pragma unroll
+        for (int P = 0; P < 3; ++P) {
+          if (P < p.np) {
+            uint32_t w;
+            if (p.vsign && P == p.np - 1) {
+              w = swr[g];
+            } else {
+              const int m = p.vmask[P];
+              w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u);
+            }
+            uint8_t* row = smem + Lo.off_av + (b * p.np + P) * Lo.av_bytes;
+            const uint4 lo4 = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
+            const uint4 hi4 = make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
+            *(uint4*)(row + sw128_offset(t, g * 32, 128)) = lo4;
+            *(uint4*)(row + sw128_offset(t, g * 32 + 16, 128)) = hi4;
           }
-          uint8_t* row = smem + Lo.off_av + (b * p.np + P) * Lo.av_bytes;
-          const uint4 lo4 = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
-          const uint4 hi4 = make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
-          *(uint4*)(row + sw128_offset(t, g * 32, 128)) = lo4;
-          *(uint4*)(row + sw128_offset(t, g * 32 + 16, 128)) = hi4;
         }
       }
       fence_proxy_async_smem();
@@ -593,14 +666,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
     const float rowscale = ldexpf(1.0f, -s);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
-    float acc[3][8];                             // [value plane][head]
-    float Wrun[8], Zrun[8], Lrun[8], Mrun[8];
+    float acc[3][HG];                            // [value plane][head]
+    float Wrun[HG], Zrun[HG], Lrun[HG], Mrun[HG];
     for (int c = 0; c < nmy; ++c) {
       const int b = c & 1;
       const ChunkPos cp = chunk_pos(p, c_begin + c);
       if (seg_first(c)) {
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
+        for (int h = 0; h < HG; ++h) {
           acc[0][h] = acc[1][h] = acc[2][h] = 0.0f;
           Wrun[h] = Zrun[h] = Lrun[h] = 0.0f;
           Mrun[h] = -INFINITY;
@@ -610,9 +683,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       if (!mbar_wait_warp(&bar[V_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
       const float* sc = scal + (c & 3) * 64;
-      float corr[8];
+      float corr[HG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < HG; ++h) {
         corr[h] = sc[h];
         Lrun[h] = Lrun[h] * corr[h] + sc[8 + h];
         Wrun[h] = Wrun[h] * corr[h] + sc[16 + h];
@@ -620,23 +693,21 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
         Mrun[h] = sc[32 + h];
       }
       const float fw = sc[40] * rowscale, fz = sc[41] * rowscale;
-      for (int P = 0; P < p.np; ++P) {
-        const bool sgn = p.vsign && P == p.np - 1;
-        uint32_t dv[32];
-        const uint32_t col = tbase + lane_base + kDV0 + (b * p.np + P) * p.nvc;
-        tmem_ld16(col, *(uint32_t(*)[16]) & dv[0]);
-        if (p.nvc > 16) tmem_ld16(col + 16, *(uint32_t(*)[16]) & dv[16]);
-        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          if (h < Hg) {
+      for (int P = 0; P < 3; ++P) {
+        if (P < p.np) {
+          const bool sgn = p.vsign && P == p.np - 1;
+          uint32_t dv[4 * HG];
+          const uint32_t col = tbase + lane_base + kDV0 + (b * p.np + P) * (4 * HG);
+          tmem_ld16(col, *(uint32_t(*)[16]) & dv[0]);
+          if (HG > 4) tmem_ld16(col + 16, *(uint32_t(*)[16]) & dv[HG > 4 ? 16 : 0]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
             const unsigned long long y = (unsigned long long)dv[4 * h] + ((unsigned long long)dv[4 * h + 1] << 8) +
                                          ((unsigned long long)dv[4 * h + 2] << 16) +
                                          ((unsigned long long)dv[4 * h + 3] << 24);
-            const float val = (float)y * (sgn ? fz : fw);
-#pragma unroll
-            for (int pp = 0; pp < 3; ++pp)
-              if (pp == P) acc[pp][h] = fmaf(acc[pp][h], corr[h], val);
+            acc[P][h] = fmaf(acc[P][h], corr[h], (float)y * (sgn ? fz : fw));
           }
         }
       }
@@ -648,25 +719,26 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
         const int sg = cp.slice;
         const int seg = (c_begin + c) / p.per_cta - (sg * p.nchunk) / p.per_cta;   // CTA ordinal inside the slice
         float* rec = p.partial + ((size_t)sg * p.maxseg + seg) * Hg * att_rec(d);
-        for (int h = 0; h < Hg; ++h) {
-          float* rh = rec + h * att_rec(d);
-          float om = 0.0f;
-          for (int P = 0; P < p.mv; ++P)
 #pragma unroll
-            for (int pp = 0; pp < 3; ++pp)
-              if (pp == P) om += p.beta_v[P] * (Wrun[h] - 2.0f * acc[pp][h]);
-          float oz = 0.0f;
-          if (p.vsign)
+        for (int h = 0; h < HG; ++h) {
+          if (h < Hg) {
+            float* rh = rec + h * att_rec(d);
+            float om = 0.0f;
 #pragma unroll
-            for (int pp = 0; pp < 3; ++pp)
-              if (pp == p.np - 1) oz = 2.0f * acc[pp][h] - Zrun[h];
-          rh[4 + coord] = om;
-          rh[4 + d + coord] = oz;
-          if (m == 0) {
-            rh[0] = Mrun[h];
-            rh[1] = Lrun[h];
-            rh[2] = 1.0f;                       // marks a written record
-            rh[3] = 0.0f;
+            for (int P = 0; P < 3; ++P)
+              if (P < p.mv) om += p.beta_v[P] * (Wrun[h] - 2.0f * acc[P][h]);
+            float oz = 0.0f;
+#pragma unroll
+            for (int P = 0; P < 3; ++P)
+              if (p.vsign && P == p.np - 1) oz = 2.0f * acc[P][h] - Zrun[h];
+            rh[4 + coord] = om;
+            rh[4 + d + coord] = oz;
+            if (m == 0) {
+              rh[0] = Mrun[h];
+              rh[1] = Lrun[h];
+              rh[2] = 1.0f;                       // marks a written record
+              rh[3] = 0.0f;
+            }
           }
         }
       }
@@ -774,7 +846,7 @@ bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl) {
   const int ncta = (int)std::min<long long>(nsm, totalc);
   p.per_cta = (int)((totalc + ncta - 1) / ncta);
   p.maxseg = (p.nchunk + p.per_cta - 1) / p.per_cta + 1;
-  p.nq = ((p.Hg * 4 + 15) / 16) * 16;
+  p.nq = p.Hg <= 4 ? 16 : 32;      // the kernel is built for 4 or 8 heads per KV head
   p.nvc = p.nq;
   pl.bq_bytes = (size_t)p.slices * p.nq * 4 * d;       // mk <= 4
   pl.hc_bytes = (size_t)p.slices * 16 * sizeof(float);
@@ -873,11 +945,12 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   cudaError_t e;
   attend_prep_kernel<<<p.slices, 128, 0, st>>>(p);
   const AttLayout Lo = att_layout(p);
-  e = cudaFuncSetAttribute(attend_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
+  auto kern = p.Hg <= 4 ? attend_main_kernel<4> : attend_main_kernel<8>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode: shared memory attribute");
   const long long totalc = (long long)p.slices * p.nchunk;
   const int grid = (int)((totalc + p.per_cta - 1) / p.per_cta);
-  attend_main_kernel<<<grid, kAttThreads, Lo.total, st>>>(p);
+  kern<<<grid, kAttThreads, Lo.total, st>>>(p);
   attend_combine_kernel<<<B * Hq, 128, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tq_attend_decode: launch");
   return TQ_OK;
