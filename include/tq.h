@@ -182,6 +182,27 @@ TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb
                            const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
                            float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed scratch array behind tq_attend_decode_noalloc (8 MiB per device). It covers,
+ * for example, B = 16, Hkv = 8, Hq = 32, T = 131072 (about 2.7 MB). */
+#define TQ_ATTEND_NOALLOC_MAX_BYTES (8u << 20)
+
+/* tq_attend_decode without a caller workspace: the same computation, arguments, layouts and
+ * limits, but the scratch is a fixed array of TQ_ATTEND_NOALLOC_MAX_BYTES bytes that the library
+ * holds in device memory (one per device). No counterpart in the TurboQuant write-ups: it exists
+ * for callers that cannot allocate device memory -- a plain C host holding only the cache
+ * pointers, a runtime whose memory pool already owns all of HBM, a latency-critical stream that
+ * must not meet cudaFree's device-wide wait. The call allocates and frees nothing.
+ * Errors: TQ_ERR_WORKSPACE when tq_attend_workspace_bytes(B, Hq, Hkv, T, d) exceeds the array
+ * (nothing is enqueued); otherwise those of tq_attend_decode. Every call on a device shares that
+ * device's array: calls whose GPU work overlaps (different streams, different host threads) race
+ * and give wrong results, so order them (one stream, or events). Nothing in the array needs to be
+ * zero beforehand; no state carries from one call to the next. */
+TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                   int32_t Hkv, int64_t T, int32_t d, const void* q, int32_t q_dtype,
+                                   const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
+                                   const uint32_t* v_codes, const uint32_t* v_signs, const uint16_t* v_norms,
+                                   const uint16_t* v_gammas, float scale, float* out, void* stream);
+
 /* Synchronises `stream`, then reports a pending CUDA error (TQ_ERR_CUDA) or a device-side
  * timeout recorded by any libtq kernel since the last check (TQ_ERR_DEVICE_TIMEOUT, which this
  * call clears). TQ_OK otherwise. */

@@ -71,6 +71,8 @@ _SIGNATURES = {
     "tq_attend_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
     "tq_attend_decode": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P,
                                 _F, _P, _P, _SZ, _P]),
+    "tq_attend_decode_noalloc": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
+                                        _P, _F, _P, _P]),
     "tq_sync_check": (_I32, [_P]),
 }
 
@@ -223,6 +225,29 @@ def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v
                                   _ptr(v_norms, "v_norms", [torch.float16]),
                                   _ptr(v_gammas, "v_gammas", [torch.float16], True), float(scale),
                                   _ptr(out, "out", [torch.float32]), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
+                             v_signs=None, v_gammas=None, scale=None, stream=None):
+    """tq_attend_decode with the library's fixed scratch array (no workspace, no allocation)."""
+    import math
+    import torch
+    B, Hq, d = q.shape
+    Hkv, T = k_norms.shape[1], k_norms.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib().tq_attend_decode_noalloc(ctypes.byref(cb_k), ctypes.byref(cb_v), B, Hq, Hkv, T, d,
+                                          _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q), _ptr(rot, "rot"),
+                                          _ptr(k_codes, "k_codes", [torch.int32]),
+                                          _ptr(k_norms, "k_norms", [torch.float16]),
+                                          _ptr(v_codes, "v_codes", [torch.int32]),
+                                          _ptr(v_signs, "v_signs", [torch.int32], True),
+                                          _ptr(v_norms, "v_norms", [torch.float16]),
+                                          _ptr(v_gammas, "v_gammas", [torch.float16], True), float(scale),
+                                          _ptr(out, "out", [torch.float32]), _stream(stream)))
+
+
+TQ_ATTEND_NOALLOC_MAX_BYTES = 8 << 20
 
 
 def tq_sync_check(stream=None):
