@@ -183,7 +183,7 @@ TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb
                            float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Size of the fixed scratch array behind tq_attend_decode_noalloc (8 MiB per device). It covers,
- * for example, B = 16, Hkv = 8, Hq = 32, T = 131072 (about 2.7 MB). */
+ * for example, B = 16, Hkv = 8, Hq = 32, T = 131072 (about 3.4 MB). */
 #define TQ_ATTEND_NOALLOC_MAX_BYTES (8u << 20)
 
 /* tq_attend_decode without a caller workspace: the same computation, arguments, layouts and

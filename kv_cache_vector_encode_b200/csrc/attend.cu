@@ -12,24 +12,33 @@
 //       <q', c[idx]> = sum_S beta_S (Q - 2 <q', b_S>),   Q = sum_i q'_i,
 //     and <q', b_S> is an exact integer tensor-core product: A = the bits b_S (0/1 bytes, scaled
 //     by 2^s, see below), B = beta_S q' in 32-bit fixed point as four signed 8-bit limbs;
-//   * values are accumulated in the rotated / sign domain: for each V plane P (the Walsh
-//     planes of the value codes and the sign plane), Y_P[i] = sum_t w_t b_P,t,i with the softmax
-//     weights w_t (times the value norm, times gamma for the sign plane) in 32-bit unsigned fixed
-//     point as four 8-bit limbs; then o_rot = sum_S beta_S (W - 2 Y_S), o_sign = 2 Y_z - W'
-//     (W = sum_t w_t) and, once per query head, out = Pi^T o_rot / l + alpha S^T o_sign / l.
+//   * values are accumulated in the rotated / sign domain. For each value plane P (the Walsh
+//     planes of the value codes, then the sign plane) the value MMA gives Y_P[i] = sum_t w_t b_P,t,i
+//     with the softmax weights w_t (times the value norm, times gamma for the sign plane) in 32-bit
+//     unsigned fixed point (24 bits) as 8-bit limbs. The chunk sums W = sum_t w_t (and of the other
+//     weight kinds) are exact integer warp reductions, and the per-chunk folds
+//       O_P = sum_t w_t (1 - 2 b_P,t) = W - 2 Y_P,   O_z = sum_t w'_t (2 z_t - 1) = 2 Y_z - W'
+//     are formed per chunk before the running (rescaled) accumulation;
+//   * once per query head: out = (Pi^T sum_P beta_P O_P + alpha S^T O_z) / sum_t p_t.
 //
 // Bit expansion: a 32-bit plane word w covers 32 coordinates; register s (s = 0..7) of
 // (w & (0x01010101 << s)) holds coordinates s, 8+s, 16+s, 24+s as bytes 0 or 2^s. The tensor-core
 // index order inside each 32-coordinate group is therefore k = 4 s + j for coordinate 8 j + s,
 // and the 2^s factor is divided out of the query limbs (scores) or of the output rows (values).
 //
+// Online softmax: a running maximum per head and running maxima of the value weights (which fix
+// the fixed-point scales). A chunk needs the four softmax warps to exchange maxima only when some
+// token exceeds a running maximum; one barrier with an OR-reduction decides that, so after the
+// first chunks of a segment most chunks take no exchange at all.
+//
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
-// (merges the per-CTA partial softmax states of a slice and applies Pi^T, S^T).
+// (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
 // Main-kernel roles (14 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the MMAs;
-// 2-5 token warps (thread = token: expand K into TMEM, then softmax of the chunk); 6-9 expand V
-// into shared memory; 10-13 accumulate the value products (thread = coordinate).
-// All waits are bounded (sm100.cuh).
+// 2-5 softmax (thread = token); 6-9 expand K into TMEM and V into shared memory (thread = token);
+// 10-13 accumulate the value products (thread = coordinate).
+// All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
+// same number of times by all four warps (their loop never exits early).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -44,7 +53,8 @@ namespace {
 
 constexpr int kAttThreads = 448;
 constexpr int kChunk = 128;                 // tokens per chunk
-constexpr int kStages = 4;                  // packed-chunk ring
+constexpr int kMaxStages = 8;               // packed-chunk ring (depth chosen from shared memory)
+constexpr int kMaxSmem = 232448;            // 227 KB of dynamic shared memory per block
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------------------
@@ -54,10 +64,10 @@ struct AttParams {
   int B, Hq, Hkv, Hg, d, G;
   int64_t T;
   int slices, nchunk, per_cta, maxseg;
-  int bk, mk, kmask[4];          // key bits, number of key Walsh planes, plane subsets
-  int bv, mv, vmask[4], vsign;   // value codebook bits, value Walsh planes, subsets, sign plane?
-  int np;                        // value planes (mv + vsign)
-  int nq, nvc;                   // MMA N for scores / values (Hg * 4 rounded up to 16)
+  int nst;                       // depth of the packed-chunk ring
+  int bk, mk;                    // key bits, key Walsh planes
+  int bv, mv, vsign, np;         // value codebook bits, value Walsh planes, sign plane?, planes
+  int nq;                        // MMA N of the scores / of one value weight kind (16 or 32)
   float beta_k[4], beta_v[4];
   float scale_log2e, alpha;
   const void* q;
@@ -71,13 +81,15 @@ struct AttParams {
   const uint16_t* v_norms;
   const uint16_t* v_gammas;
   uint8_t* bq_img;               // [slices][nq rows x mk*d bytes] K-major SW128 image
-  float* head_c;                 // [slices][8][2]: 2^-F_h, Q_h * sum beta
-  float* partial;                // [slices][maxseg][Hg][4 + 2d]
+  float* head_c;                 // [slices][8][2]: 2^-F, Q_h * sum beta
+  float* partial;                // [slices][maxseg][Hg][att_rec(d)]
   float* out;
   uint32_t* err;
 };
 
-__host__ __device__ inline int att_rec(int d) { return 4 + 2 * d; }
+// partial record of one (segment, head): [0] running max (log2 domain), [1] sum of p, [2] 1 when
+// written, [3] unused, then the folded value planes O_P[d] for P = 0..2
+__host__ __device__ inline int att_rec(int d) { return 4 + 3 * d; }
 
 // ------------------------------------------------------------------------------------------------
 // prep: q' = Pi q per query head, fixed-point limbs of beta_S q' (scaled by 2^-s), constants
@@ -173,74 +185,129 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
 // main kernel
 // ------------------------------------------------------------------------------------------------
 struct AttLayout {
-  uint32_t stage_bytes, kc_bytes, vc_bytes;
-  uint32_t off_stage, off_av, av_bytes, off_bw, bw_bytes, off_bq, bq_bytes, off_sc, off_red, off_bar, total;
+  uint32_t kc_bytes, vc_bytes, sg_off, stage_bytes;
+  uint32_t off_stage, av_bytes, off_av, bw_kind, bw_buf, off_bw, bq_bytes, off_bq, off_sc, off_red, off_sum,
+      off_bar, total;
 };
 
 __host__ __device__ inline uint32_t aru(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline AttLayout att_layout(const AttParams& p) {
+__host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   AttLayout L{};
   L.kc_bytes = kChunk * p.G * p.bk * 4;
+  L.sg_off = L.kc_bytes + kChunk * p.G * p.bv * 4;     // sign words of the chunk
   L.vc_bytes = kChunk * p.G * (p.bv + (p.vsign ? 1 : 0)) * 4;
   L.stage_bytes = aru(L.kc_bytes + L.vc_bytes, 1024);
   uint32_t off = 0;
-  L.off_stage = off; off += kStages * L.stage_bytes;
+  L.off_stage = off; off += nst * L.stage_bytes;
   L.av_bytes = kChunk * 128;                       // one plane: 128 tokens x 128 coordinates
   L.off_av = off; off += 2 * p.np * L.av_bytes;
-  L.bw_bytes = (p.nvc / 16) * kChunk * 16;         // one kind: nvc/16 blocks of 128 x 16 bytes
-  L.off_bw = off; off += 2 * 2 * L.bw_bytes;
+  L.bw_kind = (p.nq / 16) * kChunk * 16;           // one weight kind: nq/16 blocks of 128 x 16 bytes
+  L.bw_buf = 2 * L.bw_kind;                        // kinds: w, w * gamma
+  L.off_bw = off; off += 2 * L.bw_buf;
   L.bq_bytes = aru(p.nq * p.mk * p.d, 1024);
   L.off_bq = off; off += 2 * L.bq_bytes;
   L.off_sc = off; off += 4 * 64 * 4;               // chunk scalars, 4-deep ring of 64 floats
-  L.off_red = off; off += 512 * 4;                 // cross-warp reductions of the token warps
+  L.off_red = off; off += 4 * 16 * 4;              // max exchange of the softmax warps
+  L.off_sum = off; off += 4 * 4 * 24 * 4;          // chunk sums of the weights: [ring][warp][kind][head]
   L.off_bar = aru(off, 8); off = L.off_bar + 64 * 8;
   L.total = off + 1024;
   return L;
 }
 
 enum ABars {
-  ST_FULL = 0,                       // [kStages]
-  ST_EMPTY = ST_FULL + kStages,      // [kStages]  (K and V expanders: 8 warps)
-  BQ_FULL = ST_EMPTY + kStages,      // [2]
-  BQ_EMPTY = BQ_FULL + 2,            // [2]
-  AK_FULL = BQ_EMPTY + 2,            // [2]  token warps -> MMA (4 warps)
-  SC_DONE = AK_FULL + 2,             // [2]  scores MMA complete (commit)
-  BW_FULL = SC_DONE + 2,             // [2]  token warps -> MMA (4 warps)
-  AV_FULL = BW_FULL + 2,             // [2]  V expanders -> MMA (4 warps)
-  V_DONE = AV_FULL + 2,              // [2]  value MMA complete (commit)
-  DV_EMPTY = V_DONE + 2,             // [2]  accumulators -> MMA (4 warps)
-  SCAL_FULL = DV_EMPTY + 2,          // [4]  token warps -> accumulators: chunk scalars (4 warps)
-  TOK = SCAL_FULL + 4,               // token-warp group sync (4 warps)
-  ANBARS = TOK + 1
+  ST_FULL = 0,                         // [kMaxStages]
+  ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (expander warps: 4)
+  BQ_FULL = ST_EMPTY + kMaxStages,     // [2]
+  BQ_EMPTY = BQ_FULL + 2,              // [2]
+  AK_FULL = BQ_EMPTY + 2,              // [2]  expanders -> MMA (4 warps)
+  SC_DONE = AK_FULL + 2,               // [2]  scores MMA complete (commit)
+  BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA (4 warps)
+  AV_FULL = BW_FULL + 2,               // [2]  expanders -> MMA (4 warps)
+  V_DONE = AV_FULL + 2,                // [2]  value MMA complete (commit)
+  DV_EMPTY = V_DONE + 2,               // [2]  accumulators -> MMA (4 warps)
+  SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (4 warps)
+  ANBARS = SCAL_FULL + 4
 };
 
-// TMEM columns
-constexpr uint32_t kAK0 = 0;     // [2][128]
-constexpr uint32_t kDS0 = 256;   // [2][<=32]
-constexpr uint32_t kDV0 = 320;   // [2][np][<=32]
+// TMEM columns: A_K [2][128] at 0, scores [2][nq] at 256, value accumulators [2][np][nq] from
+// 256 + 2 nq (at most 512 columns in all: np <= 3, nq <= 32).
+constexpr uint32_t kAK0 = 0;
+constexpr uint32_t kDS0 = 256;
 
-// chunk c of this CTA -> (slice, chunk within slice)
-struct ChunkPos {
-  int slice, cis;   // cis = chunk index inside the slice
+// Walks this CTA's chunks in order (slice, chunk inside the slice, segment ordinal) without
+// integer division.
+struct ChunkIter {
+  int slice, cis, seg, nchunk;
+  __device__ __forceinline__ void init(const AttParams& p, int gchunk) {
+    nchunk = p.nchunk;
+    slice = gchunk / nchunk;
+    cis = gchunk - slice * nchunk;
+    seg = 0;
+  }
+  __device__ __forceinline__ void next() {
+    if (++cis == nchunk) {
+      cis = 0;
+      ++slice;
+      ++seg;
+    }
+  }
 };
-__device__ __forceinline__ ChunkPos chunk_pos(const AttParams& p, int gchunk) {
-  ChunkPos r;
-  r.slice = gchunk / p.nchunk;
-  r.cis = gchunk - r.slice * p.nchunk;
+
+// odd subsets of `bits` bit planes in increasing order (the Walsh planes of a symmetric codebook)
+__host__ __device__ constexpr int walsh_count(int bits) { return bits == 1 ? 1 : (bits == 2 ? 2 : 4); }
+__host__ __device__ constexpr int walsh_mask(int bits, int S) {
+  return bits == 3 ? (S == 0 ? 1 : (S == 1 ? 2 : (S == 2 ? 4 : 7))) : (S == 0 ? 1 : 2);
+}
+
+// Exact int -> float for |x| < 2^22 with two full-rate operations (exponent-field trick).
+__device__ __forceinline__ float small_i2f(int x) {
+  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+}
+// Round-to-nearest of 0 <= v <= 2^23 to an integer with one FMA (v = a * b).
+__device__ __forceinline__ uint32_t fixed24(float a, float b) {
+  return __float_as_uint(fmaf(a, b, 8388608.0f)) - 0x4B000000u;
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz; |relative error| about 2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
   return r;
 }
 
-template <int HG>
+// HG: query heads per KV head (4 or 8, Hg <= HG); BK: key bits; BV: value codebook bits;
+// VS: value sign plane (Algorithm 2 values)
+template <int HG, int BK, int BV, int VS>
 __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __grid_constant__ AttParams p) {
+  constexpr int MK = walsh_count(BK);
+  constexpr int MV = walsh_count(BV);
+  constexpr int NP = MV + VS;
+  constexpr int NQ = HG <= 4 ? 16 : 32;
+  constexpr int NBLK = NQ / 16;
+  constexpr int KSTEPS = MK * 128 / 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const AttLayout Lo = att_layout(p);
+  const int nst = p.nst;
+  const AttLayout Lo = att_layout(p, nst);
   uint64_t* bar = (uint64_t*)(smem + Lo.off_bar);
   uint32_t* tmem_slot = (uint32_t*)(bar + ANBARS);
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + ANBARS) + 1;
   float* scal = (float*)(smem + Lo.off_sc);
   float* red = (float*)(smem + Lo.off_red);
+  uint32_t* sums = (uint32_t*)(smem + Lo.off_sum);   // [4 ring][4 warps][3 kinds][8 heads]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = p.slices * p.nchunk;
   const int c_begin = blockIdx.x * p.per_cta;
@@ -248,11 +315,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
   const int nmy = max(0, c_end - c_begin);
   const int d = p.d, G = p.G;
   const int64_t T = p.T;
+  const uint32_t dv0 = kDS0 + 2 * NQ;
+  const uint32_t dv_cols = NP * NQ;
+  // tokens in the last chunk of every slice (all other chunks are full)
+  const int tail = (int)(T - (int64_t)(p.nchunk - 1) * kChunk);
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < nst; ++s) {
       mbar_init(&bar[ST_FULL + s], 1);
-      mbar_init(&bar[ST_EMPTY + s], 8);
+      mbar_init(&bar[ST_EMPTY + s], 4);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
@@ -265,7 +336,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       mbar_init(&bar[DV_EMPTY + s], 4);
     }
     for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 4);
-    mbar_init(&bar[TOK], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -278,127 +348,265 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  // segment bookkeeping: a new segment starts at the first chunk and whenever the slice changes
-  auto seg_index = [&](int c) -> int {     // ordinal of the segment chunk c (0-based, local) belongs to
-    const int s0 = chunk_pos(p, c_begin).slice;
-    return chunk_pos(p, c_begin + c).slice - s0;
-  };
-  auto seg_first = [&](int c) -> bool {
-    return c == 0 || chunk_pos(p, c_begin + c).cis == 0;
-  };
-  auto seg_last = [&](int c) -> bool {
-    return c == nmy - 1 || chunk_pos(p, c_begin + c).cis == p.nchunk - 1;
-  };
+  ChunkIter it;
+  it.init(p, c_begin);
 
   if (warp == 0) {
     // ------------------------------------ producer -------------------------------------------------
     if (lane == 0) {
-      for (int c = 0; c < nmy; ++c) {
-        const ChunkPos cp = chunk_pos(p, c_begin + c);
-        if (seg_first(c)) {
-          const int sg = seg_index(c);
+      const uint32_t nb = (uint32_t)(NQ * MK * d);
+      for (int c = 0; c < nmy; ++c, it.next()) {
+        if (c == 0 || it.cis == 0) {
+          const int sg = it.seg;
           if (!mbar_wait(&bar[BQ_EMPTY + (sg & 1)], ((sg >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-          const uint32_t nb = (uint32_t)(p.nq * p.mk * d);
           mbar_arrive_expect_tx(&bar[BQ_FULL + (sg & 1)], nb);
-          bulk_g2s(smem + Lo.off_bq + (sg & 1) * Lo.bq_bytes, p.bq_img + (size_t)cp.slice * nb, nb,
+          bulk_g2s(smem + Lo.off_bq + (sg & 1) * Lo.bq_bytes, p.bq_img + (size_t)it.slice * nb, nb,
                    &bar[BQ_FULL + (sg & 1)]);
         }
-        const int st = c % kStages;
-        if (!mbar_wait(&bar[ST_EMPTY + st], ((c / kStages) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        const int64_t t0 = (int64_t)cp.cis * kChunk;
-        const int tc = (int)min((int64_t)kChunk, T - t0);
-        const int64_t vec0 = (int64_t)cp.slice * T + t0;       // record index of the first token
-        const uint32_t kb = (uint32_t)tc * G * p.bk * 4;
-        const uint32_t vb = (uint32_t)tc * G * p.bv * 4;
-        const uint32_t sb = p.vsign ? (uint32_t)tc * G * 4 : 0u;
+        const int st = c % nst;
+        if (!mbar_wait(&bar[ST_EMPTY + st], ((c / nst) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
+        const int64_t vec0 = (int64_t)it.slice * T + (int64_t)it.cis * kChunk;   // record of the first token
+        const uint32_t kb = (uint32_t)tc * G * BK * 4;
+        const uint32_t vb = (uint32_t)tc * G * BV * 4;
+        const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
         mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb);
         uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
-        bulk_g2s(stg, p.k_codes + vec0 * G * p.bk, kb, &bar[ST_FULL + st]);
-        bulk_g2s(stg + Lo.kc_bytes, p.v_codes + vec0 * G * p.bv, vb, &bar[ST_FULL + st]);
-        if (p.vsign)
-          bulk_g2s(stg + Lo.kc_bytes + kChunk * G * p.bv * 4, p.v_signs + vec0 * G, sb, &bar[ST_FULL + st]);
+        bulk_g2s(stg, p.k_codes + vec0 * G * BK, kb, &bar[ST_FULL + st]);
+        bulk_g2s(stg + Lo.kc_bytes, p.v_codes + vec0 * G * BV, vb, &bar[ST_FULL + st]);
+        if (VS) bulk_g2s(stg + Lo.sg_off, p.v_signs + vec0 * G, sb, &bar[ST_FULL + st]);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer -----------------------------------------------
     if (lane == 0) {
-      const uint32_t id_s = idesc_i8_s32(128, p.nq, false, true, false, false);
-      const uint32_t id_v = idesc_i8_s32(128, p.nvc, false, false, true, true);
-      const int ksteps = p.mk * d / 32;
+      const uint32_t id_s = idesc_i8_s32(128, NQ, false, true, false, false);
+      const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
+      // descriptors at the start of each buffer; offsets below are added in 16-byte units
+      const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_bq));
+      const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
+      const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
       auto issue_v = [&](int c) -> bool {
         const int b = c & 1;
         if (!mbar_wait(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
         if (!mbar_wait(&bar[AV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
-        if (!mbar_wait(&bar[DV_EMPTY + b], ((c >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) return false;
+        if (c >= 2 && !mbar_wait(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+          return false;
         tc_fence_after();
-        for (int P = 0; P < p.np; ++P) {
-          const bool sgn = p.vsign && P == p.np - 1;
-          const uint32_t a0 = smem_u32(smem + Lo.off_av + (b * p.np + P) * Lo.av_bytes);
-          const uint32_t b0 = smem_u32(smem + Lo.off_bw + (b * 2 + (sgn ? 1 : 0)) * Lo.bw_bytes);
-          const uint32_t dcol = tbase + kDV0 + (b * p.np + P) * p.nvc;
-          for (int ks = 0; ks < kChunk / 32; ++ks) {
-            const uint64_t da = desc_smem(a0 + ks * 32 * 128, 1024, 1024, 2);
-            const uint64_t db = desc_smem(b0 + ks * 32 * 16, 128, kChunk * 16, 0);
-            mma_i8_ss(dcol, da, db, id_v, ks > 0);
-          }
+        const uint32_t dcol = tbase + dv0 + b * dv_cols;
+        const uint64_t da = da0 + ((b * NP * Lo.av_bytes) >> 4);
+        const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
+#pragma unroll
+        for (int P = 0; P < NP; ++P) {
+          const bool sgn = VS && P == NP - 1;
+#pragma unroll
+          for (int ks = 0; ks < kChunk / 32; ++ks)
+            mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
+                      db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
         }
         mma_commit(&bar[V_DONE + b]);
         return true;
       };
       bool ok = true;
-      for (int c = 0; c < nmy && ok; ++c) {
+      for (int c = 0; c < nmy && ok; ++c, it.next()) {
         const int b = c & 1;
-        const int sg = seg_index(c);
-        if (seg_first(c)) {
+        const int sg = it.seg;
+        if (c == 0 || it.cis == 0) {
           if (!mbar_wait(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
         }
         if (!mbar_wait(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        // D_s[b] is free once the token warps finished chunk c-2 (they arrive BW_FULL after reading it)
+        // the scores buffer b is free once the softmax warps finished chunk c-2 (BW_FULL)
         if (c >= 2 && !mbar_wait(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
         tc_fence_after();
-        const uint32_t bq = smem_u32(smem + Lo.off_bq + (sg & 1) * Lo.bq_bytes);
+        const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
         const uint32_t ak = tbase + kAK0 + b * 128;
-        for (int ks = 0; ks < ksteps; ++ks) {
+        const uint32_t ds = tbase + kDS0 + b * NQ;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
           const uint32_t kbyte = ks * 32, blk = kbyte >> 7, inb = kbyte & 127;
-          mma_i8_ts(tbase + kDS0 + b * 32, ak + ks * 8, desc_kmajor_sw128(bq + blk * p.nq * 128 + inb), id_s, ks > 0);
+          mma_i8_ts(ds, ak + ks * 8, dq + ((blk * NQ * 128 + inb) >> 4), id_s, ks > 0);
         }
         mma_commit(&bar[SC_DONE + b]);
-        if (seg_last(c)) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
+        if (c == nmy - 1 || it.cis == p.nchunk - 1) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
         if (c >= 1) ok = issue_v(c - 1);
       }
       if (ok && nmy >= 1 && !*abort_flag) issue_v(nmy - 1);
     }
   } else if (warp < 6) {
-    // ------------------------------------ token warps ----------------------------------------------
+    // ------------------------------------ softmax warps (thread = token) ---------------------------
     const int q = warp & 3;
     const int t = q * 32 + lane;                    // token inside the chunk == TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
-    uint32_t tok_uses = 0;
-    auto tok_sync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[TOK]);
-      const bool ok = mbar_wait_warp(&bar[TOK], tok_uses & 1, p.err, kDevTimeoutSync, abort_flag);
-      ++tok_uses;
-      return ok;
+    float mrun[HG], ha[HG], hb[HG];
+    float vmax_run = 0.0f, gmax_run = 0.0f, sw = 1.0f, sw2 = 1.0f, isw = 1.0f, isw2 = 1.0f;
+    bool ok = true;
+    // fp16 norms of the next chunk, loaded one chunk ahead and converted only when used (dead
+    // tokens read as zero)
+    uint16_t nk_n = 0, nv_n = 0, gm_n = 0;
+    ChunkIter nx = it;                              // position of the chunk whose norms are prefetched
+    auto load_norms = [&]() {
+      nk_n = nv_n = gm_n = 0;
+      if (t < (nx.cis == p.nchunk - 1 ? tail : kChunk)) {
+        const int64_t rec = (int64_t)nx.slice * T + (int64_t)nx.cis * kChunk + t;
+        nk_n = __ldg(p.k_norms + rec);
+        nv_n = __ldg(p.v_norms + rec);
+        if (VS) gm_n = __ldg(p.v_gammas + rec);
+      }
     };
-    // expand the key codes of chunk c into TMEM (A operand of the scores MMA)
-    auto expand_k = [&](int c) -> bool {
-      const int st = c % kStages, b = c & 1;
-      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / kStages) & 1, p.err, kDevTimeoutLoad, abort_flag)) return false;
-      if (c >= 2 && !mbar_wait_warp(&bar[SC_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
-        return false;
-      tc_fence_after();
-      const ChunkPos cp = chunk_pos(p, c_begin + c);
-      const int tc = (int)min((int64_t)kChunk, T - (int64_t)cp.cis * kChunk);
-      const bool live = t < tc;
-      // the token's G * bk plane words (<= 16, contiguous, 16-byte aligned)
-      const uint4* kw4 = (const uint4*)((const uint32_t*)(smem + Lo.off_stage + st * Lo.stage_bytes) + t * 4 * p.bk);
-      uint32_t kw[16];
+    if (nmy > 0) load_norms();
+    for (int c = 0; c < nmy; ++c, it.next()) {     // no early exit: the named barriers must match
+      const int b = c & 1;
+      const float nk = __half2float(__ushort_as_half(nk_n)), nv = __half2float(__ushort_as_half(nv_n));
+      const float gm = VS ? __half2float(__ushort_as_half(gm_n)) : 0.0f;
+      const bool live = t < (it.cis == p.nchunk - 1 ? tail : kChunk);
+      if (c + 1 < nmy) {
+        nx.next();
+        load_norms();
+      }
+      if (c == 0 || it.cis == 0) {
+        vmax_run = gmax_run = 0.0f;
+        const float2* hc = (const float2*)(p.head_c + it.slice * 16);
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (v4 < p.bk && live) x = kw4[v4];
+        for (int h = 0; h < HG; ++h) {
+          mrun[h] = -INFINITY;
+          const float2 x = h < Hg ? __ldg(hc + h) : make_float2(0.0f, 0.0f);
+          ha[h] = -2.0f * x.x * p.scale_log2e;
+          hb[h] = x.y * p.scale_log2e;
+        }
+      }
+      ok = mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
+      tc_fence_after();
+      uint32_t dsr[NQ];
+      tmem_ld16(tbase + lane_base + kDS0 + b * NQ, *(uint32_t(*)[16]) & dsr[0]);
+      if (NQ > 16) tmem_ld16(tbase + lane_base + kDS0 + b * NQ + 16, *(uint32_t(*)[16]) & dsr[NQ > 16 ? 16 : 0]);
+      tmem_ld_wait();
+      tc_fence_before();
+      float lg[HG];
+      bool up = nv > vmax_run || nv * gm > gmax_run;
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        // the four limb products are exact integers below 2^21 in magnitude
+        const float dot = fmaf(fmaf(fmaf(small_i2f((int)dsr[4 * h + 3]), 256.0f, small_i2f((int)dsr[4 * h + 2])), 256.0f,
+                                    small_i2f((int)dsr[4 * h + 1])),
+                               256.0f, small_i2f((int)dsr[4 * h]));
+        lg[h] = (h < Hg && live) ? nk * fmaf(ha[h], dot, hb[h]) : -INFINITY;
+        up = up || lg[h] > mrun[h];
+      }
+      float corr[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h) corr[h] = 1.0f;
+      if (bar_red_or(1, 128, up)) {
+        // some token raised a running maximum: exchange the chunk maxima of the four warps
+        float* rb = red + q * 16;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const float v = warp_max(lg[h]);
+          if (lane == 0) rb[h] = v;
+        }
+        const float vm = warp_max(nv), gmx = warp_max(nv * gm);
+        if (lane == 0) {
+          rb[8] = vm;
+          rb[9] = gmx;
+        }
+        bar_sync_named(2, 128);
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const float cm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+          const float mn = fmaxf(mrun[h], cm);
+          corr[h] = (mn == -INFINITY) ? 1.0f : fast_exp2(mrun[h] - mn);
+          mrun[h] = mn;
+        }
+        vmax_run = fmaxf(vmax_run, fmaxf(fmaxf(red[8], red[24]), fmaxf(red[40], red[56])));
+        gmax_run = fmaxf(gmax_run, fmaxf(fmaxf(red[9], red[25]), fmaxf(red[41], red[57])));
+        int E1 = 0, E2 = 0;
+        frexpf(fmaxf(vmax_run, 1e-30f), &E1);
+        frexpf(fmaxf(gmax_run, 1e-30f), &E2);
+        E1 = max(E1, -80);
+        E2 = max(E2, -80);
+        sw = ldexpf(1.0f, 23 - E1);                // w * sw <= 2^23 for every w <= vmax_run
+        sw2 = ldexpf(1.0f, 23 - E2);               // likewise for w * gamma
+        isw = ldexpf(1.0f, E1 - 23);
+        isw2 = ldexpf(1.0f, E2 - 23);
+      }
+      // weights: p = 2^(lg - m) <= 1, w = p |v|, w' = w gamma, as 24-bit unsigned fixed point
+      uint32_t wv[HG], wz[HG], pv[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const float pr = (lg[h] == -INFINITY) ? 0.0f : fast_exp2(lg[h] - mrun[h]);
+        const float w = pr * nv;
+        wv[h] = fixed24(w, sw);
+        wz[h] = VS ? fixed24(w * gm, sw2) : 0u;
+        pv[h] = fixed24(pr, 4194304.0f);            // p * 2^22
+      }
+      // chunk sums of each weight kind per head (exact: 32 values below 2^24 per warp)
+      uint32_t* su = sums + ((c & 3) * 4 + q) * 24;
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const uint32_t s0 = warp_sum_u32(wv[h]);
+        const uint32_t s1 = VS ? warp_sum_u32(wz[h]) : 0u;
+        const uint32_t s2 = warp_sum_u32(pv[h]);
+        if (lane == 0) {
+          su[h] = s0;
+          su[8 + h] = s1;
+          su[16 + h] = s2;
+        }
+      }
+      // the weight tiles of chunk c-2 (same buffer) must have been consumed by its value MMA
+      if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
+      uint8_t* bwb = smem + Lo.off_bw + b * Lo.bw_buf + t * 16;
+#pragma unroll
+      for (int blk = 0; blk < NBLK; ++blk) {
+        *(uint4*)(bwb + blk * kChunk * 16) = make_uint4(wv[4 * blk], wv[4 * blk + 1], wv[4 * blk + 2], wv[4 * blk + 3]);
+        if (VS)
+          *(uint4*)(bwb + Lo.bw_kind + blk * kChunk * 16) =
+              make_uint4(wz[4 * blk], wz[4 * blk + 1], wz[4 * blk + 2], wz[4 * blk + 3]);
+      }
+      fence_proxy_async_smem();
+      if (warp == 2) {
+        // chunk scalars for the accumulators (4-deep ring): rescale factors, running maxima, scales
+        float* sc = scal + (c & 3) * 64;
+#pragma unroll
+        for (int h = 0; h < HG; ++h)
+          if (lane == h) {
+            sc[h] = corr[h];
+            sc[16 + h] = mrun[h];
+          }
+        if (lane == 0) {
+          sc[32] = isw;
+          sc[33] = isw2;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[BW_FULL + b]);
+        mbar_arrive(&bar[SCAL_FULL + (c & 3)]);
+      }
+    }
+    (void)ok;
+  } else if (warp < 10) {
+    // ------------------------------------ expanders (thread = token) -------------------------------
+    const int q = warp & 3;
+    const int t = q * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint32_t voff[8];                               // this token's 16-byte slots in a value plane
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      voff[2 * g] = sw128_offset(t, g * 32, 128);
+      voff[2 * g + 1] = sw128_offset(t, g * 32 + 16, 128);
+    }
+    for (int c = 0; c < nmy; ++c) {
+      const int st = c % nst, b = c & 1;
+      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / nst) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+      if (c >= 2 && !mbar_wait_warp(&bar[SC_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
+        break;
+      tc_fence_after();
+      const uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
+      // keys: the token's 4 x BK plane words -> MK Walsh planes of expanded bytes in TMEM
+      uint32_t kw[4 * BK];
+#pragma unroll
+      for (int v4 = 0; v4 < BK; ++v4) {
+        const uint4 x = *(const uint4*)(stg + t * 16 * BK + v4 * 16);
         kw[4 * v4] = x.x;
         kw[4 * v4 + 1] = x.y;
         kw[4 * v4 + 2] = x.z;
@@ -407,252 +615,58 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       const uint32_t ak = tbase + lane_base + kAK0 + b * 128;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        uint32_t pw[4];
 #pragma unroll
-        for (int pl = 0; pl < 4; ++pl) {
-          // word (g, pl) of a bk-plane record sits at g * bk + pl; bk is 1..3 (selects keep kw in registers)
-          const uint32_t w3 = pl < 3 ? kw[3 * g + (pl < 3 ? pl : 0)] : 0u;
-          const uint32_t w2 = pl < 2 ? kw[2 * g + (pl < 2 ? pl : 0)] : 0u;
-          const uint32_t w1 = pl < 1 ? kw[g] : 0u;
-          pw[pl] = p.bk == 3 ? w3 : (p.bk == 2 ? w2 : w1);
+        for (int S = 0; S < MK; ++S) {
+          const int m = walsh_mask(BK, S);
+          uint32_t w = 0;
+          if (m & 1) w ^= kw[g * BK];
+          if (BK > 1 && (m & 2)) w ^= kw[g * BK + (BK > 1 ? 1 : 0)];
+          if (BK > 2 && (m & 4)) w ^= kw[g * BK + (BK > 2 ? 2 : 0)];
+          uint32_t r[8];
+#pragma unroll
+          for (int s8 = 0; s8 < 8; ++s8) r[s8] = w & (0x01010101u << s8);
+          tmem_st8(ak + S * 32 + g * 8, r);
         }
+      }
+      // values: plane words (and sign words) -> expanded bytes, one token row per plane
+      if (c >= 2 && !mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
+        break;
+      uint32_t vw[4 * BV];
 #pragma unroll
-        for (int S = 0; S < 4; ++S) {
-          if (S < p.mk) {
-            const int m = p.kmask[S];
-            const uint32_t w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u) ^ ((m & 4) ? pw[2] : 0u);
-            uint32_t r[8];
+      for (int v4 = 0; v4 < BV; ++v4) {
+        const uint4 x = *(const uint4*)(stg + Lo.kc_bytes + t * 16 * BV + v4 * 16);
+        vw[4 * v4] = x.x;
+        vw[4 * v4 + 1] = x.y;
+        vw[4 * v4 + 2] = x.z;
+        vw[4 * v4 + 3] = x.w;
+      }
+      uint32_t sg[4] = {0u, 0u, 0u, 0u};
+      if (VS) {
+        const uint4 x = *(const uint4*)(stg + Lo.sg_off + t * 16);
+        sg[0] = x.x;
+        sg[1] = x.y;
+        sg[2] = x.z;
+        sg[3] = x.w;
+      }
+      uint8_t* avb = smem + Lo.off_av + b * NP * Lo.av_bytes;
 #pragma unroll
-            for (int s8 = 0; s8 < 8; ++s8) r[s8] = w & (0x01010101u << s8);
-            tmem_st8(ak + S * 32 + g * 8, r);
-          }
+      for (int g = 0; g < 4; ++g) {
+#pragma unroll
+        for (int P = 0; P < NP; ++P) {
+          // the Walsh planes of a 1- or 2-bit codebook are its bit planes
+          const uint32_t w = (VS && P == NP - 1) ? sg[g] : vw[g * BV + (P < BV ? P : 0)];
+          uint8_t* row = avb + P * Lo.av_bytes;
+          *(uint4*)(row + voff[2 * g]) = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
+          *(uint4*)(row + voff[2 * g + 1]) =
+              make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
         }
       }
       tmem_st_wait();
       tc_fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[AK_FULL + b]);
-        mbar_arrive(&bar[ST_EMPTY + st]);
-      }
-      return true;
-    };
-    float m2run[HG];   // running max (log2 domain), kept by every thread
-    bool ok = nmy > 0 ? expand_k(0) : true;
-    for (int c = 0; c < nmy && ok; ++c) {
-      const int b = c & 1;
-      const ChunkPos cp = chunk_pos(p, c_begin + c);
-      const int64_t t0 = (int64_t)cp.cis * kChunk;
-      const int tc = (int)min((int64_t)kChunk, T - t0);
-      const bool live = t < tc;
-      if (seg_first(c)) {
-#pragma unroll
-        for (int h = 0; h < HG; ++h) m2run[h] = -INFINITY;
-      }
-      // per-token inputs (plain loads, issued before the waits)
-      const int64_t rec = (int64_t)cp.slice * T + t0 + t;
-      const float nk = live ? __half2float(__ushort_as_half(__ldg(p.k_norms + rec))) : 0.0f;
-      const float nv = live ? __half2float(__ushort_as_half(__ldg(p.v_norms + rec))) : 0.0f;
-      const float gm = (live && p.vsign) ? __half2float(__ushort_as_half(__ldg(p.v_gammas + rec))) : 0.0f;
-      const float4* hc4 = (const float4*)(p.head_c + cp.slice * 16);
-      float hcf[2 * HG];
-#pragma unroll
-      for (int h2 = 0; h2 < HG / 2; ++h2) {
-        const float4 x = __ldg(hc4 + h2);
-        hcf[4 * h2] = x.x;
-        hcf[4 * h2 + 1] = x.y;
-        hcf[4 * h2 + 2] = x.z;
-        hcf[4 * h2 + 3] = x.w;
-      }
-      if (c + 1 < nmy && !expand_k(c + 1)) break;
-      if (!mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-      tc_fence_after();
-      uint32_t dsr[4 * HG];
-      tmem_ld16(tbase + lane_base + kDS0 + b * 32, *(uint32_t(*)[16]) & dsr[0]);
-      if (HG > 4) tmem_ld16(tbase + lane_base + kDS0 + b * 32 + 16, *(uint32_t(*)[16]) & dsr[HG > 4 ? 16 : 0]);
-      tmem_ld_wait();
-      float lg[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        lg[h] = -INFINITY;
-        if (h < Hg && live) {
-          const long long dot = (long long)(int)dsr[4 * h] + ((long long)(int)dsr[4 * h + 1] << 8) +
-                                ((long long)(int)dsr[4 * h + 2] << 16) + ((long long)(int)dsr[4 * h + 3] << 24);
-          const float score = nk * fmaf(-2.0f * hcf[2 * h], (float)dot, hcf[2 * h + 1]);
-          lg[h] = score * p.scale_log2e;
-        }
-      }
-      // chunk max per head, across the 128 tokens; max |v| (and |v| gamma) for the fixed point
-      float mx[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        float v = lg[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        mx[h] = v;
-      }
-      float vmx = nv, gmx = nv * gm;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
-        gmx = fmaxf(gmx, __shfl_xor_sync(0xffffffffu, gmx, o));
-      }
-      float* rb = red + (c & 1) * 128;
-      if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < HG; ++h) rb[q * 32 + h] = mx[h];
-        rb[q * 32 + 8] = vmx;
-        rb[q * 32 + 9] = gmx;
-      }
-      if (!tok_sync()) break;
-      float m2new[HG], corr[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float cm = fmaxf(fmaxf(rb[h], rb[32 + h]), fmaxf(rb[64 + h], rb[96 + h]));
-        m2new[h] = fmaxf(m2run[h], cm);
-        corr[h] = (m2new[h] == -INFINITY) ? 1.0f : exp2f(m2run[h] - m2new[h]);
-      }
-      const float U = fmaxf(fmaxf(rb[8], rb[40]), fmaxf(rb[72], rb[104]));
-      const float U2 = fmaxf(fmaxf(rb[9], rb[41]), fmaxf(rb[73], rb[105]));
-      int E1 = 0, E2 = 0;
-      frexpf(fmaxf(U, 1e-30f), &E1);
-      frexpf(fmaxf(U2, 1e-30f), &E2);
-      const float sw = ldexpf(1.0f, 32 - E1), sw2 = ldexpf(1.0f, 32 - E2);   // w * sw < 2^32
-      // weights, their fixed-point limbs (one 32-bit word per head = its four limbs) and sums
-      uint32_t wv[HG], wz[HG];
-      float sp[HG], sw_[HG], sz_[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float pr = (lg[h] == -INFINITY) ? 0.0f : exp2f(lg[h] - m2new[h]);
-        const float w = pr * nv, wg = w * gm;
-        wv[h] = __float2uint_rn(w * sw);
-        wz[h] = __float2uint_rn(wg * sw2);
-        sp[h] = pr;
-        sw_[h] = w;
-        sz_[h] = wg;
-      }
-      // the B tiles of the value MMA: token rows of 16 bytes per 4 heads
-      if (c >= 2 && !mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-      uint8_t* bw = smem + Lo.off_bw + (b * 2 + 0) * Lo.bw_bytes;
-      uint8_t* bz = smem + Lo.off_bw + (b * 2 + 1) * Lo.bw_bytes;
-#pragma unroll
-      for (int blk = 0; blk < HG / 4; ++blk) {
-        *(uint4*)(bw + blk * kChunk * 16 + t * 16) = make_uint4(wv[4 * blk], wv[4 * blk + 1], wv[4 * blk + 2], wv[4 * blk + 3]);
-        *(uint4*)(bz + blk * kChunk * 16 + t * 16) = make_uint4(wz[4 * blk], wz[4 * blk + 1], wz[4 * blk + 2], wz[4 * blk + 3]);
-      }
-      // chunk sums per head
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          sp[h] += __shfl_xor_sync(0xffffffffu, sp[h], o);
-          sw_[h] += __shfl_xor_sync(0xffffffffu, sw_[h], o);
-          sz_[h] += __shfl_xor_sync(0xffffffffu, sz_[h], o);
-        }
-      }
-      float* rs = red + 256 + (c & 1) * 128;
-      if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          rs[q * 32 + h] = sp[h];
-          rs[q * 32 + 8 + h] = sw_[h];
-          rs[q * 32 + 16 + h] = sz_[h];
-        }
-      }
-      fence_proxy_async_smem();
-      if (!tok_sync()) break;
-      // chunk scalars for the accumulators (4-deep ring)
-      float* sc = scal + (c & 3) * 64;
-      if (q == 0 && lane < HG) {
-        const int h = lane;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-          a0 += rs[w4 * 32 + h];
-          a1 += rs[w4 * 32 + 8 + h];
-          a2 += rs[w4 * 32 + 16 + h];
-        }
-        float ch = 1.0f, mh = 0.0f;
-#pragma unroll
-        for (int hh = 0; hh < HG; ++hh)
-          if (hh == h) {
-            ch = corr[hh];
-            mh = m2new[hh];
-          }
-        sc[h] = ch;                 // rescale of the running sums
-        sc[8 + h] = a0;             // sum of p
-        sc[16 + h] = a1;            // sum of w = p * |v|
-        sc[24 + h] = a2;            // sum of w' = p * |v| * gamma
-        sc[32 + h] = mh;
-        if (h == 0) {
-          sc[40] = 1.0f / sw;       // fixed-point scales of the two weight kinds
-          sc[41] = 1.0f / sw2;
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < HG; ++h) m2run[h] = m2new[h];
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[SCAL_FULL + (c & 3)]);
-        mbar_arrive(&bar[BW_FULL + b]);
-      }
-    }
-  } else if (warp < 10) {
-    // ------------------------------------ V expanders ----------------------------------------------
-    const int t = (warp - 6) * 32 + lane;
-    for (int c = 0; c < nmy; ++c) {
-      const int st = c % kStages, b = c & 1;
-      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / kStages) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
-      if (c >= 2 && !mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-      const ChunkPos cp = chunk_pos(p, c_begin + c);
-      const int tc = (int)min((int64_t)kChunk, T - (int64_t)cp.cis * kChunk);
-      const bool live = t < tc;
-      const uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
-      const uint4* vw4 = (const uint4*)((const uint32_t*)(stg + Lo.kc_bytes) + t * 4 * p.bv);
-      const uint4* sw4 = (const uint4*)((const uint32_t*)(stg + Lo.kc_bytes + kChunk * 16 * p.bv) + t * 4);
-      uint32_t vwr[8];
-#pragma unroll
-      for (int v4 = 0; v4 < 2; ++v4) {
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (v4 < p.bv && live) x = vw4[v4];
-        vwr[4 * v4] = x.x;
-        vwr[4 * v4 + 1] = x.y;
-        vwr[4 * v4 + 2] = x.z;
-        vwr[4 * v4 + 3] = x.w;
-      }
-      uint4 sx = make_uint4(0, 0, 0, 0);
-      if (p.vsign && live) sx = *sw4;
-      const uint32_t swr[4] = {sx.x, sx.y, sx.z, sx.w};
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t pw[2];
-#pragma unroll
-        for (int pl = 0; pl < 2; ++pl) {
-          const uint32_t w2 = vwr[2 * g + pl];
-          const uint32_t w1 = pl < 1 ? vwr[g] : 0u;
-          pw[pl] = p.bv == 2 ? w2 : w1;
-        }
-#pragma unroll
-        for (int P = 0; P < 3; ++P) {
-          if (P < p.np) {
-            uint32_t w;
-            if (p.vsign && P == p.np - 1) {
-              w = swr[g];
-            } else {
-              const int m = p.vmask[P];
-              w = ((m & 1) ? pw[0] : 0u) ^ ((m & 2) ? pw[1] : 0u);
-            }
-            uint8_t* row = smem + Lo.off_av + (b * p.np + P) * Lo.av_bytes;
-            const uint4 lo4 = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
-            const uint4 hi4 = make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
-            *(uint4*)(row + sw128_offset(t, g * 32, 128)) = lo4;
-            *(uint4*)(row + sw128_offset(t, g * 32 + 16, 128)) = hi4;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
         mbar_arrive(&bar[AV_FULL + b]);
         mbar_arrive(&bar[ST_EMPTY + st]);
       }
@@ -664,79 +678,82 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
     const int g = m >> 5, r = m & 31, s = r >> 2, jj = r & 3;
     const int coord = 32 * g + 8 * jj + s;       // coordinate this row holds
     const float rowscale = ldexpf(1.0f, -s);
+    const float two_s = ldexpf(1.0f, s);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
-    float acc[3][HG];                            // [value plane][head]
-    float Wrun[HG], Zrun[HG], Lrun[HG], Mrun[HG];
-    for (int c = 0; c < nmy; ++c) {
+    float acc[NP][HG];                           // folded planes O_P per head
+    float Lr[HG];                                // sum of p
+    for (int c = 0; c < nmy; ++c, it.next()) {
       const int b = c & 1;
-      const ChunkPos cp = chunk_pos(p, c_begin + c);
-      if (seg_first(c)) {
+      if (c == 0 || it.cis == 0) {
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-          acc[0][h] = acc[1][h] = acc[2][h] = 0.0f;
-          Wrun[h] = Zrun[h] = Lrun[h] = 0.0f;
-          Mrun[h] = -INFINITY;
+          Lr[h] = 0.0f;
+#pragma unroll
+          for (int P = 0; P < NP; ++P) acc[P][h] = 0.0f;
         }
       }
       if (!mbar_wait_warp(&bar[SCAL_FULL + (c & 3)], (c >> 2) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
       if (!mbar_wait_warp(&bar[V_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
+      const uint32_t col = tbase + lane_base + dv0 + b * dv_cols;
+      uint32_t dv[NP][NQ];
+#pragma unroll
+      for (int P = 0; P < NP; ++P) {
+        tmem_ld16(col + P * NQ, *(uint32_t(*)[16]) & dv[P][0]);
+        if (NQ > 16) tmem_ld16(col + P * NQ + 16, *(uint32_t(*)[16]) & dv[P][NQ > 16 ? 16 : 0]);
+      }
+      // chunk sums of the weight kinds (four warp partials each), rescale factors, scales
       const float* sc = scal + (c & 3) * 64;
-      float corr[HG];
+      const uint32_t* su = sums + (c & 3) * 96;
+      float corr[HG], Ws[HG], Zs[HG];
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         corr[h] = sc[h];
-        Lrun[h] = Lrun[h] * corr[h] + sc[8 + h];
-        Wrun[h] = Wrun[h] * corr[h] + sc[16 + h];
-        Zrun[h] = Zrun[h] * corr[h] + sc[24 + h];
-        Mrun[h] = sc[32 + h];
-      }
-      const float fw = sc[40] * rowscale, fz = sc[41] * rowscale;
-#pragma unroll
-      for (int P = 0; P < 3; ++P) {
-        if (P < p.np) {
-          const bool sgn = p.vsign && P == p.np - 1;
-          uint32_t dv[4 * HG];
-          const uint32_t col = tbase + lane_base + kDV0 + (b * p.np + P) * (4 * HG);
-          tmem_ld16(col, *(uint32_t(*)[16]) & dv[0]);
-          if (HG > 4) tmem_ld16(col + 16, *(uint32_t(*)[16]) & dv[HG > 4 ? 16 : 0]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int h = 0; h < HG; ++h) {
-            const unsigned long long y = (unsigned long long)dv[4 * h] + ((unsigned long long)dv[4 * h + 1] << 8) +
-                                         ((unsigned long long)dv[4 * h + 2] << 16) +
-                                         ((unsigned long long)dv[4 * h + 3] << 24);
-            acc[P][h] = fmaf(acc[P][h], corr[h], (float)y * (sgn ? fz : fw));
-          }
+        const uint32_t W = su[h] + su[24 + h] + su[48 + h] + su[72 + h];   // < 2^31
+        Ws[h] = (float)W * two_s;
+        if (VS) Zs[h] = (float)(su[8 + h] + su[32 + h] + su[56 + h] + su[80 + h]) * two_s;
+        if (m == 0) {
+          const uint32_t Lq = su[16 + h] + su[40 + h] + su[64 + h] + su[88 + h];
+          Lr[h] = fmaf(Lr[h], corr[h], (float)Lq * (1.0f / 4194304.0f));
         }
       }
+      const float fw = sc[32] * rowscale, fz = sc[33] * rowscale;
+      const bool last = c == nmy - 1 || it.cis == p.nchunk - 1;
+      float mseg[HG];                            // running maxima, read before the ring slot is released
+#pragma unroll
+      for (int h = 0; h < HG; ++h) mseg[h] = last ? sc[16 + h] : 0.0f;
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[DV_EMPTY + b]);
-      if (seg_last(c)) {
-        // fold the Walsh planes and write this segment's partial state
-        const int sg = cp.slice;
-        const int seg = (c_begin + c) / p.per_cta - (sg * p.nchunk) / p.per_cta;   // CTA ordinal inside the slice
-        float* rec = p.partial + ((size_t)sg * p.maxseg + seg) * Hg * att_rec(d);
+#pragma unroll
+      for (int P = 0; P < NP; ++P) {
+        const bool sgn = VS && P == NP - 1;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          // Y = sum_t 2^s b w (limb sums below 2^22: exact), then the fold 2^s W - 2 Y (or 2 Y - 2^s W')
+          const float y = fmaf(fmaf(small_i2f((int)dv[P][4 * h + 2]), 256.0f, small_i2f((int)dv[P][4 * h + 1])), 256.0f,
+                               small_i2f((int)dv[P][4 * h]));
+          const float o = sgn ? fmaf(2.0f, y, -Zs[h]) : fmaf(-2.0f, y, Ws[h]);
+          acc[P][h] = fmaf(acc[P][h], corr[h], o * (sgn ? fz : fw));
+        }
+      }
+      if (last) {
+        // this segment's partial state
+        const int sgs = it.slice;
+        const int seg = (c_begin + c) / p.per_cta - (sgs * p.nchunk) / p.per_cta;   // CTA ordinal inside the slice
+        float* rec = p.partial + ((size_t)sgs * p.maxseg + seg) * Hg * att_rec(d);
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
           if (h < Hg) {
             float* rh = rec + h * att_rec(d);
-            float om = 0.0f;
 #pragma unroll
-            for (int P = 0; P < 3; ++P)
-              if (P < p.mv) om += p.beta_v[P] * (Wrun[h] - 2.0f * acc[P][h]);
-            float oz = 0.0f;
-#pragma unroll
-            for (int P = 0; P < 3; ++P)
-              if (p.vsign && P == p.np - 1) oz = 2.0f * acc[P][h] - Zrun[h];
-            rh[4 + coord] = om;
-            rh[4 + d + coord] = oz;
+            for (int P = 0; P < NP; ++P) rh[4 + P * d + coord] = acc[P][h];
             if (m == 0) {
-              rh[0] = Mrun[h];
-              rh[1] = Lrun[h];
-              rh[2] = 1.0f;                       // marks a written record
+              rh[0] = mseg[h];
+              rh[1] = Lr[h];
+              rh[2] = 1.0f;
               rh[3] = 0.0f;
             }
           }
@@ -783,16 +800,17 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
   }
   __syncthreads();
   if (i < d) {
-    float a = 0.0f, z = 0.0f;
+    float y[3] = {0.0f, 0.0f, 0.0f};
     for (int sgi = 0; sgi < nseg; ++sgi) {
       const float ms = base[sgi * stride];
       if (ms == -INFINITY) continue;
       const float f = exp2f(ms - mmax);
-      a = fmaf(base[sgi * stride + 4 + i], f, a);
-      z = fmaf(base[sgi * stride + 4 + d + i], f, z);
+      for (int P = 0; P < p.np; ++P) y[P] = fmaf(base[sgi * stride + 4 + P * d + i], f, y[P]);
     }
+    float a = 0.0f;
+    for (int P = 0; P < p.mv; ++P) a = fmaf(p.beta_v[P], y[P], a);
     orot[i] = a * linv;
-    osgn[i] = z * linv;
+    osgn[i] = p.vsign ? y[p.np - 1] * linv : 0.0f;
   }
   __syncthreads();
   if (i < d) {
@@ -825,6 +843,23 @@ int walsh_planes(const tq_codebook* cb, int* mask, float* beta) {
   return n;
 }
 
+using MainKernel = void (*)(AttParams);
+
+template <int HG, int BK>
+MainKernel pick_v(int bv, int vs) {
+  if (bv == 1) return vs ? attend_main_kernel<HG, BK, 1, 1> : attend_main_kernel<HG, BK, 1, 0>;
+  return vs ? attend_main_kernel<HG, BK, 2, 1> : attend_main_kernel<HG, BK, 2, 0>;
+}
+template <int HG>
+MainKernel pick_k(int bk, int bv, int vs) {
+  if (bk == 1) return pick_v<HG, 1>(bv, vs);
+  if (bk == 2) return pick_v<HG, 2>(bv, vs);
+  return pick_v<HG, 3>(bv, vs);
+}
+MainKernel pick_main(int hg, int bk, int bv, int vs) {
+  return hg <= 4 ? pick_k<4>(bk, bv, vs) : pick_k<8>(bk, bv, vs);
+}
+
 struct AttPlan {
   AttParams p;
   size_t bq_bytes, hc_bytes, part_bytes, total;
@@ -847,7 +882,6 @@ bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl) {
   p.per_cta = (int)((totalc + ncta - 1) / ncta);
   p.maxseg = (p.nchunk + p.per_cta - 1) / p.per_cta + 1;
   p.nq = p.Hg <= 4 ? 16 : 32;      // the kernel is built for 4 or 8 heads per KV head
-  p.nvc = p.nq;
   pl.bq_bytes = (size_t)p.slices * p.nq * 4 * d;       // mk <= 4
   pl.hc_bytes = (size_t)p.slices * 16 * sizeof(float);
   pl.part_bytes = (size_t)p.slices * p.maxseg * p.Hg * att_rec(d) * sizeof(float);
@@ -913,13 +947,13 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   if (ws_bytes < pl.total || ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
     return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
   AttParams& p = pl.p;
+  int kmask[4], vmask[4];
   p.bk = cb_k->bits;
-  p.mk = walsh_planes(cb_k, p.kmask, p.beta_k);
+  p.mk = walsh_planes(cb_k, kmask, p.beta_k);
   p.bv = cb_v->bits;
-  p.mv = walsh_planes(cb_v, p.vmask, p.beta_v);
+  p.mv = walsh_planes(cb_v, vmask, p.beta_v);
   p.vsign = vsign ? 1 : 0;
   p.np = p.mv + p.vsign;
-  if (p.np > 3) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": too many value planes");
   p.scale_log2e = scale * kLog2e;
   p.alpha = (float)(std::sqrt(M_PI / 2.0) / d);
   p.q = q;
@@ -941,11 +975,15 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   p.out = out;
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, std::string(f) + ": no device error word");
+  const AttLayout L0 = att_layout(p, 0);
+  const int nst = (int)std::min<long long>(kMaxStages, ((long long)kMaxSmem - (long long)L0.total) / L0.stage_bytes);
+  if (nst < 2) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": shared memory too small for these bit widths");
+  p.nst = nst;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   attend_prep_kernel<<<p.slices, 128, 0, st>>>(p);
-  const AttLayout Lo = att_layout(p);
-  auto kern = p.Hg <= 4 ? attend_main_kernel<4> : attend_main_kernel<8>;
+  const AttLayout Lo = att_layout(p, nst);
+  const MainKernel kern = pick_main(p.Hg, p.bk, p.bv, p.vsign);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode: shared memory attribute");
   const long long totalc = (long long)p.slices * p.nchunk;

@@ -71,9 +71,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // one second per wait
 // Bounded wait for the phase with the given parity. Gives up (returns false) after about one
 // second, or as soon as *abort is non-zero; on its own timeout it records `code` in *err and sets
 // *abort so that the other roles of the block stop waiting too.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
-                                       volatile uint32_t* abort) {
-  if (mbar_try_wait(bar, phase)) return true;
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
+                                            volatile uint32_t* abort) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1; i < (1u << 30); ++i) {
     if (mbar_try_wait(bar, phase)) return true;
@@ -85,6 +84,10 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uin
   if (err) atomicCAS(err, 0u, code);
   if (abort) *abort = 1u;
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
+                                          volatile uint32_t* abort) {
+  return mbar_try_wait(bar, phase) || mbar_wait_slow(bar, phase, err, code, abort);
 }
 
 // Bounded wait made by every lane of a warp with a warp-uniform result, so a warp that arrives on
@@ -257,6 +260,27 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---- named barriers ---------------------------------------------------------------------------
+// Only for groups of warps that all execute the same sequence of these barriers (no early exit).
+
+__device__ __forceinline__ void bar_sync_named(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ uint32_t elect_one_sync() {
   uint32_t pred = 0;
