@@ -151,7 +151,13 @@ TQ_API size_t tq_scores_workspace_bytes(int64_t nq, int64_t n, int32_t d, int32_
  * unbiased estimates; vector-database nearest-neighbour search).
  * scores: optional [nq][n] fp32 output (NULL: not written).
  * k: 0, or 1..16 -- then topk_ids [nq][k] (int32) and topk_scores [nq][k] receive, per query,
- * the k largest scores in descending order, ties to the lower id (ids < 2^31).
+ * the k largest scores in descending order, ties to the lower id (ids < 2^31); when n < k the
+ * missing entries are id -1 with score -inf. k = 0 needs scores.
+ * cb: the codebook the codes use (1..4 bits; b-1 bits for Algorithm 2 codes). d: a multiple of
+ * 64 up to 4096. n may be 0 (codes / norms may then be NULL).
+ * Arithmetic: one tensor-core GEMM over the Walsh bit planes of the codes (exact 0/1 operands) and
+ * the sign plane, against the rotated / projected query in two fp16 parts (about 22 bits);
+ * fp32 accumulation. Without `scores` the database is scanned in chunks and only the top-k kept.
  * ws: caller device workspace of at least tq_scores_workspace_bytes(nq, n, d, k) bytes. */
 TQ_API tq_status tq_scores(const tq_codebook* cb, int64_t nq, int64_t n, int32_t d, const void* q, int32_t q_dtype,
                     const void* rot, const uint32_t* codes, const uint32_t* signs, const uint16_t* norms,

@@ -825,24 +825,6 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
   }
 }
 
-// Walsh coefficients of an exactly symmetric codebook over the odd subsets of its bit planes.
-int walsh_planes(const tq_codebook* cb, int* mask, float* beta) {
-  const int L = cb->levels, bits = cb->bits;
-  int n = 0;
-  for (int m = 1; m < (1 << bits); ++m) {
-    if (!(__builtin_popcount(m) & 1)) continue;
-    double acc = 0.0;
-    for (int idx = 0; idx < L; ++idx) {
-      int par = __builtin_popcount(idx & m) & 1;            // XOR of the planes in the subset
-      acc += (double)cb->c[idx] * (par ? -1.0 : 1.0);       // prod (1 - 2 bit) = 1 - 2 parity
-    }
-    mask[n] = m;
-    beta[n] = (float)(acc / L);
-    ++n;
-  }
-  return n;
-}
-
 using MainKernel = void (*)(AttParams);
 
 template <int HG, int BK>
@@ -947,11 +929,14 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   if (ws_bytes < pl.total || ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
     return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
   AttParams& p = pl.p;
-  int kmask[4], vmask[4];
+  int kmask[8], vmask[8];
+  float kbeta[8], vbeta[8];
   p.bk = cb_k->bits;
-  p.mk = walsh_planes(cb_k, kmask, p.beta_k);
+  p.mk = walsh_planes(cb_k, kmask, kbeta);
+  for (int i = 0; i < p.mk; ++i) p.beta_k[i] = kbeta[i];
   p.bv = cb_v->bits;
-  p.mv = walsh_planes(cb_v, vmask, p.beta_v);
+  p.mv = walsh_planes(cb_v, vmask, vbeta);
+  for (int i = 0; i < p.mv; ++i) p.beta_v[i] = vbeta[i];
   p.vsign = vsign ? 1 : 0;
   p.np = p.mv + p.vsign;
   p.scale_log2e = scale * kLog2e;

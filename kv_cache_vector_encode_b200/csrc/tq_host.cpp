@@ -167,3 +167,24 @@ extern "C" TQ_API tq_status tq_codebook_init(int32_t d, int32_t bits, tq_codeboo
   out->distortion = 1.0 - d * acc;
   return TQ_OK;
 }
+
+namespace tq {
+
+int walsh_planes(const tq_codebook* cb, int* mask, float* beta) {
+  const int L = cb->levels, bits = cb->bits;
+  int n = 0;
+  for (int m = 1; m < (1 << bits); ++m) {
+    if (!(__builtin_popcount(m) & 1)) continue;
+    double acc = 0.0;
+    for (int idx = 0; idx < L; ++idx) {
+      const int par = __builtin_popcount(idx & m) & 1;      // XOR of the planes in the subset
+      acc += (double)cb->c[idx] * (par ? -1.0 : 1.0);       // prod (1 - 2 bit) = 1 - 2 parity
+    }
+    mask[n] = m;
+    beta[n] = (float)(acc / L);
+    ++n;
+  }
+  return n;
+}
+
+}  // namespace tq

@@ -49,6 +49,12 @@ uint32_t* device_error_word();
 // Number of SMs of the current device.
 int sm_count();
 
+// Walsh expansion of an exactly symmetric codebook (c[L-1-k] = -c[k]): for every odd subset m of
+// its bit planes (increasing m), beta_m = mean over idx of c[idx] (1 - 2 parity(idx & m)), so that
+// c[idx] = sum_m beta_m prod_{p in m} (1 - 2 bit_p(idx)). Returns the number of subsets (1, 2, 4
+// or 8 for 1..4 bits); mask and beta must hold 8 entries.
+int walsh_planes(const tq_codebook* cb, int* mask, float* beta);
+
 // 2-D TMA tensor map (128-byte swizzle, zero fill out of range) for a row-major [rows][cols]
 // matrix of esize-byte elements; `tmap` points at a 64-byte-aligned 128-byte CUtensorMap.
 bool make_tmap_2d_sw128(void* tmap, const void* base, int esize, uint64_t cols, uint64_t rows, uint32_t box_cols,
