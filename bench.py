@@ -73,7 +73,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
@@ -434,18 +434,69 @@ def run_ours(args):
     return 0
 
 
+def run_only_attend(args):
+    """Times tq_attend_decode alone on the decode-attention shape with `--att-tokens` cached tokens
+    (a profiling entry point; prints one JSON line with the mean time of a call)."""
+    import torch
+    import kv_cache_vector_encode_b200 as tq
+    import workloads as W
+    dev = torch.device("cuda")
+    T = args.att_tokens
+    Pi, S = W.rotation(D), W.jl_matrix(D)
+    rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    cbk, cbv2 = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS_CACHE - 1)
+    n = ATT_B * ATT_HKV * T
+    kc, kn = tq.empty_mse(n, D, K_BITS, dev)
+    vc, vs, vn, vg = tq.empty_prod(n, D, V_BITS_CACHE, dev)
+    per = ATT_HKV * T
+    for b in range(ATT_B):
+        sl = slice(b * per, (b + 1) * per)
+        tq.tq_encode_mse(cbk, gen_kv(ATT_HKV, T, D, 3, 20.0, 0.5, 1000 + 2 * b, dev), rot, kc[sl], kn[sl])
+        tq.tq_encode_prod(cbv2, gen_kv(ATT_HKV, T, D, 3, 20.0, 0.5, 1001 + 2 * b, dev), rot, vc[sl], vs[sl], vn[sl],
+                          vg[sl])
+    q = torch.randn((ATT_B, ATT_HQ, D), generator=torch.Generator(device=dev).manual_seed(2), device=dev)
+    q = q.to(torch.bfloat16)
+    out = torch.empty((ATT_B, ATT_HQ, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(ATT_B, ATT_HQ, ATT_HKV, T, D), dtype=torch.uint8, device=dev)
+    kn3, vn3, vg3 = kn.view(ATT_B, ATT_HKV, T), vn.view(ATT_B, ATT_HKV, T), vg.view(ATT_B, ATT_HKV, T)
+
+    def call():
+        tq.tq_attend_decode(cbk, cbv2, q, rot, kc, kn3, vc, vn3, out, v_signs=vs, v_gammas=vg3, ws=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        call()
+    b2.record()
+    torch.cuda.synchronize()
+    tq.tq_sync_check()
+    ms = a.elapsed_time(b2) / args.steps
+    byts = B_ATT_TOKEN_HEAD * ATT_B * ATT_HKV * T
+    print(json.dumps({"only": "attend", "tokens": T, "us_per_call": ms * 1e3, "GB/s": byts / (ms * 1e-3) / 1e9}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["attend"], default=None,
+                    help="profiling entry point: time one path alone (not a bench line)")
+    ap.add_argument("--att-tokens", type=int, default=ATT_T)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.only == "attend":
+        return run_only_attend(args)
     return run_ours(args)
 
 
