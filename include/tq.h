@@ -120,18 +120,25 @@ TQ_API tq_status tq_rotation_prepare(int32_t d, const float* Pi, const float* S,
 /* Algorithm 1 encode of n vectors x [n][d] (x_dtype TQ_F32 or TQ_BF16) with a b-bit codebook
  * (cb->d must equal d): writes codes [n][d/32][b] and norms [n] (fp16 bits).
  * (ai-navigate-news page: Algorithm 1 = rotation, Lloyd-Max scalar quantisation, MSE-optimal;
- * keys use it.) d in {32, 64, 96, 128, ..., 256} on the fused tensor-core path; larger d
- * (multiples of 128 up to 4096) on the tiled path. n may be 0 (no work). */
+ * keys use it.) d <= 128 (any multiple of 32) runs the fused kernel; d > 128 must be a multiple of
+ * 128 (up to 4096) and runs the tiled kernel. n may be 0 (no work). */
 TQ_API tq_status tq_encode_mse(const tq_codebook* cb, int64_t n, int32_t d, const void* x, int32_t x_dtype,
                         const void* rot, uint32_t* codes, uint16_t* norms, void* stream);
 
 /* Algorithm 2 encode at b bits: Algorithm 1 with the (b-1)-bit codebook `cb_bm1`, then the
  * residual sign bits and the residual norm (ai-navigate-news page: Algorithm 2 = Algorithm 1 at
  * b-1 bits plus sign(S r), unbiased inner products; values use it). Writes codes
- * [n][d/32][b-1], signs [n][d/32], norms [n], gammas [n]. Limits as tq_encode_mse. */
+ * [n][d/32][b-1], signs [n][d/32], norms [n], gammas [n]. Limits as tq_encode_mse.
+ * ws: caller device workspace of tq_encode_workspace_bytes(n, d, 2) bytes (16-byte aligned); that
+ * is 0 for d <= 128 (ws may then be NULL). For d > 128 it holds the residuals of the tiles in
+ * flight (one slot per SM). */
 TQ_API tq_status tq_encode_prod(const tq_codebook* cb_bm1, int64_t n, int32_t d, const void* x, int32_t x_dtype,
                          const void* rot, uint32_t* codes, uint32_t* signs, uint16_t* norms, uint16_t* gammas,
-                         void* stream);
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes an encode of n vectors of length d needs (alg 1: tq_encode_mse, which needs
+ * none; alg 2: tq_encode_prod). Depends on the SM count of the current device. */
+TQ_API size_t tq_encode_workspace_bytes(int64_t n, int32_t d, int32_t alg);
 
 /* Dequantise n packed vectors: x_hat = n (Pi^T c[idx] (+ alpha gamma S^T (2z-1))) into
  * out [n][d] of out_dtype (TQ_F32 or TQ_BF16). signs and gammas both NULL for Algorithm 1

@@ -64,7 +64,8 @@ _SIGNATURES = {
     "tq_rotation_bytes": (_SZ, [_I32]),
     "tq_rotation_prepare": (_I32, [_I32, _P, _P, _P, _SZ, _P]),
     "tq_encode_mse": (_I32, [_CB, _I64, _I32, _P, _I32, _P, _P, _P, _P]),
-    "tq_encode_prod": (_I32, [_CB, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P]),
+    "tq_encode_prod": (_I32, [_CB, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tq_encode_workspace_bytes": (_SZ, [_I64, _I32, _I32]),
     "tq_decode": (_I32, [_CB, _I64, _I32, _P, _P, _P, _P, _P, _P, _I32, _P]),
     "tq_scores_workspace_bytes": (_SZ, [_I64, _I64, _I32, _I32]),
     "tq_scores": (_I32, [_CB, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
@@ -162,13 +163,21 @@ def tq_encode_mse(cb: Codebook, x, rot, codes, norms, stream=None):
                                _ptr(norms, "norms", [torch.float16]), _stream(stream)))
 
 
-def tq_encode_prod(cb_bm1: Codebook, x, rot, codes, signs, norms, gammas, stream=None):
+def tq_encode_workspace_bytes(n: int, d: int, alg: int) -> int:
+    return int(lib().tq_encode_workspace_bytes(n, d, alg))
+
+
+def tq_encode_prod(cb_bm1: Codebook, x, rot, codes, signs, norms, gammas, ws=None, stream=None):
     import torch
     n, d = x.shape
+    wsb = tq_encode_workspace_bytes(n, d, 2)
+    if ws is None and wsb > 0:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=x.device)
     _check(lib().tq_encode_prod(ctypes.byref(cb_bm1), n, d, _ptr(x, "x", [torch.float32, torch.bfloat16]),
                                 _xdtype(x), _ptr(rot, "rot"), _ptr(codes, "codes", [torch.int32]),
                                 _ptr(signs, "signs", [torch.int32]), _ptr(norms, "norms", [torch.float16]),
-                                _ptr(gammas, "gammas", [torch.float16]), _stream(stream)))
+                                _ptr(gammas, "gammas", [torch.float16]), _ptr(ws, "ws", None, True),
+                                ws.numel() if ws is not None else 0, _stream(stream)))
 
 
 def tq_decode(cb: Codebook, rot, codes, norms, out, signs=None, gammas=None, stream=None):

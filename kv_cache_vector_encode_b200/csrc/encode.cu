@@ -38,6 +38,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "quant_device.cuh"
 #include "sm100.cuh"
 #include "tq_internal.h"
 
@@ -70,7 +71,6 @@ struct EncLayout {
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
 
 // raw tile: bf16 -> NV rows x KP columns (KP/64 boxes of 64 columns); fp32 -> NV rows x DF columns
 // (DF = d rounded up to 32, DF/32 boxes of 32 columns).
@@ -117,40 +117,6 @@ __device__ __forceinline__ float transpose_reduce16(float (&r)[16], int lane) {
     }
   }
   return r[0] + __shfl_xor_sync(0xffffffffu, r[0], 16);
-}
-
-// m = #{positive boundaries < a} by binary search over the H-1 positive boundaries.
-template <int BITS>
-__device__ __forceinline__ int sym_m(float a, const float (&P)[8]) {
-  if (BITS == 1) return 0;
-  if (BITS == 2) return a > P[0] ? 1 : 0;
-  if (BITS == 3) {
-    const int m1 = a > P[1] ? 1 : 0;
-    const int m0 = a > (m1 ? P[2] : P[0]) ? 1 : 0;
-    return 2 * m1 + m0;
-  }
-  const int m2 = a > P[3] ? 1 : 0;
-  const int m1 = a > (m2 ? P[5] : P[1]) ? 1 : 0;
-  const float p0 = m2 ? (m1 ? P[6] : P[4]) : (m1 ? P[2] : P[0]);
-  const int m0 = a > p0 ? 1 : 0;
-  return 4 * m2 + 2 * m1 + m0;
-}
-
-template <int BITS>
-__device__ __forceinline__ float sym_c(int m, const float (&C)[8]) {
-  if (BITS == 1) return C[0];
-  if (BITS == 2) return m ? C[1] : C[0];
-  if (BITS == 3) return (m & 2) ? ((m & 1) ? C[3] : C[2]) : ((m & 1) ? C[1] : C[0]);
-  const float lo = (m & 2) ? ((m & 1) ? C[3] : C[2]) : ((m & 1) ? C[1] : C[0]);
-  const float hi = (m & 2) ? ((m & 1) ? C[7] : C[6]) : ((m & 1) ? C[5] : C[4]);
-  return (m & 4) ? hi : lo;
-}
-
-// two exact power-of-two factors whose product is 2^e (e may exceed the fp32 exponent range)
-__device__ __forceinline__ void pow2_pair(int e, float& f1, float& f2) {
-  const int e1 = max(min(e, 120), -120);
-  f1 = __int_as_float((127 + e1) << 23);
-  f2 = __int_as_float((127 + (e - e1)) << 23);
 }
 
 template <int XT, bool ALG2, int NV, int BITS>
@@ -525,7 +491,7 @@ tq_status launch_bits(EncodeParams& p, int bits, const void* x, cudaStream_t st)
 
 tq_status encode_common(const char* fn, const tq_codebook* cb, int64_t n, int32_t d, const void* x, int32_t xt,
                         const void* rot, uint32_t* codes, uint32_t* signs, uint16_t* norms, uint16_t* gammas,
-                        bool alg2, void* stream) {
+                        bool alg2, void* ws, size_t ws_bytes, void* stream) {
   clear_error();
   std::string f(fn);
   if (!cb || !rot || !codes || !norms || (n > 0 && !x)) return fail(TQ_ERR_INVALID_ARG, f + ": NULL pointer");
@@ -544,8 +510,8 @@ tq_status encode_common(const char* fn, const tq_codebook* cb, int64_t n, int32_
       (alg2 && (!aligned16(signs) || !aligned16(gammas))))
     return fail(TQ_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
   if (n == 0) return TQ_OK;
-  if (d > 128) return fail(TQ_ERR_UNSUPPORTED, f + ": d > 128 is not supported by this build");
   if (n > ((int64_t)1 << 31) - 256) return fail(TQ_ERR_UNSUPPORTED, f + ": n >= 2^31");
+  if (d > 128) return encode_tiled(cb, n, d, x, xt, rot, codes, signs, norms, gammas, alg2, ws, ws_bytes, stream);
   RotLayout RL = rot_layout(d);
   const uint8_t* base = (const uint8_t*)rot;
   EncodeParams p{};
@@ -581,13 +547,26 @@ tq_status encode_common(const char* fn, const tq_codebook* cb, int64_t n, int32_
 
 using namespace tq;
 
+extern "C" TQ_API size_t tq_encode_workspace_bytes(int64_t n, int32_t d, int32_t alg) {
+  if (n < 0 || (alg != 1 && alg != 2) || !valid_dim(d)) return 0;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      nsm <= 0) {
+    cudaGetLastError();
+    nsm = 148;
+  }
+  return encode_tiled_ws_bytes(n, d, alg == 2, nsm);
+}
+
 extern "C" TQ_API tq_status tq_encode_mse(const tq_codebook* cb, int64_t n, int32_t d, const void* x, int32_t x_dtype,
                                    const void* rot, uint32_t* codes, uint16_t* norms, void* stream) {
-  return encode_common("tq_encode_mse", cb, n, d, x, x_dtype, rot, codes, nullptr, norms, nullptr, false, stream);
+  return encode_common("tq_encode_mse", cb, n, d, x, x_dtype, rot, codes, nullptr, norms, nullptr, false, nullptr, 0,
+                       stream);
 }
 
 extern "C" TQ_API tq_status tq_encode_prod(const tq_codebook* cb_bm1, int64_t n, int32_t d, const void* x, int32_t x_dtype,
                                     const void* rot, uint32_t* codes, uint32_t* signs, uint16_t* norms,
-                                    uint16_t* gammas, void* stream) {
-  return encode_common("tq_encode_prod", cb_bm1, n, d, x, x_dtype, rot, codes, signs, norms, gammas, true, stream);
+                                    uint16_t* gammas, void* ws, size_t ws_bytes, void* stream) {
+  return encode_common("tq_encode_prod", cb_bm1, n, d, x, x_dtype, rot, codes, signs, norms, gammas, true, ws, ws_bytes,
+                       stream);
 }

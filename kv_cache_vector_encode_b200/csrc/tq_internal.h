@@ -49,6 +49,12 @@ uint32_t* device_error_word();
 // Number of SMs of the current device.
 int sm_count();
 
+// Tiled encode for d > 128 (encode_tiled.cu): workspace bytes (Algorithm 2 only) and the launch.
+size_t encode_tiled_ws_bytes(int64_t n, int d, bool alg2, int nsm);
+tq_status encode_tiled(const tq_codebook* cb, int64_t n, int d, const void* x, int xt, const void* rot,
+                       uint32_t* codes, uint32_t* signs, uint16_t* norms, uint16_t* gammas, bool alg2, void* ws,
+                       size_t ws_bytes, void* stream);
+
 // Walsh expansion of an exactly symmetric codebook (c[L-1-k] = -c[k]): for every odd subset m of
 // its bit planes (increasing m), beta_m = mean over idx of c[idx] (1 - 2 parity(idx & m)), so that
 // c[idx] = sum_m beta_m prod_{p in m} (1 - 2 bit_p(idx)). Returns the number of subsets (1, 2, 4

@@ -68,8 +68,8 @@ def check_signs(gpu_words: np.ndarray, ora_z: np.ndarray, ora_s: np.ndarray, ora
     return stats
 
 
-def check_fp16(gpu16: np.ndarray, exact: np.ndarray, name: str):
-    """fp16 values: equal to RNE(exact) or one ulp away next to a rounding midpoint."""
+def check_fp16(gpu16: np.ndarray, exact: np.ndarray, name: str, mid_tol: float = 2.0 ** -20):
+    """fp16 values: equal to RNE(exact) or one ulp away within mid_tol (relative) of a rounding midpoint."""
     g = np.asarray(gpu16, dtype=np.float16)
     o = np.asarray(exact, dtype=np.float64).astype(np.float16)
     diff = g.view(np.uint16).astype(np.int64) - o.view(np.uint16).astype(np.int64)
@@ -81,7 +81,9 @@ def check_fp16(gpu16: np.ndarray, exact: np.ndarray, name: str):
         hi = np.maximum(g[bad].astype(np.float64), o[bad].astype(np.float64))
         mid = 0.5 * (lo + hi)
         ex = np.asarray(exact, dtype=np.float64)[bad]
-        assert np.all(np.abs(ex - mid) <= 2.0 ** -20 * np.abs(ex)), f"{name}: off-by-one not at a midpoint"
+        rel = np.abs(ex - mid) / np.abs(ex)
+        assert np.all(rel <= mid_tol), \
+            f"{name}: off-by-one not at a midpoint ({int((rel > mid_tol).sum())} of {nb}, max rel {rel.max():.3g})"
     return dict(total=g.size, off_by_one=nb)
 
 

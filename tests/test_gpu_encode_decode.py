@@ -92,7 +92,9 @@ def check_prod(x, d, bits, dtype, dev, decode=True):
     ora2 = Q.residual_signs(ora["u"], gidx, ora["n"], Pi, S, ora_cb)
     st["signs"] = check_signs(np_u32(signs), ora2["z"], ora2["s"], ora2["gamma"], d)
     check_fp16(np_f16(norms), ora["n"], "norms")
-    check_fp16(np_f16(gammas), ora2["gamma"], "gammas")
+    # gamma comes from y = Pi x accumulated in fp32 over K = d in the tensor core: its relative
+    # error grows with d, so for d > 128 the midpoint window grows in proportion to d / 128
+    check_fp16(np_f16(gammas), ora2["gamma"], "gammas", 2.0 ** -20 * max(1.0, d / 128))
     if decode:
         out = torch.empty((len(x), d), dtype=torch.float32, device=dev)
         tq.tq_decode(cb, rot, codes, norms, out, signs=signs, gammas=gammas)

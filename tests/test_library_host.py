@@ -80,8 +80,16 @@ def test_device_calls_reject_bad_arguments_on_host(L):
         == tq.TQ_ERR_INVALID_ARG
     assert L.tq_encode_mse(ctypes.byref(cb), 10, 128, good, tq.TQ_F16, good, good, good, None) == tq.TQ_ERR_UNSUPPORTED
     assert L.tq_encode_mse(ctypes.byref(cb), 0, 128, good, tq.TQ_BF16, good, good, good, None) == tq.TQ_OK
-    assert L.tq_encode_prod(ctypes.byref(cb), 10, 128, good, tq.TQ_BF16, good, good, None, good, good, None) \
+    assert L.tq_encode_prod(ctypes.byref(cb), 10, 128, good, tq.TQ_BF16, good, good, None, good, good, None, 0, None) \
         == tq.TQ_ERR_INVALID_ARG
+    # d > 128 must be a multiple of 128; Algorithm 2 there needs its workspace
+    cb256 = tq.tq_codebook_init(256, 2)
+    assert L.tq_encode_mse(ctypes.byref(tq.tq_codebook_init(160, 2)), 10, 160, good, tq.TQ_BF16, good, good, good,
+                           None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_workspace_bytes(10, 128, 2) == 0 and L.tq_encode_workspace_bytes(1000, 256, 1) == 0
+    assert L.tq_encode_workspace_bytes(1000, 256, 2) > 0
+    assert L.tq_encode_prod(ctypes.byref(cb256), 1000, 256, good, tq.TQ_BF16, good, good, good, good, good, None, 0,
+                            None) == tq.TQ_ERR_WORKSPACE
     assert L.tq_decode(ctypes.byref(cb), 10, 128, good, good, good, good, None, good, tq.TQ_F32, None) \
         == tq.TQ_ERR_INVALID_ARG
     assert L.tq_rotation_prepare(128, good, good, good, 16, None) == tq.TQ_ERR_WORKSPACE
