@@ -353,49 +353,56 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
 
   if (warp == 0) {
     // ------------------------------------ producer -------------------------------------------------
-    if (lane == 0) {
-      const uint32_t nb = (uint32_t)(NQ * MK * d);
-      for (int c = 0; c < nmy; ++c, it.next()) {
-        if (c == 0 || it.cis == 0) {
-          const int sg = it.seg;
-          if (!mbar_wait(&bar[BQ_EMPTY + (sg & 1)], ((sg >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+    // warp-uniform schedule; one elected lane issues the copies
+    const uint32_t nb = (uint32_t)(NQ * MK * d);
+    for (int c = 0; c < nmy; ++c, it.next()) {
+      if (c == 0 || it.cis == 0) {
+        const int sg = it.seg;
+        if (!mbar_wait_warp(&bar[BQ_EMPTY + (sg & 1)], ((sg >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (elect_one_sync()) {
           mbar_arrive_expect_tx(&bar[BQ_FULL + (sg & 1)], nb);
           bulk_g2s(smem + Lo.off_bq + (sg & 1) * Lo.bq_bytes, p.bq_img + (size_t)it.slice * nb, nb,
                    &bar[BQ_FULL + (sg & 1)]);
         }
-        const int st = c % nst;
-        if (!mbar_wait(&bar[ST_EMPTY + st], ((c / nst) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
-        const int64_t vec0 = (int64_t)it.slice * T + (int64_t)it.cis * kChunk;   // record of the first token
-        const uint32_t kb = (uint32_t)tc * G * BK * 4;
-        const uint32_t vb = (uint32_t)tc * G * BV * 4;
-        const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
+        __syncwarp();
+      }
+      const int st = c % nst;
+      if (!mbar_wait_warp(&bar[ST_EMPTY + st], ((c / nst) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
+      const int64_t vec0 = (int64_t)it.slice * T + (int64_t)it.cis * kChunk;   // record of the first token
+      const uint32_t kb = (uint32_t)tc * G * BK * 4;
+      const uint32_t vb = (uint32_t)tc * G * BV * 4;
+      const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
+      uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
+      if (elect_one_sync()) {
         mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb);
-        uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
         bulk_g2s(stg, p.k_codes + vec0 * G * BK, kb, &bar[ST_FULL + st]);
         bulk_g2s(stg + Lo.kc_bytes, p.v_codes + vec0 * G * BV, vb, &bar[ST_FULL + st]);
         if (VS) bulk_g2s(stg + Lo.sg_off, p.v_signs + vec0 * G, sb, &bar[ST_FULL + st]);
       }
+      __syncwarp();
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer -----------------------------------------------
-    if (lane == 0) {
-      const uint32_t id_s = idesc_i8_s32(128, NQ, false, true, false, false);
-      const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
-      // descriptors at the start of each buffer; offsets below are added in 16-byte units
-      const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_bq));
-      const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
-      const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
-      auto issue_v = [&](int c) -> bool {
-        const int b = c & 1;
-        if (!mbar_wait(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
-        if (!mbar_wait(&bar[AV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
-        if (c >= 2 && !mbar_wait(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
-          return false;
-        tc_fence_after();
-        const uint32_t dcol = tbase + dv0 + b * dv_cols;
-        const uint64_t da = da0 + ((b * NP * Lo.av_bytes) >> 4);
-        const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
+    // The whole warp walks the schedule (its values are warp-uniform and stay in uniform
+    // registers); one elected lane issues each group of tcgen05 instructions and their commits.
+    const uint32_t id_s = idesc_i8_s32(128, NQ, false, true, false, false);
+    const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
+    // descriptors at the start of each buffer; offsets below are added in 16-byte units
+    const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_bq));
+    const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
+    const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
+    auto issue_v = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
+      if (!mbar_wait_warp(&bar[AV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
+      if (c >= 2 && !mbar_wait_warp(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+        return false;
+      tc_fence_after();
+      const uint32_t dcol = tbase + dv0 + b * dv_cols;
+      const uint64_t da = da0 + ((b * NP * Lo.av_bytes) >> 4);
+      const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
+      if (elect_one_sync()) {
 #pragma unroll
         for (int P = 0; P < NP; ++P) {
           const bool sgn = VS && P == NP - 1;
@@ -405,33 +412,39 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
                       db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
         }
         mma_commit(&bar[V_DONE + b]);
-        return true;
-      };
-      bool ok = true;
-      for (int c = 0; c < nmy && ok; ++c, it.next()) {
-        const int b = c & 1;
-        const int sg = it.seg;
-        if (c == 0 || it.cis == 0) {
-          if (!mbar_wait(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
-        }
-        if (!mbar_wait(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        // the scores buffer b is free once the softmax warps finished chunk c-2 (BW_FULL)
-        if (c >= 2 && !mbar_wait(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        tc_fence_after();
-        const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
-        const uint32_t ak = tbase + kAK0 + b * 128;
-        const uint32_t ds = tbase + kDS0 + b * NQ;
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = true;
+    for (int c = 0; c < nmy && ok; ++c, it.next()) {
+      const int b = c & 1;
+      const int sg = it.seg;
+      if (c == 0 || it.cis == 0) {
+        if (!mbar_wait_warp(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+      }
+      if (!mbar_wait_warp(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      // the scores buffer b is free once the softmax warps finished chunk c-2 (BW_FULL)
+      if (c >= 2 && !mbar_wait_warp(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+        break;
+      tc_fence_after();
+      const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
+      const uint32_t ak = tbase + kAK0 + b * 128;
+      const uint32_t ds = tbase + kDS0 + b * NQ;
+      const bool last = c == nmy - 1 || it.cis == p.nchunk - 1;
+      if (elect_one_sync()) {
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
           const uint32_t kbyte = ks * 32, blk = kbyte >> 7, inb = kbyte & 127;
           mma_i8_ts(ds, ak + ks * 8, dq + ((blk * NQ * 128 + inb) >> 4), id_s, ks > 0);
         }
         mma_commit(&bar[SC_DONE + b]);
-        if (c == nmy - 1 || it.cis == p.nchunk - 1) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
-        if (c >= 1) ok = issue_v(c - 1);
+        if (last) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
       }
-      if (ok && nmy >= 1 && !*abort_flag) issue_v(nmy - 1);
+      __syncwarp();
+      if (c >= 1) ok = issue_v(c - 1);
     }
+    if (ok && nmy >= 1 && !*abort_flag) issue_v(nmy - 1);
   } else if (warp < 6) {
     // ------------------------------------ softmax warps (thread = token) ---------------------------
     const int q = warp & 3;

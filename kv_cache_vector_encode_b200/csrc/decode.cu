@@ -104,12 +104,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   const int my_tiles = p.ntiles > (int)blockIdx.x ? (p.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (elect_one_sync()) {
       mbar_arrive_expect_tx(&bar[A_FULL], na * p.img_bytes);
       for (int m = 0; m < na; ++m) bulk_g2s(smem + Lo.off_a[m], p.img[m], p.img_bytes, &bar[A_FULL]);
     }
+    __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && mbar_wait(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
+    // warp-uniform schedule (descriptors stay in uniform registers); one elected lane issues
+    if (mbar_wait_warp(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
@@ -118,25 +120,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       const int ksteps = KP / 16;
       for (int k = 0; k < my_tiles; ++k) {
         const int a = k & 1;
-        if (!mbar_wait(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        if (!mbar_wait(&bar[B_FULL], k & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[B_FULL], k & 1, p.err, kDevTimeoutSync, abort_flag)) break;
         tc_fence_after();
         const uint32_t d1a = tbase + a * COLS, d1b = d1a + NV, d2a = d1a + 2 * NV, d2b = d1a + 3 * NV;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
-          const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
-          const uint64_t dch = desc_kmajor_sw128(bch + bo);
-          mma_f16_ss(d1a, desc_kmajor_sw128(a0 + ao), dch, idesc, ks > 0);
-          mma_f16_ss(d1b, desc_kmajor_sw128(a1 + ao), dch, idesc, ks > 0);
-          mma_f16_ss(d1b, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bcl + bo), idesc, 1);
-          if (ALG2) {
-            const uint64_t dsg = desc_kmajor_sw128(bs + bo);
-            mma_f16_ss(d2a, desc_kmajor_sw128(a2 + ao), dsg, idesc, ks > 0);
-            mma_f16_ss(d2b, desc_kmajor_sw128(a3 + ao), dsg, idesc, ks > 0);
+        if (elect_one_sync()) {
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
+            const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
+            const uint64_t dch = desc_kmajor_sw128(bch + bo);
+            mma_f16_ss(d1a, desc_kmajor_sw128(a0 + ao), dch, idesc, ks > 0);
+            mma_f16_ss(d1b, desc_kmajor_sw128(a1 + ao), dch, idesc, ks > 0);
+            mma_f16_ss(d1b, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bcl + bo), idesc, 1);
+            if (ALG2) {
+              const uint64_t dsg = desc_kmajor_sw128(bs + bo);
+              mma_f16_ss(d2a, desc_kmajor_sw128(a2 + ao), dsg, idesc, ks > 0);
+              mma_f16_ss(d2b, desc_kmajor_sw128(a3 + ao), dsg, idesc, ks > 0);
+            }
           }
+          mma_commit(&bar[B_EMPTY]);
+          mma_commit(&bar[ACC_FULL + a]);
         }
-        mma_commit(&bar[B_EMPTY]);
-        mma_commit(&bar[ACC_FULL + a]);
+        __syncwarp();
       }
     }
   } else if (warp < 6) {

@@ -174,23 +174,29 @@ __global__ void __launch_bounds__(kEncThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer: resident operands (bulk), input tiles (TMA) ----------------------
-    if (lane == 0) {
+    // warp-uniform schedule; one elected lane issues the copies
+    if (elect_one_sync()) {
       mbar_arrive_expect_tx(&bar[A_FULL], na * p.img_bytes);
       for (int m = 0; m < na; ++m) bulk_g2s(smem + Lo.off_a[m], p.img[m], p.img_bytes, &bar[A_FULL]);
-      const int nbox = F32 ? (d + 31) / 32 : KP / 64;
-      const uint32_t box_bytes = NV * 128;
-      for (int k = 0; k < my_tiles; ++k) {
-        const int s = k & 1;
-        const int t = blockIdx.x + k * gridDim.x;
-        if (!mbar_wait(&bar[STAGE_EMPTY + s], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+    }
+    __syncwarp();
+    const int nbox = F32 ? (d + 31) / 32 : KP / 64;
+    const uint32_t box_bytes = NV * 128;
+    for (int k = 0; k < my_tiles; ++k) {
+      const int s = k & 1;
+      const int t = blockIdx.x + k * gridDim.x;
+      if (!mbar_wait_warp(&bar[STAGE_EMPTY + s], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      if (elect_one_sync()) {
         mbar_arrive_expect_tx(&bar[RAW_FULL + s], nbox * box_bytes);
         for (int b = 0; b < nbox; ++b)
           tma_load_2d(smem + raw_off(s) + b * box_bytes, &tmap, b * (F32 ? 32 : 64), t * NV, &bar[RAW_FULL + s]);
       }
+      __syncwarp();
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ---------------------------------------------------------------
-    if (lane == 0 && mbar_wait(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
+    // warp-uniform schedule (descriptors stay in uniform registers); one elected lane issues
+    if (mbar_wait_warp(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
@@ -198,38 +204,44 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       const int ksteps = KP / 16;
       auto issue_T = [&](int j) -> bool {
         const int a = j & 1;
-        if (!mbar_wait(&bar[RHO_FULL], j & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
+        if (!mbar_wait_warp(&bar[RHO_FULL], j & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
         tc_fence_after();
         const uint32_t dT1 = tbase + a * COLS + 2 * NV, dT2 = dT1 + NV;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
-          const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
-          mma_f16_ss(dT1, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
-          mma_f16_ss(dT2, desc_kmajor_sw128(a3 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
-          mma_f16_ss(dT2, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r1 + bo), idesc, 1);
+        if (elect_one_sync()) {
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
+            const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
+            mma_f16_ss(dT1, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
+            mma_f16_ss(dT2, desc_kmajor_sw128(a3 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
+            mma_f16_ss(dT2, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r1 + bo), idesc, 1);
+          }
+          mma_commit(&bar[T_FULL + a]);
         }
-        mma_commit(&bar[T_FULL + a]);
+        __syncwarp();
         return true;
       };
       bool ok = true;
       for (int k = 0; k < my_tiles && ok; ++k) {
         const int a = k & 1, s = k & 1;
-        if (!mbar_wait(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        if (!mbar_wait(&bar[STAGE_READY + s], (k >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[STAGE_READY + s], (k >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
         tc_fence_after();
         const uint32_t bh = smem_u32(smem + (F32 ? bxh_off(s) : raw_off(s)));
         const uint32_t bl = F32 ? smem_u32(smem + bxh_off(s) + bx_lo) : 0u;
         const uint32_t dhi = tbase + a * COLS, dlo = dhi + NV;
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
-          const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
-          const uint64_t db = desc_kmajor_sw128(bh + bo);
-          mma_f16_ss(dhi, desc_kmajor_sw128(a0 + ao), db, idesc, ks > 0);
-          mma_f16_ss(dlo, desc_kmajor_sw128(a1 + ao), db, idesc, ks > 0);
-          if (F32) mma_f16_ss(dlo, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bl + bo), idesc, 1);
+        if (elect_one_sync()) {
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
+            const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
+            const uint64_t db = desc_kmajor_sw128(bh + bo);
+            mma_f16_ss(dhi, desc_kmajor_sw128(a0 + ao), db, idesc, ks > 0);
+            mma_f16_ss(dlo, desc_kmajor_sw128(a1 + ao), db, idesc, ks > 0);
+            if (F32) mma_f16_ss(dlo, desc_kmajor_sw128(a0 + ao), desc_kmajor_sw128(bl + bo), idesc, 1);
+          }
+          mma_commit(&bar[STAGE_EMPTY + s]);
+          mma_commit(&bar[ACC_FULL + a]);
         }
-        mma_commit(&bar[STAGE_EMPTY + s]);
-        mma_commit(&bar[ACC_FULL + a]);
+        __syncwarp();
         if (ALG2 && k >= 1) ok = issue_T(k - 1);
       }
       if (ALG2 && ok && my_tiles >= 1 && !*abort_flag) issue_T(my_tiles - 1);

@@ -181,71 +181,78 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------ producer -------------------------------------------------
-    if (lane == 0) {
-      uint32_t jr = 0, jb = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
-        for (int s = 0; s < nsweeps && ok; ++s) {
-          const bool phase2 = s > NB;
-          const int nb = phase2 ? s - 1 - NB : s - 1;
-          for (int kb = 0; kb < KB; ++kb) {
-            if (s <= NB) {
-              const int rs = jr & 1;
-              if (!mbar_wait(&bar[RAW_EMPTY + rs], ((jr >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
-                ok = false;
-                break;
-              }
-              uint8_t* dst = smem + Lo.raw + rs * 2 * kBlk;
+    // warp-uniform schedule; one elected lane issues the copies
+    uint32_t jr = 0, jb = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
+      for (int s = 0; s < nsweeps && ok; ++s) {
+        const bool phase2 = s > NB;
+        const int nb = phase2 ? s - 1 - NB : s - 1;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (s <= NB) {
+            const int rs = jr & 1;
+            if (!mbar_wait_warp(&bar[RAW_EMPTY + rs], ((jr >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t* dst = smem + Lo.raw + rs * 2 * kBlk;
+            if (elect_one_sync()) {
               mbar_arrive_expect_tx(&bar[RAW_FULL + rs], F32 ? 2 * kBlk : kBlk);
               tma_load_2d(dst, &tmap, kb * 64, tile * 128, &bar[RAW_FULL + rs]);
               if (F32) tma_load_2d(dst + kBlk, &tmap, kb * 64 + 32, tile * 128, &bar[RAW_FULL + rs]);
-              ++jr;
             }
-            if (s >= 1) {
-              const int bs = jb & 1;
-              if (!mbar_wait(&bar[B_EMPTY + bs], ((jb >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
-                ok = false;
-                break;
-              }
-              const size_t off = (size_t)nb * p.band_bytes + (size_t)kb * kBlk;
-              uint8_t* dst = smem + Lo.b + bs * 2 * kBlk;
+            __syncwarp();
+            ++jr;
+          }
+          if (s >= 1) {
+            const int bs = jb & 1;
+            if (!mbar_wait_warp(&bar[B_EMPTY + bs], ((jb >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const size_t off = (size_t)nb * p.band_bytes + (size_t)kb * kBlk;
+            uint8_t* dst = smem + Lo.b + bs * 2 * kBlk;
+            if (elect_one_sync()) {
               mbar_arrive_expect_tx(&bar[B_FULL + bs], 2 * kBlk);
               bulk_g2s(dst, (phase2 ? p.t_hi : p.pi_hi) + off, kBlk, &bar[B_FULL + bs]);
               bulk_g2s(dst + kBlk, (phase2 ? p.t_lo : p.pi_lo) + off, kBlk, &bar[B_FULL + bs]);
-              ++jb;
             }
+            __syncwarp();
+            ++jb;
           }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer -----------------------------------------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(128, 128);
-      const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + Lo.a));
-      const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + Lo.b));
-      uint32_t ja = 0, jb = 0, jacc = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
-        for (int s = 1; s < nsweeps && ok; ++s) {
-          const bool has_lo = F32 || s > NB;        // fp32 x or the rho operand carry a low part
-          const int acc = jacc & 1;
-          if (jacc >= 2 && !mbar_wait(&bar[ACC_EMPTY + acc], ((jacc >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag)) {
+    // warp-uniform schedule (descriptors stay in uniform registers); one elected lane issues
+    const uint32_t idesc = idesc_f16_f32(128, 128);
+    const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + Lo.a));
+    const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + Lo.b));
+    uint32_t ja = 0, jb = 0, jacc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
+      for (int s = 1; s < nsweeps && ok; ++s) {
+        const bool has_lo = F32 || s > NB;        // fp32 x or the rho operand carry a low part
+        const int acc = jacc & 1;
+        if (jacc >= 2 &&
+            !mbar_wait_warp(&bar[ACC_EMPTY + acc], ((jacc >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dhi = tbase + acc * 256, dlo = dhi + 128;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int as = ja & 1, bs = jb & 1;
+          if (!mbar_wait_warp(&bar[A_FULL + as], (ja >> 1) & 1, p.err, kDevTimeoutSync, abort_flag) ||
+              !mbar_wait_warp(&bar[B_FULL + bs], (jb >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t dhi = tbase + acc * 256, dlo = dhi + 128;
-          for (int kb = 0; kb < KB; ++kb) {
-            const int as = ja & 1, bs = jb & 1;
-            if (!mbar_wait(&bar[A_FULL + as], (ja >> 1) & 1, p.err, kDevTimeoutSync, abort_flag) ||
-                !mbar_wait(&bar[B_FULL + bs], (jb >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t ah = da0 + ((as * 2 * kBlk) >> 4), al = ah + (kBlk >> 4);
-            const uint64_t bh = db0 + ((bs * 2 * kBlk) >> 4), bl = bh + (kBlk >> 4);
+          const uint64_t ah = da0 + ((as * 2 * kBlk) >> 4), al = ah + (kBlk >> 4);
+          const uint64_t bh = db0 + ((bs * 2 * kBlk) >> 4), bl = bh + (kBlk >> 4);
+          if (elect_one_sync()) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint32_t accum = (kb > 0 || ks > 0) ? 1u : 0u;
@@ -255,12 +262,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
             mma_commit(&bar[A_EMPTY + as]);
             mma_commit(&bar[B_EMPTY + bs]);
-            ++ja;
-            ++jb;
           }
-          if (ok) mma_commit(&bar[ACC_FULL + acc]);
-          ++jacc;
+          __syncwarp();
+          ++ja;
+          ++jb;
         }
+        if (ok && elect_one_sync()) mma_commit(&bar[ACC_FULL + acc]);
+        __syncwarp();
+        ++jacc;
       }
     }
   } else if (warp < 6) {

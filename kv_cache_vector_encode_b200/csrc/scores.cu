@@ -229,56 +229,61 @@ __global__ void __launch_bounds__(kScThreads, 1) scores_main_kernel(const __grid
 
   if (warp == 0) {
     // ------------------------------------ producer: B blocks ---------------------------------------
-    if (lane == 0) {
-      int64_t j = 0;                               // running block counter of this CTA
-      bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
-        const int nt = it % p.ntq;
-        const uint8_t* src = p.bimg + (size_t)nt * nblk * kBBytes;
-        for (int k = 0; k < nblk; ++k, ++j) {
-          const int slot = (int)(j % kBRing);
-          const uint32_t use = (uint32_t)(j / kBRing);
-          if (!mbar_wait(&bar[B_EMPTY + slot], (use & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
-            ok = false;
-            break;
-          }
+    // warp-uniform schedule; one elected lane issues the copies
+    int64_t j = 0;                                 // running block counter of this CTA
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int nt = it % p.ntq;
+      const uint8_t* src = p.bimg + (size_t)nt * nblk * kBBytes;
+      for (int k = 0; k < nblk; ++k, ++j) {
+        const int slot = (int)(j % kBRing);
+        const uint32_t use = (uint32_t)(j / kBRing);
+        if (!mbar_wait_warp(&bar[B_EMPTY + slot], (use & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one_sync()) {
           mbar_arrive_expect_tx(&bar[B_FULL + slot], kBBytes);
           bulk_g2s(smem + Lo.off_b + slot * kBBytes, src + (size_t)k * kBBytes, kBBytes, &bar[B_FULL + slot]);
         }
+        __syncwarp();
       }
     }
   } else if (warp == 1) {
     // ------------------------------------ MMA issuer -----------------------------------------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(128, 256);
-      const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_a));
-      const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_b));
-      int64_t j = 0;
-      int li = 0;                                  // local work-item counter
-      bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
-        const int acc = li & 1;
-        if (li >= 2 && !mbar_wait(&bar[ACC_EMPTY + acc], ((li >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+    // warp-uniform schedule (descriptors stay in uniform registers); one elected lane issues
+    const uint32_t idesc = idesc_f16_f32(128, 256);
+    const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_a));
+    const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_b));
+    int64_t j = 0;
+    int li = 0;                                    // local work-item counter
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+      const int acc = li & 1;
+      if (li >= 2 && !mbar_wait_warp(&bar[ACC_EMPTY + acc], ((li >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+        break;
+      tc_fence_after();
+      const uint32_t dcol = tbase + acc * 256;
+      for (int k = 0; k < nblk; ++k, ++j) {
+        const int as = (int)(j % kARing), bs = (int)(j % kBRing);
+        if (!mbar_wait_warp(&bar[A_FULL + as], (uint32_t)(j / kARing) & 1, p.err, kDevTimeoutSync, abort_flag) ||
+            !mbar_wait_warp(&bar[B_FULL + bs], (uint32_t)(j / kBRing) & 1, p.err, kDevTimeoutLoad, abort_flag)) {
+          ok = false;
           break;
+        }
         tc_fence_after();
-        const uint32_t dcol = tbase + acc * 256;
-        for (int k = 0; k < nblk; ++k, ++j) {
-          const int as = (int)(j % kARing), bs = (int)(j % kBRing);
-          if (!mbar_wait(&bar[A_FULL + as], (uint32_t)(j / kARing) & 1, p.err, kDevTimeoutSync, abort_flag) ||
-              !mbar_wait(&bar[B_FULL + bs], (uint32_t)(j / kBRing) & 1, p.err, kDevTimeoutLoad, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t da = da0 + ((as * kABytes) >> 4);
-          const uint64_t db = db0 + ((bs * kBBytes) >> 4);
+        const uint64_t da = da0 + ((as * kABytes) >> 4);
+        const uint64_t db = db0 + ((bs * kBBytes) >> 4);
+        if (elect_one_sync()) {
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) mma_f16_ss(dcol, da + ks * 2, db + ks * 2, idesc, (k > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar[A_EMPTY + as]);
           mma_commit(&bar[B_EMPTY + bs]);
         }
-        if (ok) mma_commit(&bar[ACC_FULL + acc]);
+        __syncwarp();
       }
+      if (ok && elect_one_sync()) mma_commit(&bar[ACC_FULL + acc]);
+      __syncwarp();
     }
   } else if (warp < 6) {
     // ------------------------------------ expanders (thread = vector) ------------------------------
