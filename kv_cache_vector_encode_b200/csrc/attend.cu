@@ -34,9 +34,10 @@
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
 // (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
-// Main-kernel roles (14 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the MMAs;
-// 2-5 softmax (thread = token); 6-9 expand K into TMEM and V into shared memory (thread = token);
-// 10-13 accumulate the value products (thread = coordinate).
+// Main-kernel roles (18 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the MMAs;
+// 2-9 softmax (thread = token; two groups of four warps, each group owning half of the query
+// heads); 10-13 expand K into TMEM and V into shared memory (thread = token); 14-17 accumulate the
+// value products (thread = coordinate).
 // All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
 // same number of times by all four warps (their loop never exits early).
 #include <cuda_fp16.h>
@@ -51,7 +52,7 @@
 namespace tq {
 namespace {
 
-constexpr int kAttThreads = 448;
+constexpr int kAttThreads = 576;                // 18 warps
 constexpr int kChunk = 128;                 // tokens per chunk
 constexpr int kMaxStages = 8;               // packed-chunk ring (depth chosen from shared memory)
 constexpr int kMaxSmem = 232448;            // 227 KB of dynamic shared memory per block
@@ -208,7 +209,7 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.bq_bytes = aru(p.nq * p.mk * p.d, 1024);
   L.off_bq = off; off += 2 * L.bq_bytes;
   L.off_sc = off; off += 4 * 64 * 4;               // chunk scalars, 4-deep ring of 64 floats
-  L.off_red = off; off += 4 * 16 * 4;              // max exchange of the softmax warps
+  L.off_red = off; off += 2 * 4 * 16 * 4;          // max exchange of the softmax warps: [group][warp][16]
   L.off_sum = off; off += 4 * 4 * 24 * 4;          // chunk sums of the weights: [ring][warp][kind][head]
   L.off_bar = aru(off, 8); off = L.off_bar + 64 * 8;
   L.total = off + 1024;
@@ -291,7 +292,7 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
 // HG: query heads per KV head (4 or 8, Hg <= HG); BK: key bits; BV: value codebook bits;
 // VS: value sign plane (Algorithm 2 values)
 template <int HG, int BK, int BV, int VS>
-__global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __grid_constant__ AttParams p) {
+__global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttParams p) {
   constexpr int MK = walsh_count(BK);
   constexpr int MV = walsh_count(BV);
   constexpr int NP = MV + VS;
@@ -330,12 +331,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       mbar_init(&bar[BQ_EMPTY + s], 1);
       mbar_init(&bar[AK_FULL + s], 4);
       mbar_init(&bar[SC_DONE + s], 1);
-      mbar_init(&bar[BW_FULL + s], 4);
+      mbar_init(&bar[BW_FULL + s], 8);
       mbar_init(&bar[AV_FULL + s], 4);
       mbar_init(&bar[V_DONE + s], 1);
       mbar_init(&bar[DV_EMPTY + s], 4);
     }
-    for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 4);
+    for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -445,13 +446,19 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       if (c >= 1) ok = issue_v(c - 1);
     }
     if (ok && nmy >= 1 && !*abort_flag) issue_v(nmy - 1);
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ------------------------------------ softmax warps (thread = token) ---------------------------
+    // group gq of four warps owns query heads [h0, h0 + HH); both groups track the same value-norm
+    // maxima (same tokens, same rule), so the fixed-point scales agree
+    constexpr int HH = HG / 2;
     const int q = warp & 3;
+    const int gq = (warp - 2) >> 2;
+    const int h0 = gq * HH;
     const int t = q * 32 + lane;                    // token inside the chunk == TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
-    float mrun[HG], ha[HG], hb[HG];
+    float* rgrp = red + gq * 64;
+    float mrun[HH], ha[HH], hb[HH];
     float vmax_run = 0.0f, gmax_run = 0.0f, sw = 1.0f, sw2 = 1.0f, isw = 1.0f, isw2 = 1.0f;
     bool ok = true;
     // fp16 norms of the next chunk, loaded one chunk ahead and converted only when used (dead
@@ -481,57 +488,58 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
         vmax_run = gmax_run = 0.0f;
         const float2* hc = (const float2*)(p.head_c + it.slice * 16);
 #pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          mrun[h] = -INFINITY;
-          const float2 x = h < Hg ? __ldg(hc + h) : make_float2(0.0f, 0.0f);
-          ha[h] = -2.0f * x.x * p.scale_log2e;
-          hb[h] = x.y * p.scale_log2e;
+        for (int i = 0; i < HH; ++i) {
+          mrun[i] = -INFINITY;
+          const float2 x = h0 + i < Hg ? __ldg(hc + h0 + i) : make_float2(0.0f, 0.0f);
+          ha[i] = -2.0f * x.x * p.scale_log2e;
+          hb[i] = x.y * p.scale_log2e;
         }
       }
       ok = mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
       tc_fence_after();
-      uint32_t dsr[NQ];
-      tmem_ld16(tbase + lane_base + kDS0 + b * NQ, *(uint32_t(*)[16]) & dsr[0]);
-      if (NQ > 16) tmem_ld16(tbase + lane_base + kDS0 + b * NQ + 16, *(uint32_t(*)[16]) & dsr[NQ > 16 ? 16 : 0]);
+      uint32_t dsr[4 * HH];
+      const uint32_t scol = tbase + lane_base + kDS0 + b * NQ + 4 * h0;
+      if (HH == 2) tmem_ld8(scol, *(uint32_t(*)[8]) & dsr[0]);
+      else tmem_ld16(scol, *(uint32_t(*)[16]) & dsr[0]);
       tmem_ld_wait();
       tc_fence_before();
-      float lg[HG];
+      float lg[HH];
       bool up = nv > vmax_run || nv * gm > gmax_run;
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
+      for (int i = 0; i < HH; ++i) {
         // the four limb products are exact integers below 2^21 in magnitude
-        const float dot = fmaf(fmaf(fmaf(small_i2f((int)dsr[4 * h + 3]), 256.0f, small_i2f((int)dsr[4 * h + 2])), 256.0f,
-                                    small_i2f((int)dsr[4 * h + 1])),
-                               256.0f, small_i2f((int)dsr[4 * h]));
-        lg[h] = (h < Hg && live) ? nk * fmaf(ha[h], dot, hb[h]) : -INFINITY;
-        up = up || lg[h] > mrun[h];
+        const float dot = fmaf(fmaf(fmaf(small_i2f((int)dsr[4 * i + 3]), 256.0f, small_i2f((int)dsr[4 * i + 2])), 256.0f,
+                                    small_i2f((int)dsr[4 * i + 1])),
+                               256.0f, small_i2f((int)dsr[4 * i]));
+        lg[i] = (h0 + i < Hg && live) ? nk * fmaf(ha[i], dot, hb[i]) : -INFINITY;
+        up = up || lg[i] > mrun[i];
       }
-      float corr[HG];
+      float corr[HH];
 #pragma unroll
-      for (int h = 0; h < HG; ++h) corr[h] = 1.0f;
-      if (bar_red_or(1, 128, up)) {
-        // some token raised a running maximum: exchange the chunk maxima of the four warps
-        float* rb = red + q * 16;
+      for (int i = 0; i < HH; ++i) corr[i] = 1.0f;
+      if (bar_red_or(1 + 2 * gq, 128, up)) {
+        // some token raised a running maximum: exchange the chunk maxima of the group's warps
+        float* rb = rgrp + q * 16;
 #pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const float v = warp_max(lg[h]);
-          if (lane == 0) rb[h] = v;
+        for (int i = 0; i < HH; ++i) {
+          const float v = warp_max(lg[i]);
+          if (lane == 0) rb[i] = v;
         }
         const float vm = warp_max(nv), gmx = warp_max(nv * gm);
         if (lane == 0) {
           rb[8] = vm;
           rb[9] = gmx;
         }
-        bar_sync_named(2, 128);
+        bar_sync_named(2 + 2 * gq, 128);
 #pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const float cm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
-          const float mn = fmaxf(mrun[h], cm);
-          corr[h] = (mn == -INFINITY) ? 1.0f : fast_exp2(mrun[h] - mn);
-          mrun[h] = mn;
+        for (int i = 0; i < HH; ++i) {
+          const float cm = fmaxf(fmaxf(rgrp[i], rgrp[16 + i]), fmaxf(rgrp[32 + i], rgrp[48 + i]));
+          const float mn = fmaxf(mrun[i], cm);
+          corr[i] = (mn == -INFINITY) ? 1.0f : fast_exp2(mrun[i] - mn);
+          mrun[i] = mn;
         }
-        vmax_run = fmaxf(vmax_run, fmaxf(fmaxf(red[8], red[24]), fmaxf(red[40], red[56])));
-        gmax_run = fmaxf(gmax_run, fmaxf(fmaxf(red[9], red[25]), fmaxf(red[41], red[57])));
+        vmax_run = fmaxf(vmax_run, fmaxf(fmaxf(rgrp[8], rgrp[24]), fmaxf(rgrp[40], rgrp[56])));
+        gmax_run = fmaxf(gmax_run, fmaxf(fmaxf(rgrp[9], rgrp[25]), fmaxf(rgrp[41], rgrp[57])));
         int E1 = 0, E2 = 0;
         frexpf(fmaxf(vmax_run, 1e-30f), &E1);
         frexpf(fmaxf(gmax_run, 1e-30f), &E2);
@@ -543,49 +551,50 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
         isw2 = ldexpf(1.0f, E2 - 23);
       }
       // weights: p = 2^(lg - m) <= 1, w = p |v|, w' = w gamma, as 24-bit unsigned fixed point
-      uint32_t wv[HG], wz[HG], pv[HG];
+      uint32_t wv[HH], wz[HH], pv[HH];
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float pr = (lg[h] == -INFINITY) ? 0.0f : fast_exp2(lg[h] - mrun[h]);
+      for (int i = 0; i < HH; ++i) {
+        const float pr = (lg[i] == -INFINITY) ? 0.0f : fast_exp2(lg[i] - mrun[i]);
         const float w = pr * nv;
-        wv[h] = fixed24(w, sw);
-        wz[h] = VS ? fixed24(w * gm, sw2) : 0u;
-        pv[h] = fixed24(pr, 4194304.0f);            // p * 2^22
+        wv[i] = fixed24(w, sw);
+        wz[i] = VS ? fixed24(w * gm, sw2) : 0u;
+        pv[i] = fixed24(pr, 4194304.0f);            // p * 2^22
       }
       // chunk sums of each weight kind per head (exact: 32 values below 2^24 per warp)
-      uint32_t* su = sums + ((c & 3) * 4 + q) * 24;
+      uint32_t* su = sums + ((c & 3) * 4 + q) * 24 + h0;
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const uint32_t s0 = warp_sum_u32(wv[h]);
-        const uint32_t s1 = VS ? warp_sum_u32(wz[h]) : 0u;
-        const uint32_t s2 = warp_sum_u32(pv[h]);
+      for (int i = 0; i < HH; ++i) {
+        const uint32_t s0 = warp_sum_u32(wv[i]);
+        const uint32_t s1 = VS ? warp_sum_u32(wz[i]) : 0u;
+        const uint32_t s2 = warp_sum_u32(pv[i]);
         if (lane == 0) {
-          su[h] = s0;
-          su[8 + h] = s1;
-          su[16 + h] = s2;
+          su[i] = s0;
+          su[8 + i] = s1;
+          su[16 + i] = s2;
         }
       }
       // the weight tiles of chunk c-2 (same buffer) must have been consumed by its value MMA
       if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
-      uint8_t* bwb = smem + Lo.off_bw + b * Lo.bw_buf + t * 16;
-#pragma unroll
-      for (int blk = 0; blk < NBLK; ++blk) {
-        *(uint4*)(bwb + blk * kChunk * 16) = make_uint4(wv[4 * blk], wv[4 * blk + 1], wv[4 * blk + 2], wv[4 * blk + 3]);
+      // this group's heads fill 4 HH bytes of the token's row (block h0 / 4, byte 4 (h0 % 4))
+      uint8_t* bwb = smem + Lo.off_bw + b * Lo.bw_buf + (h0 >> 2) * kChunk * 16 + t * 16 + (h0 & 3) * 4;
+      if (HH == 2) {
+        *(uint2*)bwb = make_uint2(wv[0], wv[HH > 1 ? 1 : 0]);
+        if (VS) *(uint2*)(bwb + Lo.bw_kind) = make_uint2(wz[0], wz[HH > 1 ? 1 : 0]);
+      } else {
+        *(uint4*)bwb = make_uint4(wv[0], wv[HH > 1 ? 1 : 0], wv[HH > 2 ? 2 : 0], wv[HH > 3 ? 3 : 0]);
         if (VS)
-          *(uint4*)(bwb + Lo.bw_kind + blk * kChunk * 16) =
-              make_uint4(wz[4 * blk], wz[4 * blk + 1], wz[4 * blk + 2], wz[4 * blk + 3]);
+          *(uint4*)(bwb + Lo.bw_kind) = make_uint4(wz[0], wz[HH > 1 ? 1 : 0], wz[HH > 2 ? 2 : 0], wz[HH > 3 ? 3 : 0]);
       }
       fence_proxy_async_smem();
-      if (warp == 2) {
+      if (q == 0 && lane == 0) {
         // chunk scalars for the accumulators (4-deep ring): rescale factors, running maxima, scales
         float* sc = scal + (c & 3) * 64;
 #pragma unroll
-        for (int h = 0; h < HG; ++h)
-          if (lane == h) {
-            sc[h] = corr[h];
-            sc[16 + h] = mrun[h];
-          }
-        if (lane == 0) {
+        for (int i = 0; i < HH; ++i) {
+          sc[h0 + i] = corr[i];
+          sc[16 + h0 + i] = mrun[i];
+        }
+        if (gq == 0) {
           sc[32] = isw;
           sc[33] = isw2;
         }
@@ -597,7 +606,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_main_kernel(const __gri
       }
     }
     (void)ok;
-  } else if (warp < 10) {
+  } else if (warp < 14) {
     // ------------------------------------ expanders (thread = token) -------------------------------
     const int q = warp & 3;
     const int t = q * 32 + lane;
