@@ -10,7 +10,9 @@
 //   D1a = PiT_hi c_hi,  D1b = PiT_lo c_hi + PiT_hi c_lo,  D2a = ST_hi s,  D2b = ST_lo s
 //   x_hat = n ((D1a + 2^-12 D1b) + alpha gamma (D2a + 2^-12 D2b))
 // Roles (14 warps): warp 0 bulk-copies the resident operands; warp 1 owns TMEM and issues MMAs;
-// warps 2-5 unpack (one thread per (vector, 32-coordinate group), 16-byte swizzled stores);
+// warps 2-5 unpack (one thread per (vector, 32-coordinate group): the symmetric codebook's fp16
+// magnitudes picked by byte permutes, the sign from the top bit; 16-byte swizzled stores into a
+// double-buffered operand);
 // warps 6-13 are the epilogue (two warps per TMEM lane quarter). All waits are bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -37,16 +39,29 @@ struct DecodeParams {
   const uint16_t* gammas;
   void* out;
   float alpha;
-  uint32_t lut_hi[8], lut_lo[8];   // c_hi / c_lo (fp16) of the 16 levels, two per word
+  uint32_t mag_hi[4], mag_lo[4];   // fp16 hi / lo parts of the positive levels c[L/2 + m], two per word
   uint32_t* err;
 };
 
 struct DecLayout {
   uint32_t a_bytes, b_bytes;
-  uint32_t off_a[4], off_b[3], off_info, off_bar, total;
+  uint32_t off_a[4], off_b[3], b_set, off_info, off_bar, total;   // buffer s of B plane i: off_b[i] + s * b_set
 };
 
 __host__ __device__ inline uint32_t dround(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// fp16 magnitudes of levels ma (low half) and mb (high half) of a symmetric codebook with H positive
+// levels, by byte permutes over the table t0..t3 (entry m in bytes 2m, 2m + 1).
+template <int H>
+__device__ __forceinline__ uint32_t mag2(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3, uint32_t ma,
+                                         uint32_t mb) {
+  if (H == 1) return (t0 & 0xFFFFu) | (t0 << 16);
+  const uint32_t sel = ((ma & 3u) * 0x22u + 0x10u) | (((mb & 3u) * 0x22u + 0x10u) << 8);
+  const uint32_t r0 = __byte_perm(t0, t1, sel);
+  if (H <= 4) return r0;
+  const uint32_t r1 = __byte_perm(t2, t3, sel);
+  return __byte_perm(r0, r1, 0x3210u | ((ma & 4u) * 0x11u) | ((mb & 4u) * 0x1100u));
+}
 
 template <bool ALG2>
 __host__ __device__ inline DecLayout dec_layout(int KP, int NV) {
@@ -56,13 +71,15 @@ __host__ __device__ inline DecLayout dec_layout(int KP, int NV) {
   uint32_t off = 0;
   for (int i = 0; i < (ALG2 ? 4 : 2); ++i) { L.off_a[i] = off; off += L.a_bytes; }
   for (int i = 0; i < (ALG2 ? 3 : 2); ++i) { L.off_b[i] = off; off += L.b_bytes; }
+  L.b_set = (ALG2 ? 3 : 2) * L.b_bytes;
+  off += L.b_set;
   L.off_info = off; off += 2u * 2 * NV * 4;     // [2 buffers][norm, alpha*gamma][NV]
   L.off_bar = dround(off, 8); off = L.off_bar + 16 * 8;
   L.total = off + 1024;
   return L;
 }
 
-enum DBars { A_FULL = 0, B_FULL = 1, B_EMPTY = 2, ACC_FULL = 3, ACC_EMPTY = 5, INFO_EMPTY = 7, DNBARS = 9 };
+enum DBars { A_FULL = 0, B_FULL = 1, B_EMPTY = 3, ACC_FULL = 5, ACC_EMPTY = 7, INFO_EMPTY = 9, DNBARS = 11 };
 
 __device__ __forceinline__ uint32_t pack_h2(uint32_t a, uint32_t b) { return (a & 0xFFFFu) | (b << 16); }
 
@@ -83,9 +100,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 
   if (tid == 0) {
     mbar_init(&bar[A_FULL], 1);
-    mbar_init(&bar[B_FULL], 4);                // one arrival per unpacker warp
-    mbar_init(&bar[B_EMPTY], 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_FULL + s], 4);          // one arrival per unpacker warp
+      mbar_init(&bar[B_EMPTY + s], 1);
       mbar_init(&bar[ACC_FULL + s], 1);
       mbar_init(&bar[ACC_EMPTY + s], 8);       // one arrival per epilogue warp
       mbar_init(&bar[INFO_EMPTY + s], 8);
@@ -115,14 +132,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
-      const uint32_t bch = smem_u32(smem + Lo.off_b[0]), bcl = smem_u32(smem + Lo.off_b[1]);
-      const uint32_t bs = ALG2 ? smem_u32(smem + Lo.off_b[2]) : 0u;
+
       const int ksteps = KP / 16;
       for (int k = 0; k < my_tiles; ++k) {
         const int a = k & 1;
         if (!mbar_wait_warp(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
-        if (!mbar_wait_warp(&bar[B_FULL], k & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+        if (!mbar_wait_warp(&bar[B_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
         tc_fence_after();
+        const uint32_t bch = smem_u32(smem + Lo.off_b[0] + a * Lo.b_set), bcl = bch + Lo.b_bytes;
+        const uint32_t bs = ALG2 ? bch + 2 * Lo.b_bytes : 0u;
         const uint32_t d1a = tbase + a * COLS, d1b = d1a + NV, d2a = d1a + 2 * NV, d2b = d1a + 3 * NV;
         if (elect_one_sync()) {
           for (int ks = 0; ks < ksteps; ++ks) {
@@ -138,7 +156,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
               mma_f16_ss(d2b, desc_kmajor_sw128(a3 + ao), dsg, idesc, ks > 0);
             }
           }
-          mma_commit(&bar[B_EMPTY]);
+          mma_commit(&bar[B_EMPTY + a]);
           mma_commit(&bar[ACC_FULL + a]);
         }
         __syncwarp();
@@ -147,22 +165,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   } else if (warp < 6) {
     // ---------------- unpackers: codes -> fp16 B operands -----------------------------------------
     const int ut = tid - 64;               // 0..127
-    uint32_t lhi[8], llo[8];
+    constexpr int H = 1 << (BITS - 1);
+    uint32_t th[4], tl[4];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      lhi[h] = p.lut_hi[h];
-      llo[h] = p.lut_lo[h];
+    for (int k = 0; k < 4; ++k) {
+      th[k] = p.mag_hi[k];
+      tl[k] = p.mag_lo[k];
     }
-    // 16-entry fp16 table held as 8 words; entry idx = half (idx & 1) of word idx >> 1
-    auto lut = [](const uint32_t (&t)[8], int idx) -> uint32_t {
-      uint32_t w = t[0];
-#pragma unroll
-      for (int h = 1; h < (1 << BITS) / 2; ++h) w = (idx >> 1) == h ? t[h] : w;
-      return (idx & 1) ? (w >> 16) : (w & 0xFFFFu);
-    };
-    uint8_t* bch = smem + Lo.off_b[0];
-    uint8_t* bcl = smem + Lo.off_b[1];
-    uint8_t* bsg = ALG2 ? smem + Lo.off_b[2] : nullptr;
     const int gp = KP / 32;                  // groups per operand row (padding groups included)
     const int units = NV * gp;
     for (int k = 0; k < my_tiles; ++k) {
@@ -179,7 +188,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         info[(a * 2 + 0) * NV + ut] = nv;
         info[(a * 2 + 1) * NV + ut] = ag;
       }
-      if (!mbar_wait_warp(&bar[B_EMPTY], (k & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[B_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      uint8_t* bch = smem + Lo.off_b[0] + a * Lo.b_set;
+      uint8_t* bcl = bch + Lo.b_bytes;
+      uint8_t* bsg = ALG2 ? bch + 2 * Lo.b_bytes : nullptr;
       for (int u = ut; u < units; u += 128) {
         const int v = u / gp, g = u % gp;
         const bool live = v < rows && g < G;
@@ -187,25 +199,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
         for (int pl = 0; pl < BITS; ++pl) w[pl] = live ? __ldg(p.codes + ((v0 + v) * G + g) * BITS + pl) : 0u;
         if (ALG2) sg = live ? __ldg(p.signs + (v0 + v) * G + g) : 0u;
+        // symmetric codebook: neg = !top bit, magnitude index m = low bits ^ (neg ? H-1 : 0)
+        const uint32_t negw = live ? ~w[BITS - 1] : 0u;
+        uint32_t mp[BITS > 1 ? BITS - 1 : 1];
+#pragma unroll
+        for (int pl = 0; pl < BITS - 1; ++pl) mp[pl] = w[pl] ^ negw;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {           // four 8-coordinate chunks of the group
           uint32_t hi4[4], lo4[4], s4[4];
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            uint32_t hv[2], lv[2], sv[2];
+            const int bit = 8 * c + 2 * h;       // elements bit, bit + 1 -> low, high half
+            uint32_t ma = 0, mb = 0;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int bit = 8 * c + 2 * h + e;
-              int idx = 0;
-#pragma unroll
-              for (int pl = 0; pl < BITS; ++pl) idx |= (int)((w[pl] >> bit) & 1u) << pl;
-              hv[e] = live ? lut(lhi, idx) : 0u;
-              lv[e] = live ? lut(llo, idx) : 0u;
-              sv[e] = live ? (((sg >> bit) & 1u) ? 0x3C00u : 0xBC00u) : 0u;
+            for (int pl = 0; pl < BITS - 1; ++pl) {
+              ma |= ((mp[pl] >> bit) & 1u) << pl;
+              mb |= ((mp[pl] >> (bit + 1)) & 1u) << pl;
             }
-            hi4[h] = pack_h2(hv[0], hv[1]);
-            lo4[h] = pack_h2(lv[0], lv[1]);
-            s4[h] = pack_h2(sv[0], sv[1]);
+            const uint32_t ng = (negw >> bit) & 3u;
+            const uint32_t sgnbits = ((ng & 1u) << 15) | ((ng & 2u) << 30);
+            hi4[h] = live ? (mag2<H>(th[0], th[1], th[2], th[3], ma, mb) | sgnbits) : 0u;
+            lo4[h] = live ? (mag2<H>(tl[0], tl[1], tl[2], tl[3], ma, mb) | sgnbits) : 0u;
+            if (ALG2) {
+              const uint32_t zn = (~sg >> bit) & 3u;          // z = 0 -> -1
+              s4[h] = live ? (0x3C003C00u | ((zn & 1u) << 15) | ((zn & 2u) << 30)) : 0u;
+            }
           }
           const uint32_t off = sw128_offset(v, (g * 32 + c * 8) * 2, NV);
           *(uint4*)(bch + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
@@ -215,7 +233,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_FULL]);
+      if (lane == 0) mbar_arrive(&bar[B_FULL + a]);
     }
   } else {
     // ---------------- epilogue ----------------------------------------------------------------------
@@ -340,17 +358,20 @@ extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t 
   p.gammas = gammas;
   p.out = out;
   p.alpha = (float)(std::sqrt(M_PI / 2.0) / d);
-  uint16_t hi[16], lo[16];
-  for (int k = 0; k < 16; ++k) {
-    float c = k < cb->levels ? cb->c[k] : 0.0f;
-    __half h = __float2half_rn(c);
-    __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
-    hi[k] = __half_as_ushort(h);
-    lo[k] = __half_as_ushort(l);
+  const int L = cb->levels, H = L / 2;
+  for (int k = 0; k < L; ++k)
+    if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, "tq_decode: codebook is not symmetric");
+  uint16_t hi[8] = {}, lo[8] = {};
+  for (int m = 0; m < H; ++m) {
+    const float c = cb->c[H + m];
+    const __half h = __float2half_rn(c);
+    const __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
+    hi[m] = __half_as_ushort(h);
+    lo[m] = __half_as_ushort(l);
   }
-  for (int k = 0; k < 8; ++k) {
-    p.lut_hi[k] = (uint32_t)hi[2 * k] | ((uint32_t)hi[2 * k + 1] << 16);
-    p.lut_lo[k] = (uint32_t)lo[2 * k] | ((uint32_t)lo[2 * k + 1] << 16);
+  for (int k = 0; k < 4; ++k) {
+    p.mag_hi[k] = (uint32_t)hi[2 * k] | ((uint32_t)hi[2 * k + 1] << 16);
+    p.mag_lo[k] = (uint32_t)lo[2 * k] | ((uint32_t)lo[2 * k + 1] << 16);
   }
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, "tq_decode: no device error word (is a CUDA device present?)");
