@@ -202,7 +202,7 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   uint32_t off = 0;
   L.off_stage = off; off += nst * L.stage_bytes;
   L.av_bytes = kChunk * 128;                       // one plane: 128 tokens x 128 coordinates
-  L.off_av = off; off += 2 * p.np * L.av_bytes;
+  L.off_av = off; off += 3 * p.np * L.av_bytes;     // three chunks of value planes
   L.bw_kind = (p.nq / 16) * kChunk * 16;           // one weight kind: nq/16 blocks of 128 x 16 bytes
   L.bw_buf = 2 * L.bw_kind;                        // kinds: w, w * gamma
   L.off_bw = off; off += 2 * L.bw_buf;
@@ -221,12 +221,11 @@ enum ABars {
   ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (expander warps: 4)
   BQ_FULL = ST_EMPTY + kMaxStages,     // [2]
   BQ_EMPTY = BQ_FULL + 2,              // [2]
-  AK_FULL = BQ_EMPTY + 2,              // [2]  expanders -> MMA (4 warps)
-  SC_DONE = AK_FULL + 2,               // [2]  scores MMA complete (commit)
-  BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA (4 warps)
-  AV_FULL = BW_FULL + 2,               // [2]  expanders -> MMA (4 warps)
-  V_DONE = AV_FULL + 2,                // [2]  value MMA complete (commit)
-  DV_EMPTY = V_DONE + 2,               // [2]  accumulators -> MMA (4 warps)
+  KV_FULL = BQ_EMPTY + 2,              // [2]  expanders -> MMA: key and value planes of a chunk (4 warps)
+  SC_DONE = KV_FULL + 2,               // [2]  scores MMA complete (commit)
+  BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA (8 warps)
+  V_DONE = BW_FULL + 2,                // [6]  value MMA of chunk c complete (commit), slot c % 6
+  DV_EMPTY = V_DONE + 6,               // [2]  accumulators -> MMA (4 warps)
   SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (4 warps)
   ANBARS = SCAL_FULL + 4
 };
@@ -329,13 +328,12 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
       mbar_init(&bar[BQ_EMPTY + s], 1);
-      mbar_init(&bar[AK_FULL + s], 4);
+      mbar_init(&bar[KV_FULL + s], 4);
       mbar_init(&bar[SC_DONE + s], 1);
       mbar_init(&bar[BW_FULL + s], 8);
-      mbar_init(&bar[AV_FULL + s], 4);
-      mbar_init(&bar[V_DONE + s], 1);
       mbar_init(&bar[DV_EMPTY + s], 4);
     }
+    for (int s = 0; s < 6; ++s) mbar_init(&bar[V_DONE + s], 1);
     for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 8);
     *abort_flag = 0;
     fence_mbar_init();
@@ -393,15 +391,15 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
     const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_bq));
     const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
     const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
+    // the value planes of chunk c were seen complete with its key planes (KV_FULL) one iteration earlier
     auto issue_v = [&](int c) -> bool {
       const int b = c & 1;
       if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
-      if (!mbar_wait_warp(&bar[AV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
       if (c >= 2 && !mbar_wait_warp(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
         return false;
       tc_fence_after();
       const uint32_t dcol = tbase + dv0 + b * dv_cols;
-      const uint64_t da = da0 + ((b * NP * Lo.av_bytes) >> 4);
+      const uint64_t da = da0 + (((c % 3) * NP * Lo.av_bytes) >> 4);
       const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
       if (elect_one_sync()) {
 #pragma unroll
@@ -412,7 +410,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
             mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
                       db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
         }
-        mma_commit(&bar[V_DONE + b]);
+        mma_commit(&bar[V_DONE + c % 6]);
       }
       __syncwarp();
       return true;
@@ -424,10 +422,9 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
       if (c == 0 || it.cis == 0) {
         if (!mbar_wait_warp(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
       }
-      if (!mbar_wait_warp(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      // the scores buffer b is free once the softmax warps finished chunk c-2 (BW_FULL)
-      if (c >= 2 && !mbar_wait_warp(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag))
-        break;
+      if (!mbar_wait_warp(&bar[KV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      // the scores buffer b is free once the softmax warps finished chunk c-2: this warp saw BW_FULL
+      // of chunk c-2 before issuing its value MMAs in the previous iteration
       tc_fence_after();
       const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
       const uint32_t ak = tbase + kAK0 + b * 128;
@@ -574,7 +571,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         }
       }
       // the weight tiles of chunk c-2 (same buffer) must have been consumed by its value MMA
-      if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
+      if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + (c - 2) % 6], ((c - 2) / 6) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
       // this group's heads fill 4 HH bytes of the token's row (block h0 / 4, byte 4 (h0 % 4))
       uint8_t* bwb = smem + Lo.off_bw + b * Lo.bw_buf + (h0 >> 2) * kChunk * 16 + t * 16 + (h0 & 3) * 4;
       if (HH == 2) {
@@ -650,8 +647,10 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
           tmem_st8(ak + S * 32 + g * 8, r);
         }
       }
-      // values: plane words (and sign words) -> expanded bytes, one token row per plane
-      if (c >= 2 && !mbar_wait_warp(&bar[V_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
+      // values: plane words (and sign words) -> expanded bytes, one token row per plane; the
+      // planes of chunk c - 3 (same buffer) must have been consumed
+      const int c3 = c % 3;
+      if (c >= 3 && !mbar_wait_warp(&bar[V_DONE + (c - 3) % 6], ((c - 3) / 6) & 1, p.err, kDevTimeoutMma, abort_flag))
         break;
       uint32_t vw[4 * BV];
 #pragma unroll
@@ -670,7 +669,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         sg[2] = x.z;
         sg[3] = x.w;
       }
-      uint8_t* avb = smem + Lo.off_av + b * NP * Lo.av_bytes;
+      uint8_t* avb = smem + Lo.off_av + c3 * NP * Lo.av_bytes;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
 #pragma unroll
@@ -688,8 +687,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar[AK_FULL + b]);
-        mbar_arrive(&bar[AV_FULL + b]);
+        mbar_arrive(&bar[KV_FULL + b]);
         mbar_arrive(&bar[ST_EMPTY + st]);
       }
     }
@@ -716,7 +714,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         }
       }
       if (!mbar_wait_warp(&bar[SCAL_FULL + (c & 3)], (c >> 2) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      if (!mbar_wait_warp(&bar[V_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[V_DONE + c % 6], (c / 6) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
       tc_fence_after();
       const uint32_t col = tbase + lane_base + dv0 + b * dv_cols;
       uint32_t dv[NP][NQ];
