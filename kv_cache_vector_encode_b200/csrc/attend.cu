@@ -34,10 +34,10 @@
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
 // (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
-// Main-kernel roles (18 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the MMAs;
+// Main-kernel roles (19 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the key MMAs;
 // 2-9 softmax (thread = token; two groups of four warps, each group owning half of the query
 // heads); 10-13 expand K into TMEM and V into shared memory (thread = token); 14-17 accumulate the
-// value products (thread = coordinate).
+// value products (thread = coordinate); 18 issues the value MMAs.
 // All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
 // same number of times by all four warps (their loop never exits early).
 #include <cuda_fp16.h>
@@ -52,7 +52,7 @@
 namespace tq {
 namespace {
 
-constexpr int kAttThreads = 576;                // 18 warps
+constexpr int kAttThreads = 608;                // 19 warps
 constexpr int kChunk = 128;                 // tokens per chunk
 constexpr int kMaxStages = 8;               // packed-chunk ring (depth chosen from shared memory)
 constexpr int kMaxSmem = 232448;            // 227 KB of dynamic shared memory per block
@@ -221,11 +221,12 @@ enum ABars {
   ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (expander warps: 4)
   BQ_FULL = ST_EMPTY + kMaxStages,     // [2]
   BQ_EMPTY = BQ_FULL + 2,              // [2]
-  KV_FULL = BQ_EMPTY + 2,              // [2]  expanders -> MMA: key and value planes of a chunk (4 warps)
-  SC_DONE = KV_FULL + 2,               // [2]  scores MMA complete (commit)
-  BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA (8 warps)
-  V_DONE = BW_FULL + 2,                // [6]  value MMA of chunk c complete (commit), slot c % 6
-  DV_EMPTY = V_DONE + 6,               // [2]  accumulators -> MMA (4 warps)
+  AK_FULL = BQ_EMPTY + 2,              // [2]  expanders -> key MMA warp: key planes in TMEM (4 warps)
+  SC_DONE = AK_FULL + 2,               // [2]  scores MMA complete (commit)
+  BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA warps (8 warps)
+  AV_FULL = BW_FULL + 2,               // [3]  expanders -> value MMA warp: value planes (4 warps)
+  V_DONE = AV_FULL + 3,                // [6]  value MMA of chunk c complete (commit), slot c % 6
+  DV_EMPTY = V_DONE + 6,               // [2]  accumulators -> value MMA warp (4 warps)
   SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (4 warps)
   ANBARS = SCAL_FULL + 4
 };
@@ -328,11 +329,12 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
       mbar_init(&bar[BQ_EMPTY + s], 1);
-      mbar_init(&bar[KV_FULL + s], 4);
+      mbar_init(&bar[AK_FULL + s], 4);
       mbar_init(&bar[SC_DONE + s], 1);
       mbar_init(&bar[BW_FULL + s], 8);
       mbar_init(&bar[DV_EMPTY + s], 4);
     }
+    for (int s = 0; s < 3; ++s) mbar_init(&bar[AV_FULL + s], 4);
     for (int s = 0; s < 6; ++s) mbar_init(&bar[V_DONE + s], 1);
     for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 8);
     *abort_flag = 0;
@@ -382,49 +384,22 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
       __syncwarp();
     }
   } else if (warp == 1) {
-    // ------------------------------------ MMA issuer -----------------------------------------------
+    // ------------------------------------ key MMA issuer ------------------------------------------
     // The whole warp walks the schedule (its values are warp-uniform and stay in uniform
     // registers); one elected lane issues each group of tcgen05 instructions and their commits.
     const uint32_t id_s = idesc_i8_s32(128, NQ, false, true, false, false);
-    const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
-    // descriptors at the start of each buffer; offsets below are added in 16-byte units
+    // descriptor at the start of the query images; offsets below are added in 16-byte units
     const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + Lo.off_bq));
-    const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
-    const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
-    // the value planes of chunk c were seen complete with its key planes (KV_FULL) one iteration earlier
-    auto issue_v = [&](int c) -> bool {
-      const int b = c & 1;
-      if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
-      if (c >= 2 && !mbar_wait_warp(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
-        return false;
-      tc_fence_after();
-      const uint32_t dcol = tbase + dv0 + b * dv_cols;
-      const uint64_t da = da0 + (((c % 3) * NP * Lo.av_bytes) >> 4);
-      const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
-      if (elect_one_sync()) {
-#pragma unroll
-        for (int P = 0; P < NP; ++P) {
-          const bool sgn = VS && P == NP - 1;
-#pragma unroll
-          for (int ks = 0; ks < kChunk / 32; ++ks)
-            mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
-                      db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
-        }
-        mma_commit(&bar[V_DONE + c % 6]);
-      }
-      __syncwarp();
-      return true;
-    };
-    bool ok = true;
-    for (int c = 0; c < nmy && ok; ++c, it.next()) {
+    for (int c = 0; c < nmy; ++c, it.next()) {
       const int b = c & 1;
       const int sg = it.seg;
       if (c == 0 || it.cis == 0) {
         if (!mbar_wait_warp(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
       }
-      if (!mbar_wait_warp(&bar[KV_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      // the scores buffer b is free once the softmax warps finished chunk c-2: this warp saw BW_FULL
-      // of chunk c-2 before issuing its value MMAs in the previous iteration
+      if (!mbar_wait_warp(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      // the scores buffer b is free once the softmax warps finished chunk c-2
+      if (c >= 2 && !mbar_wait_warp(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+        break;
       tc_fence_after();
       const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
       const uint32_t ak = tbase + kAK0 + b * 128;
@@ -440,9 +415,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         if (last) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
       }
       __syncwarp();
-      if (c >= 1) ok = issue_v(c - 1);
     }
-    if (ok && nmy >= 1 && !*abort_flag) issue_v(nmy - 1);
   } else if (warp < 10) {
     // ------------------------------------ softmax warps (thread = token) ---------------------------
     // group gq of four warps owns query heads [h0, h0 + HH); both groups track the same value-norm
@@ -647,6 +620,11 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
           tmem_st8(ak + S * 32 + g * 8, r);
         }
       }
+      // the key planes are complete once this warp's TMEM stores are
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[AK_FULL + b]);
       // values: plane words (and sign words) -> expanded bytes, one token row per plane; the
       // planes of chunk c - 3 (same buffer) must have been consumed
       const int c3 = c % 3;
@@ -682,16 +660,14 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
               make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar[KV_FULL + b]);
+        mbar_arrive(&bar[AV_FULL + c3]);
         mbar_arrive(&bar[ST_EMPTY + st]);
       }
     }
-  } else {
+  } else if (warp < 18) {
     // ------------------------------------ accumulators (thread = coordinate row) -------------------
     const int q = warp & 3;
     const int m = q * 32 + lane;                 // TMEM lane = M index of the value MMA
@@ -779,6 +755,36 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
           }
         }
       }
+    }
+  } else {
+    // ------------------------------------ value MMA issuer (warp 18) ------------------------------
+    // Runs beside the key MMA warp so that neither warp's barrier waits and commits sit behind the
+    // other's tensor-core work. Warp-uniform schedule, one elected lane issues.
+    const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
+    const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
+    const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
+    for (int c = 0; c < nmy; ++c) {
+      const int b = c & 1, c3 = c % 3;
+      if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      if (!mbar_wait_warp(&bar[AV_FULL + c3], (c / 3) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      if (c >= 2 && !mbar_wait_warp(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+        break;
+      tc_fence_after();
+      const uint32_t dcol = tbase + dv0 + b * dv_cols;
+      const uint64_t da = da0 + ((c3 * NP * Lo.av_bytes) >> 4);
+      const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
+      if (elect_one_sync()) {
+#pragma unroll
+        for (int P = 0; P < NP; ++P) {
+          const bool sgn = VS && P == NP - 1;
+#pragma unroll
+          for (int ks = 0; ks < kChunk / 32; ++ks)
+            mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
+                      db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
+        }
+        mma_commit(&bar[V_DONE + c % 6]);
+      }
+      __syncwarp();
     }
   }
 
