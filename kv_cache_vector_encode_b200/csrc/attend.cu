@@ -297,7 +297,6 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
   constexpr int MV = walsh_count(BV);
   constexpr int NP = MV + VS;
   constexpr int NQ = HG <= 4 ? 16 : 32;
-  constexpr int NBLK = NQ / 16;
   constexpr int KSTEPS = MK * 128 / 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);

@@ -81,8 +81,6 @@ __host__ __device__ inline DecLayout dec_layout(int KP, int NV) {
 
 enum DBars { A_FULL = 0, B_FULL = 1, B_EMPTY = 3, ACC_FULL = 5, ACC_EMPTY = 7, INFO_EMPTY = 9, DNBARS = 11 };
 
-__device__ __forceinline__ uint32_t pack_h2(uint32_t a, uint32_t b) { return (a & 0xFFFFu) | (b << 16); }
-
 template <bool ALG2, int NV, bool OUT_BF16, int BITS>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;
