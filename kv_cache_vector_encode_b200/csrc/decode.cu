@@ -172,31 +172,53 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     const int gp = KP / 32;                  // groups per operand row (padding groups included)
     const int units = NV * gp;
+    constexpr int UPT = NV * 4 / 128;        // units per thread (gp <= 4)
+    // The code words of a tile are fetched one tile ahead, all loads of a tile issued together,
+    // so the unpack does not wait on one global load after another.
+    uint32_t cw[UPT][BITS], cs[UPT];
+    uint16_t cn = 0, cg = 0;
+    auto fetch = [&](int k, uint32_t (&W)[UPT][BITS], uint32_t (&SGW)[UPT], uint16_t& nn, uint16_t& gg) {
+      const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
+      const int rows = (int)min((int64_t)NV, p.n - v0);
+#pragma unroll
+      for (int j = 0; j < UPT; ++j) {
+        const int u = ut + 128 * j, v = u / gp, g = u % gp;
+        const bool live = u < units && v < rows && g < G;
+#pragma unroll
+        for (int pl = 0; pl < BITS; ++pl) W[j][pl] = live ? __ldg(p.codes + ((v0 + v) * G + g) * BITS + pl) : 0u;
+        SGW[j] = (ALG2 && live) ? __ldg(p.signs + (v0 + v) * G + g) : 0u;
+      }
+      nn = gg = 0;
+      if (ut < rows) {
+        nn = __ldg(p.norms + v0 + ut);
+        if (ALG2) gg = __ldg(p.gammas + v0 + ut);
+      }
+    };
+    if (my_tiles > 0) fetch(0, cw, cs, cn, cg);
     for (int k = 0; k < my_tiles; ++k) {
       const int a = k & 1;
       const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
+      uint32_t nw[UPT][BITS], ns[UPT];
+      uint16_t nn = 0, ngm = 0;
+      if (k + 1 < my_tiles) fetch(k + 1, nw, ns, nn, ngm);
       if (!mbar_wait_warp(&bar[INFO_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
       if (ut < NV) {
-        float nv = 0.0f, ag = 0.0f;
-        if (ut < rows) {
-          nv = __half2float(__ushort_as_half(p.norms[v0 + ut]));
-          if (ALG2) ag = p.alpha * __half2float(__ushort_as_half(p.gammas[v0 + ut]));
-        }
-        info[(a * 2 + 0) * NV + ut] = nv;
-        info[(a * 2 + 1) * NV + ut] = ag;
+        info[(a * 2 + 0) * NV + ut] = __half2float(__ushort_as_half(cn));
+        info[(a * 2 + 1) * NV + ut] = ALG2 ? p.alpha * __half2float(__ushort_as_half(cg)) : 0.0f;
       }
       if (!mbar_wait_warp(&bar[B_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
       uint8_t* bch = smem + Lo.off_b[0] + a * Lo.b_set;
       uint8_t* bcl = bch + Lo.b_bytes;
       uint8_t* bsg = ALG2 ? bch + 2 * Lo.b_bytes : nullptr;
-      for (int u = ut; u < units; u += 128) {
+#pragma unroll
+      for (int j = 0; j < UPT; ++j) {
+        const int u = ut + 128 * j;
+        if (u >= units) break;
         const int v = u / gp, g = u % gp;
         const bool live = v < rows && g < G;
-        uint32_t w[BITS], sg = 0;
-#pragma unroll
-        for (int pl = 0; pl < BITS; ++pl) w[pl] = live ? __ldg(p.codes + ((v0 + v) * G + g) * BITS + pl) : 0u;
-        if (ALG2) sg = live ? __ldg(p.signs + (v0 + v) * G + g) : 0u;
+        const uint32_t* w = cw[j];
+        const uint32_t sg = cs[j];
         // symmetric codebook: neg = !top bit, magnitude index m = low bits ^ (neg ? H-1 : 0)
         const uint32_t negw = live ? ~w[BITS - 1] : 0u;
         uint32_t mp[BITS > 1 ? BITS - 1 : 1];
@@ -229,6 +251,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           if (ALG2) *(uint4*)(bsg + off) = make_uint4(s4[0], s4[1], s4[2], s4[3]);
         }
       }
+#pragma unroll
+      for (int j = 0; j < UPT; ++j) {
+#pragma unroll
+        for (int pl = 0; pl < BITS; ++pl) cw[j][pl] = nw[j][pl];
+        cs[j] = ns[j];
+      }
+      cn = nn;
+      cg = ngm;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_FULL + a]);
