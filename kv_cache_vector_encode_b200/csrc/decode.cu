@@ -10,10 +10,17 @@
 //   D1a = PiT_hi c_hi,  D1b = PiT_lo c_hi + PiT_hi c_lo,  D2a = ST_hi s,  D2b = ST_lo s
 //   x_hat = n ((D1a + 2^-12 D1b) + alpha gamma (D2a + 2^-12 D2b))
 // Roles (14 warps): warp 0 bulk-copies the resident operands; warp 1 owns TMEM and issues MMAs;
-// warps 2-5 unpack (one thread per (vector, 32-coordinate group): the symmetric codebook's fp16
-// magnitudes picked by byte permutes, the sign from the top bit; 16-byte swizzled stores into a
+// warps 2-5 unpack (one thread per (vector, 32-coordinate group), 16-byte swizzled stores into a
 // double-buffered operand);
 // warps 6-13 are the epilogue (two warps per TMEM lane quarter). All waits are bounded.
+//
+// Unpacking: for s = 0..3 the nibbles of ((w0 >> s) & 0x11111111) | ((w1 >> s) & 0x11111111) << 1
+// | ... are the code indices of coordinates s + 4 n (n = 0..7) of a 32-coordinate group. Used as
+// byte-permute selectors over the low and the high bytes of the fp16 levels (up to eight levels;
+// sixteen-level codebooks look up the magnitude of the symmetric codebook and flip the sign), four
+// coordinates cost two lookups and two interleaves per fp16 part. The group's K order is therefore
+// k = 8 s + 4 half + n for coordinate 16 half + 4 n + s, and the resident Pi^T / S^T images (made
+// by tq_rotation_prepare for this kernel only) store their K columns in that order.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -39,7 +46,7 @@ struct DecodeParams {
   const uint16_t* gammas;
   void* out;
   float alpha;
-  uint32_t mag_hi[4], mag_lo[4];   // fp16 hi / lo parts of the positive levels c[L/2 + m], two per word
+  uint32_t tab[8];                 // level bytes: [0,1] low / [2,3] high bytes of c_hi, [4,5] / [6,7] of c_lo
   uint32_t* err;
 };
 
@@ -49,19 +56,6 @@ struct DecLayout {
 };
 
 __host__ __device__ inline uint32_t dround(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
-
-// fp16 magnitudes of levels ma (low half) and mb (high half) of a symmetric codebook with H positive
-// levels, by byte permutes over the table t0..t3 (entry m in bytes 2m, 2m + 1).
-template <int H>
-__device__ __forceinline__ uint32_t mag2(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3, uint32_t ma,
-                                         uint32_t mb) {
-  if (H == 1) return (t0 & 0xFFFFu) | (t0 << 16);
-  const uint32_t sel = ((ma & 3u) * 0x22u + 0x10u) | (((mb & 3u) * 0x22u + 0x10u) << 8);
-  const uint32_t r0 = __byte_perm(t0, t1, sel);
-  if (H <= 4) return r0;
-  const uint32_t r1 = __byte_perm(t2, t3, sel);
-  return __byte_perm(r0, r1, 0x3210u | ((ma & 4u) * 0x11u) | ((mb & 4u) * 0x1100u));
-}
 
 template <bool ALG2>
 __host__ __device__ inline DecLayout dec_layout(int KP, int NV) {
@@ -163,13 +157,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   } else if (warp < 6) {
     // ---------------- unpackers: codes -> fp16 B operands -----------------------------------------
     const int ut = tid - 64;               // 0..127
-    constexpr int H = 1 << (BITS - 1);
-    uint32_t th[4], tl[4];
+    uint32_t tab[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      th[k] = p.mag_hi[k];
-      tl[k] = p.mag_lo[k];
-    }
+    for (int k = 0; k < 8; ++k) tab[k] = p.tab[k];
     const int gp = KP / 32;                  // groups per operand row (padding groups included)
     const int units = NV * gp;
     constexpr int UPT = NV * 4 / 128;        // units per thread (gp <= 4)
@@ -219,36 +209,43 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         const bool live = v < rows && g < G;
         const uint32_t* w = cw[j];
         const uint32_t sg = cs[j];
-        // symmetric codebook: neg = !top bit, magnitude index m = low bits ^ (neg ? H-1 : 0)
-        const uint32_t negw = live ? ~w[BITS - 1] : 0u;
-        uint32_t mp[BITS > 1 ? BITS - 1 : 1];
+        // selector planes: the index bits (up to 3), or for 16 levels the magnitude bits
+        // (low bits ^ ~top bit) with the sign taken from the top bit
+        constexpr int SB = BITS < 4 ? BITS : 3;
+        const uint32_t flip = BITS == 4 ? ~w[BITS == 4 ? 3 : 0] : 0u;
 #pragma unroll
-        for (int pl = 0; pl < BITS - 1; ++pl) mp[pl] = w[pl] ^ negw;
+        for (int s4 = 0; s4 < 4; ++s4) {
+          uint32_t x = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {           // four 8-coordinate chunks of the group
-          uint32_t hi4[4], lo4[4], s4[4];
+          for (int pl = 0; pl < SB; ++pl) x |= (((w[pl] ^ flip) >> s4) & 0x11111111u) << pl;
+          const uint32_t fl = BITS == 4 ? (flip >> s4) & 0x11111111u : 0u;
+          uint32_t o_hi[4], o_lo[4], o_s[4];
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int bit = 8 * c + 2 * h;       // elements bit, bit + 1 -> low, high half
-            uint32_t ma = 0, mb = 0;
-#pragma unroll
-            for (int pl = 0; pl < BITS - 1; ++pl) {
-              ma |= ((mp[pl] >> bit) & 1u) << pl;
-              mb |= ((mp[pl] >> (bit + 1)) & 1u) << pl;
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t sel = half ? x >> 16 : x;
+            uint32_t hb = __byte_perm(tab[2], tab[3], sel), hl = __byte_perm(tab[6], tab[7], sel);
+            if (BITS == 4) {
+              const uint32_t sb = __byte_perm(0x8000u, 0u, half ? fl >> 16 : fl);   // 0x80 where negative
+              hb ^= sb;
+              hl ^= sb;
             }
-            const uint32_t ng = (negw >> bit) & 3u;
-            const uint32_t sgnbits = ((ng & 1u) << 15) | ((ng & 2u) << 30);
-            hi4[h] = live ? (mag2<H>(th[0], th[1], th[2], th[3], ma, mb) | sgnbits) : 0u;
-            lo4[h] = live ? (mag2<H>(tl[0], tl[1], tl[2], tl[3], ma, mb) | sgnbits) : 0u;
+            const uint32_t lb = __byte_perm(tab[0], tab[1], sel), ll = __byte_perm(tab[4], tab[5], sel);
+            o_hi[2 * half] = live ? __byte_perm(lb, hb, 0x5140u) : 0u;
+            o_hi[2 * half + 1] = live ? __byte_perm(lb, hb, 0x7362u) : 0u;
+            o_lo[2 * half] = live ? __byte_perm(ll, hl, 0x5140u) : 0u;
+            o_lo[2 * half + 1] = live ? __byte_perm(ll, hl, 0x7362u) : 0u;
             if (ALG2) {
-              const uint32_t zn = (~sg >> bit) & 3u;          // z = 0 -> -1
-              s4[h] = live ? (0x3C003C00u | ((zn & 1u) << 15) | ((zn & 2u) << 30)) : 0u;
+              // z = 1 -> +1 (0x3C00), z = 0 -> -1 (0xBC00)
+              const uint32_t zs = ((~sg >> s4) & 0x11111111u) >> (half ? 16 : 0);
+              const uint32_t zb = __byte_perm(0xBC3Cu, 0u, zs);
+              o_s[2 * half] = live ? __byte_perm(0u, zb, 0x5140u) : 0u;
+              o_s[2 * half + 1] = live ? __byte_perm(0u, zb, 0x7362u) : 0u;
             }
           }
-          const uint32_t off = sw128_offset(v, (g * 32 + c * 8) * 2, NV);
-          *(uint4*)(bch + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-          *(uint4*)(bcl + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
-          if (ALG2) *(uint4*)(bsg + off) = make_uint4(s4[0], s4[1], s4[2], s4[3]);
+          const uint32_t off = sw128_offset(v, (g * 32 + s4 * 8) * 2, NV);
+          *(uint4*)(bch + off) = make_uint4(o_hi[0], o_hi[1], o_hi[2], o_hi[3]);
+          *(uint4*)(bcl + off) = make_uint4(o_lo[0], o_lo[1], o_lo[2], o_lo[3]);
+          if (ALG2) *(uint4*)(bsg + off) = make_uint4(o_s[0], o_s[1], o_s[2], o_s[3]);
         }
       }
 #pragma unroll
@@ -386,21 +383,26 @@ extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t 
   p.gammas = gammas;
   p.out = out;
   p.alpha = (float)(std::sqrt(M_PI / 2.0) / d);
-  const int L = cb->levels, H = L / 2;
+  const int L = cb->levels;
   for (int k = 0; k < L; ++k)
     if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, "tq_decode: codebook is not symmetric");
-  uint16_t hi[8] = {}, lo[8] = {};
-  for (int m = 0; m < H; ++m) {
-    const float c = cb->c[H + m];
+  // up to eight levels are looked up directly; sixteen by magnitude (the positive half c[8 + m])
+  const int base_level = L > 8 ? L / 2 : 0, nt = L > 8 ? 8 : L;
+  uint8_t hl[4][8] = {};                       // [low c_hi, high c_hi, low c_lo, high c_lo][entry]
+  for (int m = 0; m < nt; ++m) {
+    const float c = cb->c[base_level + m];
     const __half h = __float2half_rn(c);
     const __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
-    hi[m] = __half_as_ushort(h);
-    lo[m] = __half_as_ushort(l);
+    const uint16_t hu = __half_as_ushort(h), lu = __half_as_ushort(l);
+    hl[0][m] = (uint8_t)(hu & 0xFF);
+    hl[1][m] = (uint8_t)(hu >> 8);
+    hl[2][m] = (uint8_t)(lu & 0xFF);
+    hl[3][m] = (uint8_t)(lu >> 8);
   }
-  for (int k = 0; k < 4; ++k) {
-    p.mag_hi[k] = (uint32_t)hi[2 * k] | ((uint32_t)hi[2 * k + 1] << 16);
-    p.mag_lo[k] = (uint32_t)lo[2 * k] | ((uint32_t)lo[2 * k + 1] << 16);
-  }
+  for (int t = 0; t < 4; ++t)
+    for (int w = 0; w < 2; ++w)
+      p.tab[2 * t + w] = (uint32_t)hl[t][4 * w] | (uint32_t)hl[t][4 * w + 1] << 8 | (uint32_t)hl[t][4 * w + 2] << 16 |
+                         (uint32_t)hl[t][4 * w + 3] << 24;
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, "tq_decode: no device error word (is a CUDA device present?)");
   cudaStream_t st = (cudaStream_t)stream;

@@ -62,13 +62,22 @@ __global__ void t_matrix_kernel(const float* __restrict__ S, const float* __rest
 // hi/lo fp16 split of M (or of M^T when transpose), zero padded to dp x dp, written as the
 // shared-memory image the tensor-core kernels use (see RotLayout): element (r, c) goes to
 //   (r / 128) * (128 * dp * 2) + sw128_offset(r % 128, 2 c, 128)   bytes.
+// The transposed images (read only by the decoder) hold in column c of each 32-column group the
+// coordinate 16 half + 4 n + s for c % 32 = 8 s + 4 half + n: the order in which the decoder's
+// byte-permute unpack produces a group.
 __global__ void split_kernel(const float* __restrict__ M, int d, int dp, bool transpose, __half* __restrict__ hi,
                              __half* __restrict__ lo) {
   size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (size_t)dp * dp) return;
   int r = (int)(idx / dp), c = (int)(idx % dp);
   float v = 0.0f;
-  if (r < d && c < d) v = transpose ? M[(size_t)c * d + r] : M[(size_t)r * d + c];
+  if (transpose) {
+    const int kk = c & 31;
+    const int cc = (c & ~31) + 16 * ((kk >> 2) & 1) + 4 * (kk & 3) + (kk >> 3);
+    if (r < d && cc < d) v = M[(size_t)cc * d + r];
+  } else if (r < d && c < d) {
+    v = M[(size_t)r * d + c];
+  }
   __half h = __float2half_rn(v);
   __half l = __float2half_rn((v - __half2float(h)) * kSplitScale);
   size_t off = (size_t)(r >> 7) * (128u * dp * 2) + sw128_offset(r & 127, 2 * c, 128);
