@@ -100,9 +100,8 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   const int b = slice / p.Hkv, hk = slice % p.Hkv;
   const int d = p.d, i = threadIdx.x;            // coordinate (128 threads)
   const int warp = i >> 5, lane = i & 31;
-  __shared__ float sq[8][128];
-  __shared__ double qr[8][128];
-  __shared__ double red[128];
+  __shared__ __align__(16) float sq[8][128];
+  __shared__ double red[4][8][2];
   const int kbytes = p.mk * d;
   uint8_t* img = p.bq_img + (size_t)slice * p.nq * kbytes;
   for (int o = i; o < p.nq * kbytes / 16; o += blockDim.x) ((uint4*)img)[o] = make_uint4(0, 0, 0, 0);
@@ -112,52 +111,53 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
                         : ((const float*)p.q)[qoff + i];
   }
   __syncthreads();
-  // q'_h = Pi q_h: one warp per output coordinate, lanes across the row of Pi (coalesced)
-  for (int r = warp; r < d; r += 4) {
-    const float* row = p.Pi + (size_t)r * d;
-    double acc[8];
+  // q'_h[i] = sum_j Pi[i][j] q_h[j] for every head: one thread per output coordinate, its row of Pi
+  // read as float4, fp64 accumulation (one independent chain per head)
+  double acc[8];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h] = 0.0;
-    for (int j = lane; j < d; j += 32) {
-      const double pij = (double)row[j];
-#pragma unroll
-      for (int h = 0; h < 8; ++h)
-        if (h < p.Hg) acc[h] = fma(pij, (double)sq[h][j], acc[h]);
-    }
+  for (int h = 0; h < 8; ++h) acc[h] = 0.0;
+  const float4* row = (const float4*)(p.Pi + (size_t)i * d);
+  for (int j4 = 0; j4 < d / 4; ++j4) {
+    const float4 pv = __ldg(row + j4);
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       if (h < p.Hg) {
-        double v = acc[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) qr[h][r] = v;
+        const float4 qv = *(const float4*)&sq[h][4 * j4];
+        acc[h] = fma((double)pv.x, (double)qv.x, acc[h]);
+        acc[h] = fma((double)pv.y, (double)qv.y, acc[h]);
+        acc[h] = fma((double)pv.z, (double)qv.z, acc[h]);
+        acc[h] = fma((double)pv.w, (double)qv.w, acc[h]);
       }
     }
   }
-  __syncthreads();
   double bmax = 0.0, sb = 0.0;
   for (int S = 0; S < p.mk; ++S) {
     bmax = fmax(bmax, fabs((double)p.beta_k[S]));
     sb += (double)p.beta_k[S];
   }
-  for (int h = 0; h < p.Hg; ++h) {
-    const double qi = qr[h][i];
-    red[i] = qi;
-    __syncthreads();
-    for (int o = 64; o > 0; o >>= 1) {
-      if (i < o) red[i] += red[i + o];
-      __syncthreads();
+  // per head: Q_h = sum_i q'_i and max_i |q'_i| bmax, warp shuffles then one exchange
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    if (h < p.Hg) {
+      double sm = acc[h], mx = fabs(acc[h]) * bmax;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        red[warp][h][0] = sm;
+        red[warp][h][1] = mx;
+      }
     }
-    const double Qh = red[0];
-    __syncthreads();
-    red[i] = fabs(qi) * bmax;
-    __syncthreads();
-    for (int o = 64; o > 0; o >>= 1) {
-      if (i < o) red[i] = fmax(red[i], red[i + o]);
-      __syncthreads();
-    }
-    const double vmax = red[0];
-    __syncthreads();
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    if (h >= p.Hg) break;
+    const double qi = acc[h];
+    const double Qh = (red[0][h][0] + red[1][h][0]) + (red[2][h][0] + red[3][h][0]);
+    const double vmax = fmax(fmax(red[0][h][1], red[1][h][1]), fmax(red[2][h][1], red[3][h][1]));
     int F = 0;
     if (vmax > 0.0) {
       int E;
@@ -839,12 +839,23 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
   }
   __syncthreads();
   if (i < d) {
-    float acc = 0.0f;
-    for (int j = 0; j < d; ++j) acc = fmaf(p.Pi[(size_t)j * d + i], orot[j], acc);
+    // four independent partial sums per product (the loads of a column of Pi / S are coalesced
+    // across the threads)
+    float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+    for (int j = 0; j < d; j += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = fmaf(__ldg(p.Pi + (size_t)(j + u) * d + i), orot[j + u], a[u]);
+    }
+    float acc = (a[0] + a[1]) + (a[2] + a[3]);
     if (p.vsign) {
-      float a2 = 0.0f;
-      for (int j = 0; j < d; ++j) a2 = fmaf(p.S[(size_t)j * d + i], osgn[j], a2);
-      acc = fmaf(p.alpha, a2, acc);
+      float z[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+      for (int j = 0; j < d; j += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) z[u] = fmaf(__ldg(p.S + (size_t)(j + u) * d + i), osgn[j + u], z[u]);
+      }
+      acc = fmaf(p.alpha, (z[0] + z[1]) + (z[2] + z[3]), acc);
     }
     p.out[(size_t)bh * d + i] = acc;
   }
