@@ -202,6 +202,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       const uint32_t a2 = ALG2 ? smem_u32(smem + Lo.off_a[2]) : 0u, a3 = ALG2 ? smem_u32(smem + Lo.off_a[3]) : 0u;
       const uint32_t r0 = ALG2 ? smem_u32(smem + Lo.off_rho[0]) : 0u, r1 = ALG2 ? smem_u32(smem + Lo.off_rho[1]) : 0u;
       const int ksteps = KP / 16;
+      // With NV = 64, rho is stored MN-major: one 128-byte row (the 64 vectors) per coordinate, so
+      // the K = 16 slice of a step is 16 rows (2048 bytes) on. Otherwise K-major like x.
+      constexpr bool RHO_MN = NV == 64;
+      const uint32_t idesc_t = RHO_MN ? (idesc | (1u << 16)) : idesc;   // B (rho) MN-major
       auto issue_T = [&](int j) -> bool {
         const int a = j & 1;
         if (!mbar_wait_warp(&bar[RHO_FULL], j & 1, p.err, kDevTimeoutSync, abort_flag)) return false;
@@ -210,10 +214,13 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         if (elect_one_sync()) {
           for (int ks = 0; ks < ksteps; ++ks) {
             const uint32_t kb = ks * 32, blk = kb >> 7, inb = kb & 127;
-            const uint32_t ao = blk * 128 * 128 + inb, bo = blk * NV * 128 + inb;
-            mma_f16_ss(dT1, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
-            mma_f16_ss(dT2, desc_kmajor_sw128(a3 + ao), desc_kmajor_sw128(r0 + bo), idesc, ks > 0);
-            mma_f16_ss(dT2, desc_kmajor_sw128(a2 + ao), desc_kmajor_sw128(r1 + bo), idesc, 1);
+            const uint32_t ao = blk * 128 * 128 + inb;
+            const uint32_t bo = RHO_MN ? ks * 16 * 128 : blk * NV * 128 + inb;
+            const uint64_t d0 = RHO_MN ? desc_smem(r0 + bo, 1024, 1024, 2) : desc_kmajor_sw128(r0 + bo);
+            const uint64_t d1 = RHO_MN ? desc_smem(r1 + bo, 1024, 1024, 2) : desc_kmajor_sw128(r1 + bo);
+            mma_f16_ss(dT1, desc_kmajor_sw128(a2 + ao), d0, idesc_t, ks > 0);
+            mma_f16_ss(dT2, desc_kmajor_sw128(a3 + ao), d0, idesc_t, ks > 0);
+            mma_f16_ss(dT2, desc_kmajor_sw128(a2 + ao), d1, idesc_t, 1);
           }
           mma_commit(&bar[T_FULL + a]);
         }
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         uint32_t myw[BITS];
 #pragma unroll
         for (int pl = 0; pl < BITS; ++pl) myw[pl] = 0u;
-        float r2[16];
+        float r2[16];                       // rho * 2^14 of the 16 vectors (Algorithm 2)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int v = c0 + j;
@@ -397,15 +404,44 @@ __global__ void __launch_bounds__(kEncThreads, 1)
             const float cm = sym_c<BITS>(m, C);
             float rho = neg ? y + cm : y - cm;
             if (!active || inv == 0.0f) rho = 0.0f;
-            r2[j] = rho * rho;
-            const float rs = rho * kRhoScale;
-            const __half rh = __float2half_rn(rs);
-            const __half rl = __float2half_rn((rs - __half2float(rh)) * kSplitScale);
-            if (i < KP) {
-              const uint32_t off = sw128_offset(v, 2 * i, NV);
-              *(__half*)(rho_hi + off) = rh;
-              *(__half*)(rho_lo + off) = rl;
+            if (NV == 64) {
+              r2[j] = rho * kRhoScale;            // stored below, two vectors per word
+            } else {
+              // K-major rho (32-vector tiles): one fp16 per (vector row, coordinate)
+              r2[j] = rho * rho;
+              const float rs = rho * kRhoScale;
+              const __half rh = __float2half_rn(rs);
+              const __half rl = __float2half_rn((rs - __half2float(rh)) * kSplitScale);
+              if (i < KP) {
+                const uint32_t off = sw128_offset(v, 2 * i, NV);
+                *(__half*)(rho_hi + off) = rh;
+                *(__half*)(rho_lo + off) = rl;
+              }
             }
+          }
+        }
+        if (ALG2) {
+          // fp16 hi / lo split of rho 2^14, two vectors per word, into this coordinate's row
+          if (NV == 64 && i < KP) {
+            uint32_t hw[8], lw[8];
+#pragma unroll
+            for (int jp = 0; jp < 8; ++jp) {
+              const __half2 h2 = __floats2half2_rn(r2[2 * jp], r2[2 * jp + 1]);
+              const float2 back = __half22float2(h2);
+              hw[jp] = h2_bits(h2);
+              lw[jp] = h2_bits(__floats2half2_rn((r2[2 * jp] - back.x) * kSplitScale,
+                                                 (r2[2 * jp + 1] - back.y) * kSplitScale));
+            }
+            const uint32_t o0 = sw128_offset(i, 2 * c0, 128), o1 = sw128_offset(i, 2 * c0 + 16, 128);
+            *(uint4*)(rho_hi + o0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *(uint4*)(rho_hi + o1) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            *(uint4*)(rho_lo + o0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            *(uint4*)(rho_lo + o1) = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+          }
+          // |rho|^2 terms: (rho 2^14)^2 2^-28 rounds exactly like rho^2 (power-of-two scaling)
+          if (NV == 64) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r2[j] = r2[j] * r2[j] * (1.0f / 268435456.0f);
           }
         }
         if (q < G && lane < 16) {

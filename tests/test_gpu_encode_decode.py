@@ -197,3 +197,38 @@ def test_repeat_runs_identical(dev):
     b = run_prod(x, d, 3, torch.float32, dev)
     for ta, tb in zip(a[1:], b[1:]):
         assert torch.equal(ta, tb)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("alg2,bits", [(False, 1), (False, 2), (False, 3), (False, 4), (True, 2), (True, 3),
+                                       (True, 4), (True, 5)])
+def test_decode_precision(dev, d, alg2, bits):
+    # Decode from the codes alone, against the oracle's fp64 decode of the same codes. The fp16
+    # hi/lo split of the codebook and of Pi^T / S^T carries about 22 significant bits and the
+    # products accumulate in fp32, so the normwise error stays near 1e-6. A lost low part (2^-12)
+    # or a misplaced level would show here.
+    n = 700
+    g = np.random.default_rng(100 * d + 10 * bits + alg2)
+    cbits = bits - 1 if alg2 else bits
+    codes_np = g.integers(0, 2 ** 32, size=(n, d // 32, cbits), dtype=np.uint64).astype(np.uint32)
+    norms_np = W.round_to_bf16(np.abs(g.standard_normal(n)).astype(np.float32) + 0.1).astype(np.float16)
+    Pi, S, rot = rotation(d, dev)
+    cb = tq.tq_codebook_init(d, cbits)
+    ocb = lloyd_max(d, cbits)
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(dev)
+    codes = t(codes_np, np.int32)
+    norms = t(norms_np, np.int16).view(torch.float16)
+    out = torch.empty((n, d), dtype=torch.float32, device=dev)
+    if alg2:
+        signs_np = g.integers(0, 2 ** 32, size=(n, d // 32), dtype=np.uint64).astype(np.uint32)
+        gam_np = (np.abs(g.standard_normal(n)) * 0.3).astype(np.float16)
+        tq.tq_decode(cb, rot, codes, norms, out, signs=t(signs_np, np.int32),
+                     gammas=t(gam_np, np.int16).view(torch.float16))
+        want = Q.decode(codes_np, norms_np, Pi, ocb, signs_np, gam_np, S)
+    else:
+        tq.tq_decode(cb, rot, codes, norms, out)
+        want = Q.decode(codes_np, norms_np, Pi, ocb)
+    tq.tq_sync_check()
+    rel = normwise_rel(out.cpu().numpy(), want)
+    print("decode precision", d, alg2, bits, rel.max())
+    assert rel.max() <= 1e-5, rel.max()
