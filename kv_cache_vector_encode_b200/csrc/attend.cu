@@ -34,10 +34,12 @@
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
 // (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
-// Main-kernel roles (19 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the key MMAs;
+// Main-kernel roles (19 warps, 23 with separate value expanders): 0 bulk-copies packed chunks; 1
+// owns TMEM and issues the key MMAs;
 // 2-9 softmax (thread = token; two groups of four warps, each group owning half of the query
-// heads); 10-13 expand K into TMEM and V into shared memory (thread = token); 14-17 accumulate the
-// value products (thread = coordinate); 18 issues the value MMAs.
+// heads); 10-13 expand K into TMEM and (19 warps) V into shared memory (thread = token); 14-17
+// accumulate the value products (thread = coordinate); 18 issues the value MMAs; 19-22 (at most
+// four query heads per KV head) expand V, so that key and value expansion run side by side.
 // All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
 // same number of times by all four warps (their loop never exits early).
 #include <cuda_fp16.h>
@@ -52,7 +54,10 @@
 namespace tq {
 namespace {
 
-constexpr int kAttThreads = 608;                // 19 warps
+// warps of the main kernel: 23 when the value planes have their own expander warps (at most four
+// query heads per KV head; 80 registers a thread), else 19 (96 registers)
+__host__ __device__ constexpr bool att_split_v(int hg) { return hg <= 4; }
+__host__ __device__ constexpr int att_warps(int hg) { return att_split_v(hg) ? 23 : 19; }
 constexpr int kChunk = 128;                 // tokens per chunk
 constexpr int kMaxStages = 8;               // packed-chunk ring (depth chosen from shared memory)
 constexpr int kMaxSmem = 232448;            // 227 KB of dynamic shared memory per block
@@ -289,10 +294,46 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
   return r;
 }
 
+// Value planes of one token (thread = token t of the chunk): plane words (and sign words) ->
+// bytes 0 / 2^s, one 128-byte token row per plane (128-byte swizzle, slots voff).
+template <int BV, int VS, int NP>
+__device__ __forceinline__ void expand_v_rows(const AttParams& p, const AttLayout& Lo, const uint8_t* stg, uint8_t* avb,
+                                              int t, const uint32_t (&voff)[8]) {
+  uint32_t vw[4 * BV];
+#pragma unroll
+  for (int v4 = 0; v4 < BV; ++v4) {
+    const uint4 x = *(const uint4*)(stg + Lo.kc_bytes + t * 16 * BV + v4 * 16);
+    vw[4 * v4] = x.x;
+    vw[4 * v4 + 1] = x.y;
+    vw[4 * v4 + 2] = x.z;
+    vw[4 * v4 + 3] = x.w;
+  }
+  uint32_t sg[4] = {0u, 0u, 0u, 0u};
+  if (VS) {
+    const uint4 x = *(const uint4*)(stg + Lo.sg_off + t * 16);
+    sg[0] = x.x;
+    sg[1] = x.y;
+    sg[2] = x.z;
+    sg[3] = x.w;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+#pragma unroll
+    for (int P = 0; P < NP; ++P) {
+      // the Walsh planes of a 1- or 2-bit codebook are its bit planes
+      const uint32_t w = (VS && P == NP - 1) ? sg[g] : vw[g * BV + (P < BV ? P : 0)];
+      uint8_t* row = avb + P * Lo.av_bytes;
+      *(uint4*)(row + voff[2 * g]) = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
+      *(uint4*)(row + voff[2 * g + 1]) = make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
+    }
+  }
+}
+
 // HG: query heads per KV head (4 or 8, Hg <= HG); BK: key bits; BV: value codebook bits;
 // VS: value sign plane (Algorithm 2 values)
 template <int HG, int BK, int BV, int VS>
-__global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttParams p) {
+__global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const __grid_constant__ AttParams p) {
+  constexpr bool SPLITV = att_split_v(HG);
   constexpr int MK = walsh_count(BK);
   constexpr int MV = walsh_count(BV);
   constexpr int NP = MV + VS;
@@ -323,7 +364,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&bar[ST_FULL + s], 1);
-      mbar_init(&bar[ST_EMPTY + s], 4);
+      mbar_init(&bar[ST_EMPTY + s], SPLITV ? 8 : 4);   // key (and value) expanders
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
@@ -624,41 +665,17 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[AK_FULL + b]);
+      if (SPLITV) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[ST_EMPTY + st]);
+        continue;
+      }
       // values: plane words (and sign words) -> expanded bytes, one token row per plane; the
       // planes of chunk c - 3 (same buffer) must have been consumed
       const int c3 = c % 3;
       if (c >= 3 && !mbar_wait_warp(&bar[V_DONE + (c - 3) % 6], ((c - 3) / 6) & 1, p.err, kDevTimeoutMma, abort_flag))
         break;
-      uint32_t vw[4 * BV];
-#pragma unroll
-      for (int v4 = 0; v4 < BV; ++v4) {
-        const uint4 x = *(const uint4*)(stg + Lo.kc_bytes + t * 16 * BV + v4 * 16);
-        vw[4 * v4] = x.x;
-        vw[4 * v4 + 1] = x.y;
-        vw[4 * v4 + 2] = x.z;
-        vw[4 * v4 + 3] = x.w;
-      }
-      uint32_t sg[4] = {0u, 0u, 0u, 0u};
-      if (VS) {
-        const uint4 x = *(const uint4*)(stg + Lo.sg_off + t * 16);
-        sg[0] = x.x;
-        sg[1] = x.y;
-        sg[2] = x.z;
-        sg[3] = x.w;
-      }
-      uint8_t* avb = smem + Lo.off_av + c3 * NP * Lo.av_bytes;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-#pragma unroll
-        for (int P = 0; P < NP; ++P) {
-          // the Walsh planes of a 1- or 2-bit codebook are its bit planes
-          const uint32_t w = (VS && P == NP - 1) ? sg[g] : vw[g * BV + (P < BV ? P : 0)];
-          uint8_t* row = avb + P * Lo.av_bytes;
-          *(uint4*)(row + voff[2 * g]) = make_uint4(w & 0x01010101u, w & 0x02020202u, w & 0x04040404u, w & 0x08080808u);
-          *(uint4*)(row + voff[2 * g + 1]) =
-              make_uint4(w & 0x10101010u, w & 0x20202020u, w & 0x40404040u, w & 0x80808080u);
-        }
-      }
+      expand_v_rows<BV, VS, NP>(p, Lo, stg, smem + Lo.off_av + c3 * NP * Lo.av_bytes, t, voff);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -755,7 +772,7 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         }
       }
     }
-  } else {
+  } else if (warp == 18) {
     // ------------------------------------ value MMA issuer (warp 18) ------------------------------
     // Runs beside the key MMA warp so that neither warp's barrier waits and commits sit behind the
     // other's tensor-core work. Warp-uniform schedule, one elected lane issues.
@@ -784,6 +801,31 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
         mma_commit(&bar[V_DONE + c % 6]);
       }
       __syncwarp();
+    }
+  } else if (SPLITV) {
+    // ------------------------------------ value expanders (warps 19-22, thread = token) -----------
+    const int q = warp & 3;
+    const int t = q * 32 + lane;
+    uint32_t voff[8];                               // this token's 16-byte slots in a value plane
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      voff[2 * g] = sw128_offset(t, g * 32, 128);
+      voff[2 * g + 1] = sw128_offset(t, g * 32 + 16, 128);
+    }
+    for (int c = 0; c < nmy; ++c) {
+      const int st = c % nst, c3 = c % 3;
+      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / nst) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+      // the planes of chunk c - 3 (same buffer) must have been consumed
+      if (c >= 3 && !mbar_wait_warp(&bar[V_DONE + (c - 3) % 6], ((c - 3) / 6) & 1, p.err, kDevTimeoutMma, abort_flag))
+        break;
+      expand_v_rows<BV, VS, NP>(p, Lo, smem + Lo.off_stage + st * Lo.stage_bytes,
+                                smem + Lo.off_av + c3 * NP * Lo.av_bytes, t, voff);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[AV_FULL + c3]);
+        mbar_arrive(&bar[ST_EMPTY + st]);
+      }
     }
   }
 
@@ -1009,7 +1051,7 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode: shared memory attribute");
   const long long totalc = (long long)p.slices * p.nchunk;
   const int grid = (int)((totalc + p.per_cta - 1) / p.per_cta);
-  kern<<<grid, kAttThreads, Lo.total, st>>>(p);
+  kern<<<grid, 32 * att_warps(p.Hg <= 4 ? 4 : 8), Lo.total, st>>>(p);
   attend_combine_kernel<<<B * Hq, 128, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tq_attend_decode: launch");
   return TQ_OK;
