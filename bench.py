@@ -302,22 +302,23 @@ def run_ours(args):
     outv = torch.empty((nblk, D), dtype=torch.float32, device=dev)
     tq.tq_sync_check()
 
-    def step(ev=None):
+    def step(ev=None, bufs=None):
+        Kx, Vx, qx, (ckc, ckn, cvc, cvs, cvn, cvg, cout) = bufs or (Kb, Vb, q, (bkc, bkn, bvc, bvs, bvn, bvg, att_out))
         if ev is not None:
             ev[0].record(stream)
-        tq.tq_encode_mse(cbk, Kb, rot, bkc, bkn)
+        tq.tq_encode_mse(cbk, Kx, rot, ckc, ckn)
         if ev is not None:
             ev[1].record(stream)
-        tq.tq_encode_prod(cbv, Vb, rot, bvc, bvs, bvn, bvg)
+        tq.tq_encode_prod(cbv, Vx, rot, cvc, cvs, cvn, cvg)
         if ev is not None:
             ev[2].record(stream)
-        tq.tq_decode(cbk, rot, bkc, bkn, outk)
+        tq.tq_decode(cbk, rot, ckc, ckn, outk)
         if ev is not None:
             ev[3].record(stream)
-        tq.tq_decode(cbv, rot, bvc, bvn, outv, signs=bvs, gammas=bvg)
+        tq.tq_decode(cbv, rot, cvc, cvn, outv, signs=cvs, gammas=cvg)
         if ev is not None:
             ev[4].record(stream)
-        tq.tq_attend_decode(cbk, cbv2, q, rot, kc, kn3, vc, vn3, att_out, v_signs=vs, v_gammas=vg3, ws=ws)
+        tq.tq_attend_decode(cbk, cbv2, qx, rot, kc, kn3, vc, vn3, cout, v_signs=vs, v_gammas=vg3, ws=ws)
         if ev is not None:
             ev[5].record(stream)
 
@@ -358,23 +359,54 @@ def run_ours(args):
     h2d = Kh.numel() * 2 + Vh.numel() * 2 + qh.numel() * 2
     d2h = sum(r.numel() * r.element_size() for r in res)
 
-    def e2e_step():
-        Kb.copy_(Kh, non_blocking=True)
-        Vb.copy_(Vh, non_blocking=True)
-        q.copy_(qh, non_blocking=True)
-        step()
-        for r, t in zip(res, (bkc, bkn, bvc, bvs, bvn, bvg, att_out)):
-            r.copy_(t, non_blocking=True)
+    # Two buffer sets: the inputs of step k+1 are copied in (one copy stream) while step k computes,
+    # and the results of step k are copied out (a second copy stream) while step k+1 computes.
+    # Every step's copies lie inside the timed region, which ends when the last results are home.
+    sets = [(Kb, Vb, q, (bkc, bkn, bvc, bvs, bvn, bvg, att_out))]
+    sets.append((torch.empty_like(Kb), torch.empty_like(Vb), torch.empty_like(q),
+                 tuple(torch.empty_like(t) for t in (bkc, bkn, bvc, bvs, bvn, bvg, att_out))))
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_run(n, start=None, end=None):
+        ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of the set are on the device
+        ev_done = [torch.cuda.Event() for _ in range(2)]    # the step using the set has finished
+        ev_out = [torch.cuda.Event() for _ in range(2)]     # the set's results are home
+        if start is not None:
+            start.record(h2d_s)
+
+        def copy_in(k):
+            Kx, Vx, qx, _ = sets[k % 2]
+            with torch.cuda.stream(h2d_s):
+                if k >= 2:
+                    h2d_s.wait_event(ev_done[k % 2])           # step k-2 has read this set
+                Kx.copy_(Kh, non_blocking=True)
+                Vx.copy_(Vh, non_blocking=True)
+                qx.copy_(qh, non_blocking=True)
+                ev_in[k % 2].record(h2d_s)
+
+        copy_in(0)
+        for k in range(n):
+            if k + 1 < n:
+                copy_in(k + 1)
+            stream.wait_event(ev_in[k % 2])
+            if k >= 2:
+                stream.wait_event(ev_out[k % 2])               # results of step k-2 are home
+            step(bufs=sets[k % 2])
+            ev_done[k % 2].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[k % 2])
+                for r, t in zip(res, sets[k % 2][3]):
+                    r.copy_(t, non_blocking=True)
+                ev_out[k % 2].record(d2h_s)
+        if end is not None:
+            d2h_s.wait_stream(h2d_s)
+            end.record(d2h_s)
+
+    e2e_run(2)
     barrier()
     a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, min(args.steps, 10))
-    a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    b2.record(stream)
+    e2e_run(e2e_steps, a, b2)
     barrier()
     e2e_ms = a.elapsed_time(b2) / e2e_steps
     if world > 1:
