@@ -195,6 +195,35 @@ TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb
                            const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
                            float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Workspace bytes of tq_attend_append for these sizes (k_bits: the key codebook's bits;
+ * v_codebook_bits: the value codebook's bits, b_v - 1); 0 for invalid sizes. */
+TQ_API size_t tq_attend_append_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t T_cur, int32_t d,
+                                               int32_t k_bits, int32_t v_codebook_bits);
+
+/* One decode step on a packed KV cache with room to grow: the new token's key and value of every
+ * (batch, KV head) slice are encoded into the next free slot, then the query attends over all
+ * filled slots. This is the cache-integration step around the attention (ai-navigate-news page:
+ * keys by Algorithm 1, values by Algorithm 2, appended as tokens are generated; aiboss88 page:
+ * attention on the quantised cache). The result equals tq_encode_mse / tq_encode_prod of the new
+ * vectors written to slot T_cur, followed by tq_attend_decode over T_cur + 1 tokens.
+ *   cache   the arrays of tq_attend_decode with T_max slots per slice: k_codes [B][Hkv][T_max][d/32][b_k],
+ *           k_norms [B][Hkv][T_max], v_codes [B][Hkv][T_max][d/32][b_v-1], v_signs
+ *           [B][Hkv][T_max][d/32], v_norms, v_gammas [B][Hkv][T_max]; slots [0, T_cur) hold
+ *           earlier tokens, slot T_cur is written, slots beyond it are neither read nor written
+ *   k_new, v_new  [B][Hkv][d] in x_dtype (TQ_F32 or TQ_BF16)
+ *   q, out, scale, cb_k, cb_v (the (b_v-1)-bit codebook), rot  as in tq_attend_decode
+ * Requires 0 <= T_cur < T_max and the limits of tq_attend_decode (d = 128, ...); values are
+ * Algorithm 2 (v_signs, v_gammas required). ws: caller device workspace of at least
+ * tq_attend_append_workspace_bytes(B, Hq, Hkv, T_cur, d, b_k, b_v - 1) bytes. Errors: those of
+ * the encoders and of tq_attend_decode; on an error nothing after the failing stage is enqueued.
+ * Launches, in stream order: the two encoders, one record-scatter kernel, the attention kernels. */
+TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                  int32_t Hkv, int64_t T_cur, int64_t T_max, int32_t d, const void* q,
+                                  int32_t q_dtype, const void* k_new, const void* v_new, int32_t x_dtype,
+                                  const void* rot, uint32_t* k_codes, uint16_t* k_norms, uint32_t* v_codes,
+                                  uint32_t* v_signs, uint16_t* v_norms, uint16_t* v_gammas, float scale,
+                                  float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Size of the fixed scratch array behind tq_attend_decode_noalloc (8 MiB per device). It covers,
  * for example, B = 16, Hkv = 8, Hq = 32, T = 131072 (about 3.4 MB). */
 #define TQ_ATTEND_NOALLOC_MAX_BYTES (8u << 20)

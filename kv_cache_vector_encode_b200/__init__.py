@@ -74,6 +74,9 @@ _SIGNATURES = {
                                 _F, _P, _P, _SZ, _P]),
     "tq_attend_decode_noalloc": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
                                         _P, _F, _P, _P]),
+    "tq_attend_append_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32, _I32, _I32]),
+    "tq_attend_append": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I64, _I32, _P, _I32, _P, _P, _I32, _P, _P, _P,
+                                _P, _P, _P, _P, _F, _P, _P, _SZ, _P]),
     "tq_sync_check": (_I32, [_P]),
 }
 
@@ -257,6 +260,35 @@ def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_
 
 
 TQ_ATTEND_NOALLOC_MAX_BYTES = 8 << 20
+
+
+def tq_attend_append_workspace_bytes(B: int, Hq: int, Hkv: int, T_cur: int, d: int, k_bits: int,
+                                     v_codebook_bits: int) -> int:
+    return int(lib().tq_attend_append_workspace_bytes(B, Hq, Hkv, T_cur, d, k_bits, v_codebook_bits))
+
+
+def tq_attend_append(cb_k: Codebook, cb_v: Codebook, q, rot, k_new, v_new, T_cur: int, k_codes, k_norms, v_codes,
+                     v_signs, v_norms, v_gammas, out, scale=None, ws=None, stream=None):
+    """Encode the new token's K / V of every slice into slot T_cur of the cache, then attend over slots
+    [0, T_cur]. The cache tensors are [B][Hkv][T_max]... as for tq_attend_decode; k_new, v_new [B][Hkv][d]."""
+    import math
+    import torch
+    B, Hq, d = q.shape
+    Hkv, T_max = k_norms.shape[1], k_norms.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    wsb = tq_attend_append_workspace_bytes(B, Hq, Hkv, T_cur, d, cb_k.bits, cb_v.bits)
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().tq_attend_append(ctypes.byref(cb_k), ctypes.byref(cb_v), B, Hq, Hkv, T_cur, T_max, d,
+                                  _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q),
+                                  _ptr(k_new, "k_new", [torch.float32, torch.bfloat16]),
+                                  _ptr(v_new, "v_new", [torch.float32, torch.bfloat16]), _xdtype(k_new),
+                                  _ptr(rot, "rot"), _ptr(k_codes, "k_codes", [torch.int32]),
+                                  _ptr(k_norms, "k_norms", [torch.float16]), _ptr(v_codes, "v_codes", [torch.int32]),
+                                  _ptr(v_signs, "v_signs", [torch.int32]), _ptr(v_norms, "v_norms", [torch.float16]),
+                                  _ptr(v_gammas, "v_gammas", [torch.float16]), float(scale),
+                                  _ptr(out, "out", [torch.float32]), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
 
 
 def tq_sync_check(stream=None):

@@ -68,7 +68,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ------------------------------------------------------------------------------------------------
 struct AttParams {
   int B, Hq, Hkv, Hg, d, G;
-  int64_t T;
+  int64_t T;                     // tokens attended per slice
+  int64_t tstride;               // token slots per slice in the cache arrays (>= T)
   int slices, nchunk, per_cta, maxseg;
   int nst;                       // depth of the packed-chunk ring
   int bk, mk;                    // key bits, key Walsh planes
@@ -355,7 +356,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   const int c_end = min(total, c_begin + p.per_cta);
   const int nmy = max(0, c_end - c_begin);
   const int d = p.d, G = p.G;
-  const int64_t T = p.T;
+  const int64_t T = p.T, TS = p.tstride;
   const uint32_t dv0 = kDS0 + 2 * NQ;
   const uint32_t dv_cols = NP * NQ;
   // tokens in the last chunk of every slice (all other chunks are full)
@@ -410,7 +411,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       const int st = c % nst;
       if (!mbar_wait_warp(&bar[ST_EMPTY + st], ((c / nst) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
       const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
-      const int64_t vec0 = (int64_t)it.slice * T + (int64_t)it.cis * kChunk;   // record of the first token
+      const int64_t vec0 = (int64_t)it.slice * TS + (int64_t)it.cis * kChunk;  // record of the first token
       const uint32_t kb = (uint32_t)tc * G * BK * 4;
       const uint32_t vb = (uint32_t)tc * G * BV * 4;
       const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
@@ -478,7 +479,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     auto load_norms = [&]() {
       nk_n = nv_n = gm_n = 0;
       if (t < (nx.cis == p.nchunk - 1 ? tail : kChunk)) {
-        const int64_t rec = (int64_t)nx.slice * T + (int64_t)nx.cis * kChunk + t;
+        const int64_t rec = (int64_t)nx.slice * TS + (int64_t)nx.cis * kChunk + t;
         nk_n = __ldg(p.k_norms + rec);
         nv_n = __ldg(p.v_norms + rec);
         if (VS) gm_n = __ldg(p.v_gammas + rec);
@@ -935,6 +936,7 @@ bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl) {
   p.d = d;
   p.G = d / 32;
   p.T = T;
+  p.tstride = T;
   p.slices = B * Hkv;
   p.nchunk = (int)((T + kChunk - 1) / kChunk);
   const long long totalc = (long long)p.slices * p.nchunk;
@@ -969,20 +971,20 @@ extern "C" TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_
   return pl.total;
 }
 
-extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
-                                             int32_t Hkv, int64_t T, int32_t d, const void* q, int32_t q_dtype,
-                                             const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
-                                             const uint32_t* v_codes, const uint32_t* v_signs, const uint16_t* v_norms,
-                                             const uint16_t* v_gammas, float scale, float* out, void* ws,
-                                             size_t ws_bytes, void* stream) {
-  clear_error();
-  const char* f = "tq_attend_decode";
+namespace tq {
+// Decode attention over T tokens of every slice, whose records lie tstride apart (tstride >= T).
+tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                      int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
+                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* v_codes,
+                      const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
+                      float* out, void* ws, size_t ws_bytes, void* stream) {
   if (!cb_k || !cb_v || !q || !rot || !k_codes || !k_norms || !v_codes || !v_norms || !out || !ws)
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": NULL pointer");
   if ((v_signs == nullptr) != (v_gammas == nullptr))
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": v_signs and v_gammas must both be NULL or both be set");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || Hq % Hkv)
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": bad B / Hq / Hkv / T");
+  if (tstride < T) return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": fewer cache slots than tokens");
   if (d != 128) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": this build supports d = 128");
   if (Hq / Hkv > 8) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": at most 8 query heads per KV head");
   if (T > ((int64_t)1 << 31)) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": T too large");
@@ -1007,6 +1009,7 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   if (ws_bytes < pl.total || ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
     return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
   AttParams& p = pl.p;
+  p.tstride = tstride;
   int kmask[8], vmask[8];
   float kbeta[8], vbeta[8];
   p.bk = cb_k->bits;
@@ -1055,4 +1058,16 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   attend_combine_kernel<<<B * Hq, 128, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tq_attend_decode: launch");
   return TQ_OK;
+}
+}  // namespace tq
+
+extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                             int32_t Hkv, int64_t T, int32_t d, const void* q, int32_t q_dtype,
+                                             const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
+                                             const uint32_t* v_codes, const uint32_t* v_signs, const uint16_t* v_norms,
+                                             const uint16_t* v_gammas, float scale, float* out, void* ws,
+                                             size_t ws_bytes, void* stream) {
+  clear_error();
+  return attend_impl("tq_attend_decode", cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, v_codes,
+                     v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream);
 }

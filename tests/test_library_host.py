@@ -93,3 +93,19 @@ def test_device_calls_reject_bad_arguments_on_host(L):
     assert L.tq_decode(ctypes.byref(cb), 10, 128, good, good, good, good, None, good, tq.TQ_F32, None) \
         == tq.TQ_ERR_INVALID_ARG
     assert L.tq_rotation_prepare(128, good, good, good, 16, None) == tq.TQ_ERR_WORKSPACE
+
+
+def test_attend_append_rejects_bad_arguments_on_host(L):
+    cbk, cbv = tq.tq_codebook_init(128, 3), tq.tq_codebook_init(128, 1)
+    P = ctypes.c_void_p
+    g = P(1 << 20)
+    args = lambda T_cur, T_max, ws_bytes, vs=g: (ctypes.byref(cbk), ctypes.byref(cbv), 2, 8, 2, T_cur, T_max, 128, g,
+                                                tq.TQ_BF16, g, g, tq.TQ_BF16, g, g, g, g, vs, g, g, ctypes.c_float(0.1), g,
+                                                g, ws_bytes, None)
+    need = L.tq_attend_append_workspace_bytes(2, 8, 2, 10, 128, 3, 1)
+    assert need > L.tq_attend_workspace_bytes(2, 8, 2, 11, 128)
+    assert L.tq_attend_append_workspace_bytes(2, 8, 2, -1, 128, 3, 1) == 0
+    assert L.tq_attend_append(*args(10, 10, need)) == tq.TQ_ERR_INVALID_ARG        # no free slot
+    assert L.tq_attend_append(*args(-1, 10, need)) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_attend_append(*args(10, 20, need, vs=None)) == tq.TQ_ERR_INVALID_ARG   # values are Algorithm 2
+    assert L.tq_attend_append(*args(10, 20, need - 1)) == tq.TQ_ERR_WORKSPACE
