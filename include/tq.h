@@ -181,7 +181,11 @@ TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int6
  * scores come from the key codes, and values are accumulated in the rotated / sign domain with
  * Pi^T and S^T applied once per query head. No mask: every one of the T tokens is attended.
  *   q       [B][Hq][d]  TQ_BF16 or TQ_F32
- *   keys    Algorithm 1 with cb_k (b_k bits): k_codes [B][Hkv][T][d/32][b_k], k_norms [B][Hkv][T]
+ *   keys    Algorithm 1 with cb_k (b_k bits): k_codes [B][Hkv][T][d/32][b_k], k_norms [B][Hkv][T],
+ *           k_signs and k_gammas NULL; or Algorithm 2 with cb_k the (b_k-1)-bit codebook (1..2 bits):
+ *           k_codes [B][Hkv][T][d/32][b_k-1], k_signs [B][Hkv][T][d/32], k_norms, k_gammas
+ *           [B][Hkv][T]. Algorithm 2 keys give the unbiased inner-product estimate
+ *           <q, k_hat> = n (<Pi q, c[idx]> + alpha gamma <S q, 2z - 1>) (aiboss88 page, QJL stage).
  *   values  Algorithm 2 with cb_v the (b_v-1)-bit codebook: v_codes [B][Hkv][T][d/32][b_v-1],
  *           v_signs [B][Hkv][T][d/32], v_norms, v_gammas [B][Hkv][T];
  *           or Algorithm 1 (v_signs and v_gammas NULL, cb_v the b_v-bit codebook)
@@ -191,7 +195,8 @@ TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int6
  * ws: caller device workspace of at least tq_attend_workspace_bytes(...) bytes. */
 TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq, int32_t Hkv,
                            int64_t T, int32_t d, const void* q, int32_t q_dtype, const void* rot,
-                           const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* v_codes,
+                           const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                           const uint16_t* k_gammas, const uint32_t* v_codes,
                            const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
                            float* out, void* ws, size_t ws_bytes, void* stream);
 
@@ -242,8 +247,9 @@ TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_codebook* cb
 TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
                                    int32_t Hkv, int64_t T, int32_t d, const void* q, int32_t q_dtype,
                                    const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
-                                   const uint32_t* v_codes, const uint32_t* v_signs, const uint16_t* v_norms,
-                                   const uint16_t* v_gammas, float scale, float* out, void* stream);
+                                   const uint32_t* k_signs, const uint16_t* k_gammas, const uint32_t* v_codes,
+                                   const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas,
+                                   float scale, float* out, void* stream);
 
 /* Synchronises `stream`, then reports a pending CUDA error (TQ_ERR_CUDA) or a device-side
  * timeout recorded by any libtq kernel since the last check (TQ_ERR_DEVICE_TIMEOUT, which this

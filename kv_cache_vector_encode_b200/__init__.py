@@ -70,10 +70,10 @@ _SIGNATURES = {
     "tq_scores_workspace_bytes": (_SZ, [_I64, _I64, _I32, _I32]),
     "tq_scores": (_I32, [_CB, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tq_attend_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
-    "tq_attend_decode": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P,
-                                _F, _P, _P, _SZ, _P]),
+    "tq_attend_decode": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
+                                _P, _F, _P, _P, _SZ, _P]),
     "tq_attend_decode_noalloc": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
-                                        _P, _F, _P, _P]),
+                                        _P, _P, _P, _F, _P, _P]),
     "tq_attend_append_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32, _I32, _I32]),
     "tq_attend_append": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I64, _I32, _P, _I32, _P, _P, _I32, _P, _P, _P,
                                 _P, _P, _P, _P, _F, _P, _P, _SZ, _P]),
@@ -219,7 +219,7 @@ def tq_attend_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int) -> int:
 
 
 def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
-                     v_signs=None, v_gammas=None, scale=None, ws=None, stream=None):
+                     v_signs=None, v_gammas=None, scale=None, ws=None, stream=None, k_signs=None, k_gammas=None):
     import math
     import torch
     B, Hq, d = q.shape
@@ -232,6 +232,8 @@ def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v
     _check(lib().tq_attend_decode(ctypes.byref(cb_k), ctypes.byref(cb_v), B, Hq, Hkv, T, d,
                                   _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q), _ptr(rot, "rot"),
                                   _ptr(k_codes, "k_codes", [torch.int32]), _ptr(k_norms, "k_norms", [torch.float16]),
+                                  _ptr(k_signs, "k_signs", [torch.int32], True),
+                                  _ptr(k_gammas, "k_gammas", [torch.float16], True),
                                   _ptr(v_codes, "v_codes", [torch.int32]),
                                   _ptr(v_signs, "v_signs", [torch.int32], True),
                                   _ptr(v_norms, "v_norms", [torch.float16]),
@@ -240,7 +242,7 @@ def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v
 
 
 def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
-                             v_signs=None, v_gammas=None, scale=None, stream=None):
+                             v_signs=None, v_gammas=None, scale=None, stream=None, k_signs=None, k_gammas=None):
     """tq_attend_decode with the library's fixed scratch array (no workspace, no allocation)."""
     import math
     import torch
@@ -252,6 +254,8 @@ def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_
                                           _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q), _ptr(rot, "rot"),
                                           _ptr(k_codes, "k_codes", [torch.int32]),
                                           _ptr(k_norms, "k_norms", [torch.float16]),
+                                          _ptr(k_signs, "k_signs", [torch.int32], True),
+                                          _ptr(k_gammas, "k_gammas", [torch.float16], True),
                                           _ptr(v_codes, "v_codes", [torch.int32]),
                                           _ptr(v_signs, "v_signs", [torch.int32], True),
                                           _ptr(v_norms, "v_norms", [torch.float16]),

@@ -72,7 +72,7 @@ struct AttParams {
   int64_t tstride;               // token slots per slice in the cache arrays (>= T)
   int slices, nchunk, per_cta, maxseg;
   int nst;                       // depth of the packed-chunk ring
-  int bk, mk;                    // key bits, key Walsh planes
+  int bk, mk, ksign;             // key codebook bits, key Walsh planes, key sign plane (Algorithm 2 keys)?
   int bv, mv, vsign, np;         // value codebook bits, value Walsh planes, sign plane?, planes
   int nq;                        // MMA N of the scores / of one value weight kind (16 or 32)
   float beta_k[4], beta_v[4];
@@ -83,12 +83,14 @@ struct AttParams {
   const float* S;
   const uint32_t* k_codes;
   const uint16_t* k_norms;
+  const uint32_t* k_signs;       // Algorithm 2 keys only (else NULL)
+  const uint16_t* k_gammas;
   const uint32_t* v_codes;
   const uint32_t* v_signs;
   const uint16_t* v_norms;
   const uint16_t* v_gammas;
-  uint8_t* bq_img;               // [slices][nq rows x mk*d bytes] K-major SW128 image
-  float* head_c;                 // [slices][8][2]: 2^-F, Q_h * sum beta
+  uint8_t* bq_img;               // [slices][nq rows x (mk + ksign) d bytes] K-major SW128 image
+  float* head_c;                 // [slices][8][4]: 2^-F, Q_h * sum beta, 2^-F'', Q''_h
   float* partial;                // [slices][maxseg][Hg][att_rec(d)]
   float* out;
   uint32_t* err;
@@ -107,8 +109,8 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   const int d = p.d, i = threadIdx.x;            // coordinate (128 threads)
   const int warp = i >> 5, lane = i & 31;
   __shared__ __align__(16) float sq[8][128];
-  __shared__ double red[4][8][2];
-  const int kbytes = p.mk * d;
+  __shared__ double red[4][8][4];
+  const int kbytes = (p.mk + p.ksign) * d;
   uint8_t* img = p.bq_img + (size_t)slice * p.nq * kbytes;
   for (int o = i; o < p.nq * kbytes / 16; o += blockDim.x) ((uint4*)img)[o] = make_uint4(0, 0, 0, 0);
   for (int h = 0; h < p.Hg; ++h) {
@@ -119,12 +121,15 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   __syncthreads();
   // q'_h[i] = sum_j Pi[i][j] q_h[j] for every head: one thread per output coordinate, its row of Pi
   // read as float4, fp64 accumulation (one independent chain per head)
-  double acc[8];
+  // (q''_h = S q_h the same way, for Algorithm 2 keys)
+  double acc[8], acc2[8];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) acc[h] = 0.0;
+  for (int h = 0; h < 8; ++h) acc[h] = acc2[h] = 0.0;
   const float4* row = (const float4*)(p.Pi + (size_t)i * d);
+  const float4* srow = (const float4*)(p.S + (size_t)i * d);
   for (int j4 = 0; j4 < d / 4; ++j4) {
     const float4 pv = __ldg(row + j4);
+    const float4 sv = p.ksign ? __ldg(srow + j4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       if (h < p.Hg) {
@@ -133,6 +138,12 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
         acc[h] = fma((double)pv.y, (double)qv.y, acc[h]);
         acc[h] = fma((double)pv.z, (double)qv.z, acc[h]);
         acc[h] = fma((double)pv.w, (double)qv.w, acc[h]);
+        if (p.ksign) {
+          acc2[h] = fma((double)sv.x, (double)qv.x, acc2[h]);
+          acc2[h] = fma((double)sv.y, (double)qv.y, acc2[h]);
+          acc2[h] = fma((double)sv.z, (double)qv.z, acc2[h]);
+          acc2[h] = fma((double)sv.w, (double)qv.w, acc2[h]);
+        }
       }
     }
   }
@@ -145,15 +156,19 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
 #pragma unroll
   for (int h = 0; h < 8; ++h) {
     if (h < p.Hg) {
-      double sm = acc[h], mx = fabs(acc[h]) * bmax;
+      double sm = acc[h], mx = fabs(acc[h]) * bmax, sm2 = acc2[h], mx2 = fabs(acc2[h]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         sm += __shfl_xor_sync(0xffffffffu, sm, o);
         mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        sm2 += __shfl_xor_sync(0xffffffffu, sm2, o);
+        mx2 = fmax(mx2, __shfl_xor_sync(0xffffffffu, mx2, o));
       }
       if (lane == 0) {
         red[warp][h][0] = sm;
         red[warp][h][1] = mx;
+        red[warp][h][2] = sm2;
+        red[warp][h][3] = mx2;
       }
     }
   }
@@ -170,14 +185,26 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
       frexp(vmax, &E);              // vmax < 2^E
       F = 30 - E;                   // vmax * 2^F < 2^30
     }
+    // q'' of Algorithm 2 keys: fixed point 2^F2 with max |q''| 2^F2 < 2^30
+    const double Q2 = (red[0][h][2] + red[1][h][2]) + (red[2][h][2] + red[3][h][2]);
+    const double vmax2 = fmax(fmax(red[0][h][3], red[1][h][3]), fmax(red[2][h][3], red[3][h][3]));
+    int F2 = 0;
+    if (vmax2 > 0.0) {
+      int E;
+      frexp(vmax2, &E);
+      F2 = 30 - E;
+    }
     if (i == 0) {
-      p.head_c[(slice * 8 + h) * 2 + 0] = (float)ldexp(1.0, -F);
-      p.head_c[(slice * 8 + h) * 2 + 1] = (float)(Qh * sb);
+      p.head_c[(slice * 8 + h) * 4 + 0] = (float)ldexp(1.0, -F);
+      p.head_c[(slice * 8 + h) * 4 + 1] = (float)(Qh * sb);
+      p.head_c[(slice * 8 + h) * 4 + 2] = (float)ldexp(1.0, -F2);
+      p.head_c[(slice * 8 + h) * 4 + 3] = (float)Q2;
     }
     const int g = i >> 5, rr = i & 31, jj = rr >> 3, s = rr & 7;   // coordinate 32g + 8jj + s
     const int kin = 32 * g + 4 * s + jj;                          // its k index inside a plane
-    for (int S = 0; S < p.mk; ++S) {
-      long long v = llrint(ldexp((double)p.beta_k[S] * qi, F - s));
+    for (int S = 0; S < p.mk + p.ksign; ++S) {
+      // the Walsh planes carry beta_S q'; the key sign plane (last) carries q''
+      long long v = S < p.mk ? llrint(ldexp((double)p.beta_k[S] * qi, F - s)) : llrint(ldexp(acc2[h], F2 - s));
       const int k = S * d + kin;
       for (int l = 0; l < 4; ++l) {
         const long long dl = l < 3 ? (((v + 128) & 255) - 128) : v;   // balanced signed digits
@@ -192,7 +219,7 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
 // main kernel
 // ------------------------------------------------------------------------------------------------
 struct AttLayout {
-  uint32_t kc_bytes, vc_bytes, sg_off, stage_bytes;
+  uint32_t kc_bytes, vc_bytes, sg_off, ks_off, stage_bytes;
   uint32_t off_stage, av_bytes, off_av, bw_kind, bw_buf, off_bw, bq_bytes, off_bq, off_sc, off_red, off_sum,
       off_bar, total;
 };
@@ -204,7 +231,8 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.kc_bytes = kChunk * p.G * p.bk * 4;
   L.sg_off = L.kc_bytes + kChunk * p.G * p.bv * 4;     // sign words of the chunk
   L.vc_bytes = kChunk * p.G * (p.bv + (p.vsign ? 1 : 0)) * 4;
-  L.stage_bytes = aru(L.kc_bytes + L.vc_bytes, 1024);
+  L.ks_off = L.kc_bytes + L.vc_bytes;                 // key sign words (Algorithm 2 keys)
+  L.stage_bytes = aru(L.ks_off + (p.ksign ? kChunk * p.G * 4 : 0), 1024);
   uint32_t off = 0;
   L.off_stage = off; off += nst * L.stage_bytes;
   L.av_bytes = kChunk * 128;                       // one plane: 128 tokens x 128 coordinates
@@ -212,7 +240,7 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.bw_kind = (p.nq / 16) * kChunk * 16;           // one weight kind: nq/16 blocks of 128 x 16 bytes
   L.bw_buf = 2 * L.bw_kind;                        // kinds: w, w * gamma
   L.off_bw = off; off += 2 * L.bw_buf;
-  L.bq_bytes = aru(p.nq * p.mk * p.d, 1024);
+  L.bq_bytes = aru(p.nq * (p.mk + p.ksign) * p.d, 1024);
   L.off_bq = off; off += 2 * L.bq_bytes;
   L.off_sc = off; off += 4 * 64 * 4;               // chunk scalars, 4-deep ring of 64 floats
   L.off_red = off; off += 2 * 4 * 16 * 4;          // max exchange of the softmax warps: [group][warp][16]
@@ -237,10 +265,9 @@ enum ABars {
   ANBARS = SCAL_FULL + 4
 };
 
-// TMEM columns: A_K [2][128] at 0, scores [2][nq] at 256, value accumulators [2][np][nq] from
-// 256 + 2 nq (at most 512 columns in all: np <= 3, nq <= 32).
-constexpr uint32_t kAK0 = 0;
-constexpr uint32_t kDS0 = 256;
+// TMEM columns: A_K [2][32 (mk + ksign)] at 0, scores [2][nq (1 + ksign)] after them, value
+// accumulators [2][np][nq] after those (at most 512 columns: mk + ksign <= 4 and with a key sign
+// plane mk <= 2).
 
 // Walks this CTA's chunks in order (slice, chunk inside the slice, segment ordinal) without
 // integer division.
@@ -330,16 +357,21 @@ __device__ __forceinline__ void expand_v_rows(const AttParams& p, const AttLayou
   }
 }
 
-// HG: query heads per KV head (4 or 8, Hg <= HG); BK: key bits; BV: value codebook bits;
-// VS: value sign plane (Algorithm 2 values)
-template <int HG, int BK, int BV, int VS>
+// HG: query heads per KV head (4 or 8, Hg <= HG); BK: key codebook bits; BV: value codebook bits;
+// VS: value sign plane (Algorithm 2 values); KS: key sign plane (Algorithm 2 keys, BK <= 2)
+template <int HG, int BK, int BV, int VS, int KS>
 __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const __grid_constant__ AttParams p) {
   constexpr bool SPLITV = att_split_v(HG);
   constexpr int MK = walsh_count(BK);
+  constexpr int MKT = MK + KS;                   // key operand planes (Walsh planes, sign plane)
   constexpr int MV = walsh_count(BV);
+  static_assert(MKT <= 4, "key planes exceed the TMEM budget");
+  constexpr uint32_t kAK0 = 0, AKS = 32 * MKT;   // key operand buffers [2][AKS columns]
+  constexpr uint32_t kDS0 = 2 * AKS;             // scores [2][NQS]
   constexpr int NP = MV + VS;
   constexpr int NQ = HG <= 4 ? 16 : 32;
-  constexpr int KSTEPS = MK * 128 / 32;
+  constexpr int NQS = NQ * (1 + KS);            // score columns: Walsh part, then (KS) sign part
+  constexpr int KSTEPS = MK * 128 / 32;          // K steps of the Walsh planes (the sign plane adds 4)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nst = p.nst;
@@ -357,7 +389,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   const int nmy = max(0, c_end - c_begin);
   const int d = p.d, G = p.G;
   const int64_t T = p.T, TS = p.tstride;
-  const uint32_t dv0 = kDS0 + 2 * NQ;
+  const uint32_t dv0 = kDS0 + 2 * NQS;
   const uint32_t dv_cols = NP * NQ;
   // tokens in the last chunk of every slice (all other chunks are full)
   const int tail = (int)(T - (int64_t)(p.nchunk - 1) * kChunk);
@@ -396,7 +428,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   if (warp == 0) {
     // ------------------------------------ producer -------------------------------------------------
     // warp-uniform schedule; one elected lane issues the copies
-    const uint32_t nb = (uint32_t)(NQ * MK * d);
+    const uint32_t nb = (uint32_t)(NQ * MKT * d);
     for (int c = 0; c < nmy; ++c, it.next()) {
       if (c == 0 || it.cis == 0) {
         const int sg = it.seg;
@@ -415,12 +447,14 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       const uint32_t kb = (uint32_t)tc * G * BK * 4;
       const uint32_t vb = (uint32_t)tc * G * BV * 4;
       const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
+      const uint32_t kgb = KS ? (uint32_t)tc * G * 4 : 0u;
       uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
       if (elect_one_sync()) {
-        mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb);
+        mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb + kgb);
         bulk_g2s(stg, p.k_codes + vec0 * G * BK, kb, &bar[ST_FULL + st]);
         bulk_g2s(stg + Lo.kc_bytes, p.v_codes + vec0 * G * BV, vb, &bar[ST_FULL + st]);
         if (VS) bulk_g2s(stg + Lo.sg_off, p.v_signs + vec0 * G, sb, &bar[ST_FULL + st]);
+        if (KS) bulk_g2s(stg + Lo.ks_off, p.k_signs + vec0 * G, kgb, &bar[ST_FULL + st]);
       }
       __syncwarp();
     }
@@ -443,14 +477,17 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         break;
       tc_fence_after();
       const uint64_t dq = dq0 + (((sg & 1) * Lo.bq_bytes) >> 4);
-      const uint32_t ak = tbase + kAK0 + b * 128;
-      const uint32_t ds = tbase + kDS0 + b * NQ;
+      const uint32_t ak = tbase + kAK0 + b * AKS;
+      const uint32_t ds = tbase + kDS0 + b * NQS;
       const bool last = c == nmy - 1 || it.cis == p.nchunk - 1;
       if (elect_one_sync()) {
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) {
+        for (int ks = 0; ks < KSTEPS + 4 * KS; ++ks) {
+          // the sign plane's steps (ks >= KSTEPS) accumulate into their own columns
           const uint32_t kbyte = ks * 32, blk = kbyte >> 7, inb = kbyte & 127;
-          mma_i8_ts(ds, ak + ks * 8, dq + ((blk * NQ * 128 + inb) >> 4), id_s, ks > 0);
+          const bool sgn = ks >= KSTEPS;
+          mma_i8_ts(ds + (sgn ? NQ : 0), ak + ks * 8, dq + ((blk * NQ * 128 + inb) >> 4), id_s,
+                    sgn ? ks > KSTEPS : ks > 0);
         }
         mma_commit(&bar[SC_DONE + b]);
         if (last) mma_commit(&bar[BQ_EMPTY + (sg & 1)]);
@@ -469,20 +506,21 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
     float* rgrp = red + gq * 64;
-    float mrun[HH], ha[HH], hb[HH];
+    float mrun[HH], ha[HH], hb[HH], hs[HH], hq[HH];
     float vmax_run = 0.0f, gmax_run = 0.0f, sw = 1.0f, sw2 = 1.0f, isw = 1.0f, isw2 = 1.0f;
     bool ok = true;
     // fp16 norms of the next chunk, loaded one chunk ahead and converted only when used (dead
     // tokens read as zero)
-    uint16_t nk_n = 0, nv_n = 0, gm_n = 0;
+    uint16_t nk_n = 0, nv_n = 0, gm_n = 0, gk_n = 0;
     ChunkIter nx = it;                              // position of the chunk whose norms are prefetched
     auto load_norms = [&]() {
-      nk_n = nv_n = gm_n = 0;
+      nk_n = nv_n = gm_n = gk_n = 0;
       if (t < (nx.cis == p.nchunk - 1 ? tail : kChunk)) {
         const int64_t rec = (int64_t)nx.slice * TS + (int64_t)nx.cis * kChunk + t;
         nk_n = __ldg(p.k_norms + rec);
         nv_n = __ldg(p.v_norms + rec);
         if (VS) gm_n = __ldg(p.v_gammas + rec);
+        if (KS) gk_n = __ldg(p.k_gammas + rec);
       }
     };
     if (nmy > 0) load_norms();
@@ -490,6 +528,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       const int b = c & 1;
       const float nk = __half2float(__ushort_as_half(nk_n)), nv = __half2float(__ushort_as_half(nv_n));
       const float gm = VS ? __half2float(__ushort_as_half(gm_n)) : 0.0f;
+      const float gk = KS ? __half2float(__ushort_as_half(gk_n)) : 0.0f;
       const bool live = t < (it.cis == p.nchunk - 1 ? tail : kChunk);
       if (c + 1 < nmy) {
         nx.next();
@@ -497,21 +536,28 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       }
       if (c == 0 || it.cis == 0) {
         vmax_run = gmax_run = 0.0f;
-        const float2* hc = (const float2*)(p.head_c + it.slice * 16);
+        const float4* hc = (const float4*)(p.head_c + it.slice * 32);
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           mrun[i] = -INFINITY;
-          const float2 x = h0 + i < Hg ? __ldg(hc + h0 + i) : make_float2(0.0f, 0.0f);
+          const float4 x = h0 + i < Hg ? __ldg(hc + h0 + i) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
           ha[i] = -2.0f * x.x * p.scale_log2e;
           hb[i] = x.y * p.scale_log2e;
+          // key sign term alpha gamma <q'', 2z - 1> = alpha gamma (2 2^-F'' D_z - Q'')
+          hs[i] = 2.0f * p.alpha * x.z * p.scale_log2e;
+          hq[i] = -p.alpha * x.w * p.scale_log2e;
         }
       }
       ok = mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
       tc_fence_after();
-      uint32_t dsr[4 * HH];
-      const uint32_t scol = tbase + lane_base + kDS0 + b * NQ + 4 * h0;
+      uint32_t dsr[4 * HH], dzr[KS ? 4 * HH : 1];
+      const uint32_t scol = tbase + lane_base + kDS0 + b * NQS + 4 * h0;
       if (HH == 2) tmem_ld8(scol, *(uint32_t(*)[8]) & dsr[0]);
       else tmem_ld16(scol, *(uint32_t(*)[16]) & dsr[0]);
+      if (KS) {
+        if (HH == 2) tmem_ld8(scol + NQ, *(uint32_t(*)[8]) & dzr[0]);
+        else tmem_ld16(scol + NQ, *(uint32_t(*)[16]) & dzr[0]);
+      }
       tmem_ld_wait();
       tc_fence_before();
       float lg[HH];
@@ -522,7 +568,14 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         const float dot = fmaf(fmaf(fmaf(small_i2f((int)dsr[4 * i + 3]), 256.0f, small_i2f((int)dsr[4 * i + 2])), 256.0f,
                                     small_i2f((int)dsr[4 * i + 1])),
                                256.0f, small_i2f((int)dsr[4 * i]));
-        lg[i] = (h0 + i < Hg && live) ? nk * fmaf(ha[i], dot, hb[i]) : -INFINITY;
+        float sc = fmaf(ha[i], dot, hb[i]);
+        if (KS) {
+          const float dz = fmaf(fmaf(fmaf(small_i2f((int)dzr[4 * i + 3]), 256.0f, small_i2f((int)dzr[4 * i + 2])),
+                                     256.0f, small_i2f((int)dzr[4 * i + 1])),
+                                256.0f, small_i2f((int)dzr[4 * i]));
+          sc = fmaf(gk, fmaf(hs[i], dz, hq[i]), sc);
+        }
+        lg[i] = (h0 + i < Hg && live) ? nk * sc : -INFINITY;
         up = up || lg[i] > mrun[i];
       }
       float corr[HH];
@@ -645,7 +698,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         kw[4 * v4 + 2] = x.z;
         kw[4 * v4 + 3] = x.w;
       }
-      const uint32_t ak = tbase + lane_base + kAK0 + b * 128;
+      const uint32_t ak = tbase + lane_base + kAK0 + b * AKS;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
 #pragma unroll
@@ -659,6 +712,18 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) r[s8] = w & (0x01010101u << s8);
           tmem_st8(ak + S * 32 + g * 8, r);
+        }
+      }
+      if (KS) {
+        // the key sign plane z (Algorithm 2 keys) after the Walsh planes
+        const uint4 x = *(const uint4*)(stg + Lo.ks_off + t * 16);
+        const uint32_t zw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t r[8];
+#pragma unroll
+          for (int s8 = 0; s8 < 8; ++s8) r[s8] = zw[g] & (0x01010101u << s8);
+          tmem_st8(ak + MK * 32 + g * 8, r);
         }
       }
       // the key planes are complete once this warp's TMEM stores are
@@ -906,19 +971,20 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
 
 using MainKernel = void (*)(AttParams);
 
-template <int HG, int BK>
+template <int HG, int BK, int KS>
 MainKernel pick_v(int bv, int vs) {
-  if (bv == 1) return vs ? attend_main_kernel<HG, BK, 1, 1> : attend_main_kernel<HG, BK, 1, 0>;
-  return vs ? attend_main_kernel<HG, BK, 2, 1> : attend_main_kernel<HG, BK, 2, 0>;
+  if (bv == 1) return vs ? attend_main_kernel<HG, BK, 1, 1, KS> : attend_main_kernel<HG, BK, 1, 0, KS>;
+  return vs ? attend_main_kernel<HG, BK, 2, 1, KS> : attend_main_kernel<HG, BK, 2, 0, KS>;
 }
 template <int HG>
-MainKernel pick_k(int bk, int bv, int vs) {
-  if (bk == 1) return pick_v<HG, 1>(bv, vs);
-  if (bk == 2) return pick_v<HG, 2>(bv, vs);
-  return pick_v<HG, 3>(bv, vs);
+MainKernel pick_k(int bk, int bv, int vs, int ks) {
+  if (ks) return bk == 1 ? pick_v<HG, 1, 1>(bv, vs) : pick_v<HG, 2, 1>(bv, vs);   // key codebooks <= 2 bits
+  if (bk == 1) return pick_v<HG, 1, 0>(bv, vs);
+  if (bk == 2) return pick_v<HG, 2, 0>(bv, vs);
+  return pick_v<HG, 3, 0>(bv, vs);
 }
-MainKernel pick_main(int hg, int bk, int bv, int vs) {
-  return hg <= 4 ? pick_k<4>(bk, bv, vs) : pick_k<8>(bk, bv, vs);
+MainKernel pick_main(int hg, int bk, int bv, int vs, int ks) {
+  return hg <= 4 ? pick_k<4>(bk, bv, vs, ks) : pick_k<8>(bk, bv, vs, ks);
 }
 
 struct AttPlan {
@@ -975,13 +1041,16 @@ namespace tq {
 // Decode attention over T tokens of every slice, whose records lie tstride apart (tstride >= T).
 tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
                       int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
-                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* v_codes,
-                      const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
-                      float* out, void* ws, size_t ws_bytes, void* stream) {
+                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                      const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
+                      const uint16_t* v_norms, const uint16_t* v_gammas, float scale, float* out, void* ws,
+                      size_t ws_bytes, void* stream) {
   if (!cb_k || !cb_v || !q || !rot || !k_codes || !k_norms || !v_codes || !v_norms || !out || !ws)
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": NULL pointer");
   if ((v_signs == nullptr) != (v_gammas == nullptr))
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": v_signs and v_gammas must both be NULL or both be set");
+  if ((k_signs == nullptr) != (k_gammas == nullptr))
+    return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": k_signs and k_gammas must both be NULL or both be set");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || Hq % Hkv)
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": bad B / Hq / Hkv / T");
   if (tstride < T) return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": fewer cache slots than tokens");
@@ -991,6 +1060,9 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   if (cb_k->d != d || cb_v->d != d) return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": codebook d mismatch");
   if (cb_k->bits < 1 || cb_k->bits > 3)
     return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": key codebooks of 1..3 bits are supported");
+  const bool ksign = k_signs != nullptr;
+  if (ksign && cb_k->bits > 2)
+    return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": Algorithm 2 keys need a key codebook of 1..2 bits");
   const bool vsign = v_signs != nullptr;
   if (cb_v->bits < 1 || cb_v->bits > 2)   // value planes (Walsh planes + sign) must fit three MMA operand slots
     return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": value codebooks of 1..2 bits are supported");
@@ -1001,7 +1073,8 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
       if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": codebook not symmetric");
   }
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, std::string(f) + ": q dtype");
-  if (!aligned16(k_codes) || !aligned16(v_codes) || (vsign && !aligned16(v_signs)) || !aligned16(ws) ||
+  if (!aligned16(k_codes) || !aligned16(v_codes) || (vsign && !aligned16(v_signs)) || (ksign && !aligned16(k_signs)) ||
+      !aligned16(ws) ||
       !aligned16(rot) || !aligned16(out))
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": pointers must be 16-byte aligned");
   AttPlan pl;
@@ -1013,6 +1086,7 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   int kmask[8], vmask[8];
   float kbeta[8], vbeta[8];
   p.bk = cb_k->bits;
+  p.ksign = ksign ? 1 : 0;
   p.mk = walsh_planes(cb_k, kmask, kbeta);
   for (int i = 0; i < p.mk; ++i) p.beta_k[i] = kbeta[i];
   p.bv = cb_v->bits;
@@ -1029,6 +1103,8 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   p.S = (const float*)((const char*)rot + RL.s32);
   p.k_codes = k_codes;
   p.k_norms = k_norms;
+  p.k_signs = k_signs;
+  p.k_gammas = k_gammas;
   p.v_codes = v_codes;
   p.v_signs = v_signs;
   p.v_norms = v_norms;
@@ -1049,7 +1125,7 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   cudaError_t e;
   attend_prep_kernel<<<p.slices, 128, 0, st>>>(p);
   const AttLayout Lo = att_layout(p, nst);
-  const MainKernel kern = pick_main(p.Hg, p.bk, p.bv, p.vsign);
+  const MainKernel kern = pick_main(p.Hg, p.bk, p.bv, p.vsign, p.ksign);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode: shared memory attribute");
   const long long totalc = (long long)p.slices * p.nchunk;
@@ -1064,10 +1140,11 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
 extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
                                              int32_t Hkv, int64_t T, int32_t d, const void* q, int32_t q_dtype,
                                              const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
+                                             const uint32_t* k_signs, const uint16_t* k_gammas,
                                              const uint32_t* v_codes, const uint32_t* v_signs, const uint16_t* v_norms,
                                              const uint16_t* v_gammas, float scale, float* out, void* ws,
                                              size_t ws_bytes, void* stream) {
   clear_error();
-  return attend_impl("tq_attend_decode", cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, v_codes,
-                     v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream);
+  return attend_impl("tq_attend_decode", cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs,
+                     k_gammas, v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream);
 }

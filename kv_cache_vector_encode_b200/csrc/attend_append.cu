@@ -107,5 +107,6 @@ extern "C" TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_c
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_append: scatter launch");
   return attend_impl("tq_attend_append", cb_k, cb_v, B, Hq, Hkv, T_cur + 1, T_max, d, q, q_dtype, rot, k_codes,
-                     k_norms, v_codes, v_signs, v_norms, v_gammas, scale, out, base + w.att, w.kc - w.att, stream);
+                     k_norms, nullptr, nullptr, v_codes, v_signs, v_norms, v_gammas, scale, out, base + w.att,
+                     w.kc - w.att, stream);
 }

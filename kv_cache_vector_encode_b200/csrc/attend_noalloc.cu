@@ -48,7 +48,8 @@ tq_status scratch_for(int dev, void** out) {
 extern "C" TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B,
                                                      int32_t Hq, int32_t Hkv, int64_t T, int32_t d, const void* q,
                                                      int32_t q_dtype, const void* rot, const uint32_t* k_codes,
-                                                     const uint16_t* k_norms, const uint32_t* v_codes,
+                                                     const uint16_t* k_norms, const uint32_t* k_signs,
+                                                     const uint16_t* k_gammas, const uint32_t* v_codes,
                                                      const uint32_t* v_signs, const uint16_t* v_norms,
                                                      const uint16_t* v_gammas, float scale, float* out,
                                                      void* stream) {
@@ -69,6 +70,7 @@ extern "C" TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, co
   const tq_status s = scratch_for(dev, &scratch);
   if (s != TQ_OK) return s;
   // sizes too small to be valid (need == 0) are reported by tq_attend_decode's own checks
-  return tq_attend_decode(cb_k, cb_v, B, Hq, Hkv, T, d, q, q_dtype, rot, k_codes, k_norms, v_codes, v_signs,
-                          v_norms, v_gammas, scale, out, scratch, (size_t)TQ_ATTEND_NOALLOC_MAX_BYTES, stream);
+  return tq_attend_decode(cb_k, cb_v, B, Hq, Hkv, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas,
+                          v_codes, v_signs, v_norms, v_gammas, scale, out, scratch,
+                          (size_t)TQ_ATTEND_NOALLOC_MAX_BYTES, stream);
 }

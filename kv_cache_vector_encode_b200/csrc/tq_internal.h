@@ -71,8 +71,9 @@ bool make_tmap_2d_sw128(void* tmap, const void* base, int esize, uint64_t cols, 
 // whose slices hold tstride >= T slots (attend.cu); tq_attend_decode is the case tstride = T.
 tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
                       int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
-                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* v_codes,
-                      const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
-                      float* out, void* ws, size_t ws_bytes, void* stream);
+                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                      const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
+                      const uint16_t* v_norms, const uint16_t* v_gammas, float scale, float* out, void* ws,
+                      size_t ws_bytes, void* stream);
 
 }  // namespace tq

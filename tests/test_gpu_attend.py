@@ -28,7 +28,7 @@ def dev(gpu_required):
     return torch.device("cuda")
 
 
-def make_cache(B, Hkv, T, d, kb, vb, v_alg2, dev, n_outlier=3, sigma=0.5, seed=0):
+def make_cache(B, Hkv, T, d, kb, vb, v_alg2, dev, n_outlier=3, sigma=0.5, seed=0, k_alg2=False):
     Pi, S = W.rotation(d), W.jl_matrix(d)
     rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
     K = np.stack([W.kv_block(Hkv, T, d, n_outlier, 20.0, sigma, seed=seed, tag=W.TAG_K, batch_index=b)
@@ -36,9 +36,15 @@ def make_cache(B, Hkv, T, d, kb, vb, v_alg2, dev, n_outlier=3, sigma=0.5, seed=0
     V = np.stack([W.kv_block(Hkv, T, d, n_outlier, 20.0, sigma, seed=seed, tag=W.TAG_V, batch_index=b)
                   for b in range(B)])
     n = B * Hkv * T
-    cbk = tq.tq_codebook_init(d, kb)
-    kc, kn = tq.empty_mse(n, d, kb)
-    tq.tq_encode_mse(cbk, torch.from_numpy(K.reshape(n, d)).to(dev).to(torch.bfloat16), rot, kc, kn)
+    if k_alg2:
+        cbk = tq.tq_codebook_init(d, kb - 1)
+        kc, ks, kn, kg = tq.empty_prod(n, d, kb)
+        tq.tq_encode_prod(cbk, torch.from_numpy(K.reshape(n, d)).to(dev).to(torch.bfloat16), rot, kc, ks, kn, kg)
+    else:
+        cbk = tq.tq_codebook_init(d, kb)
+        kc, kn = tq.empty_mse(n, d, kb)
+        ks = kg = None
+        tq.tq_encode_mse(cbk, torch.from_numpy(K.reshape(n, d)).to(dev).to(torch.bfloat16), rot, kc, kn)
     if v_alg2:
         cbv = tq.tq_codebook_init(d, vb - 1)
         vc, vs, vn, vg = tq.empty_prod(n, d, vb)
@@ -49,17 +55,22 @@ def make_cache(B, Hkv, T, d, kb, vb, v_alg2, dev, n_outlier=3, sigma=0.5, seed=0
         vs = vg = None
         tq.tq_encode_mse(cbv, torch.from_numpy(V.reshape(n, d)).to(dev).to(torch.bfloat16), rot, vc, vn)
     tq.tq_sync_check()
-    return dict(Pi=Pi, S=S, rot=rot, cbk=cbk, cbv=cbv, kc=kc, kn=kn, vc=vc, vs=vs, vn=vn, vg=vg,
-                n=n, kb=kb, vb=vb, v_alg2=v_alg2)
+    return dict(Pi=Pi, S=S, rot=rot, cbk=cbk, cbv=cbv, kc=kc, kn=kn, ks=ks, kg=kg, vc=vc, vs=vs, vn=vn, vg=vg,
+                n=n, kb=kb, vb=vb, v_alg2=v_alg2, k_alg2=k_alg2)
 
 
 def oracle_attention(cache, q, B, Hq, Hkv, T, d, slices=None):
     Pi, S = cache["Pi"], cache["S"]
     n = cache["n"]
     kb, vb = cache["kb"], cache["vb"]
-    okb = lloyd_max(d, kb)
+    k_alg2 = cache.get("k_alg2", False)
+    kbits = kb - 1 if k_alg2 else kb
+    okb = lloyd_max(d, kbits)
     ovb = lloyd_max(d, vb - 1) if cache["v_alg2"] else lloyd_max(d, vb)
-    kc = np_u32(cache["kc"]).reshape(B, Hkv, T, d // 32, kb)
+    kc = np_u32(cache["kc"]).reshape(B, Hkv, T, d // 32, kbits)
+    if k_alg2:
+        ks = np_u32(cache["ks"]).reshape(B, Hkv, T, d // 32)
+        kg = np_f16(cache["kg"]).reshape(B, Hkv, T)
     kn = np_f16(cache["kn"]).reshape(B, Hkv, T)
     vbits = vb - 1 if cache["v_alg2"] else vb
     vc = np_u32(cache["vc"]).reshape(B, Hkv, T, d // 32, vbits)
@@ -70,7 +81,10 @@ def oracle_attention(cache, q, B, Hq, Hkv, T, d, slices=None):
     grp = Hq // Hkv
     out = {}
     for (b, hk) in (slices or [(b, hk) for b in range(B) for hk in range(Hkv)]):
-        kh = Q.decode(kc[b, hk], kn[b, hk], Pi, okb)
+        if k_alg2:
+            kh = Q.decode(kc[b, hk], kn[b, hk], Pi, okb, ks[b, hk], kg[b, hk], S)
+        else:
+            kh = Q.decode(kc[b, hk], kn[b, hk], Pi, okb)
         if cache["v_alg2"]:
             vh = Q.decode(vc[b, hk], vn[b, hk], Pi, ovb, vs[b, hk], vg[b, hk], S)
         else:
@@ -87,7 +101,7 @@ def run_attend(cache, q_np, B, Hq, Hkv, T, d, dev):
     n = cache["n"]
     tq.tq_attend_decode(cache["cbk"], cache["cbv"], q, cache["rot"],
                         cache["kc"], cache["kn"].view(B, Hkv, T), cache["vc"], cache["vn"].view(B, Hkv, T), out,
-                        v_signs=cache["vs"], v_gammas=cache["vg"])
+                        v_signs=cache["vs"], v_gammas=cache["vg"], k_signs=cache.get("ks"), k_gammas=cache.get("kg"))
     tq.tq_sync_check()
     return out.cpu().numpy()
 
@@ -114,4 +128,18 @@ def test_attend_bit_widths(dev, kb, vb, v_alg2):
     want = oracle_attention(cache, q_np, B, Hq, Hkv, T, d)
     rel = np.array([normwise_rel(got[b, h], want[(b, h)]) for (b, h) in want])
     print("attend bits", (kb, vb, v_alg2), "max rel", rel.max())
+    assert rel.max() <= 1e-3
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T", [(2, 8, 2, 300), (1, 16, 2, 700)])
+@pytest.mark.parametrize("kb,vb,v_alg2", [(3, 2, True), (2, 3, True), (3, 2, False)])
+def test_attend_alg2_keys(dev, B, Hq, Hkv, T, kb, vb, v_alg2):
+    # Algorithm 2 keys: scores carry the QJL term alpha gamma <S q, 2z - 1> of the unbiased estimate
+    d = 128
+    cache = make_cache(B, Hkv, T, d, kb, vb, v_alg2, dev, k_alg2=True)
+    q_np = W.queries_bf16((B, Hq, d))
+    got = run_attend(cache, q_np, B, Hq, Hkv, T, d, dev)
+    want = oracle_attention(cache, q_np, B, Hq, Hkv, T, d)
+    rel = np.array([normwise_rel(got[b, h], want[(b, h)]) for (b, h) in want])
+    print("attend alg2 keys", (B, Hq, Hkv, T, kb, vb, v_alg2), "max rel", rel.max())
     assert rel.max() <= 1e-3

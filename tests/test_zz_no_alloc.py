@@ -80,7 +80,7 @@ def test_noalloc_rejects_oversize():
     cb = tq.Codebook()
     fake = ctypes.c_void_p(1 << 20)
     st = L.tq_attend_decode_noalloc(ctypes.byref(cb), ctypes.byref(cb), B, Hq, Hkv, T, d, fake, tq.TQ_BF16, fake,
-                                    fake, fake, fake, fake, fake, fake, 0.1, fake, None)
+                                    fake, fake, None, None, fake, fake, fake, fake, 0.1, fake, None)
     assert st == tq.TQ_ERR_WORKSPACE
     msg = L.tq_last_error().decode()
     assert str(need) in msg
