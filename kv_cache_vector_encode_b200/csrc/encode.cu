@@ -29,10 +29,11 @@
 // i.e. already in the tensor-core operand layout, with out-of-range rows / columns zero-filled.
 // bf16 tiles are converted to fp16 in place.
 //
-// Roles (14 warps): warp 0 issues the bulk / TMA copies; warp 1 owns TMEM and one lane issues every
-// MMA; warps 2-5 convert (one thread per vector: norm, power-of-two scale, fp16); warps 6-13 are
-// the epilogue (two warps per TMEM lane quarter, splitting the vectors of a tile). Buffers: input
-// stage x2, TMEM accumulators x2. All waits are bounded (sm100.cuh).
+// Roles (14 warps, 15 for Algorithm 2): warp 0 issues the bulk / TMA copies; warp 1 owns TMEM and
+// issues the products of x; warp 14 (Algorithm 2) issues the T rho products; warps 2-5 convert (one
+// thread per vector: norm, power-of-two scale, fp16); warps 6-13 are the epilogue (two warps per
+// TMEM lane quarter, splitting the vectors of a tile). Buffers: input stage x2, TMEM accumulators
+// x2. All waits are bounded (sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -45,7 +46,8 @@
 namespace tq {
 namespace {
 
-constexpr int kEncThreads = 448;
+// threads: 14 warps, plus (Algorithm 2) a 15th that issues the T rho products
+__host__ __device__ constexpr int enc_threads(bool alg2) { return alg2 ? 480 : 448; }
 constexpr float kRhoScale = 16384.0f;   // 2^14: |rho| < 2 keeps rho * 2^14 below the fp16 maximum
 
 struct EncodeParams {
@@ -120,7 +122,7 @@ __device__ __forceinline__ float transpose_reduce16(float (&r)[16], int lane) {
 }
 
 template <int XT, bool ALG2, int NV, int BITS>
-__global__ void __launch_bounds__(kEncThreads, 1)
+__global__ void __launch_bounds__(enc_threads(ALG2), 1)
     encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmap) {
   constexpr bool F32 = XT == TQ_F32;
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;       // TMEM columns per accumulator buffer
@@ -193,9 +195,11 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ---------------------------------------------------------------
-    // warp-uniform schedule (descriptors stay in uniform registers); one elected lane issues
+  } else if (warp == 1 || (ALG2 && warp == 14)) {
+    // ---------------- MMA issuers ---------------------------------------------------------------
+    // warp 1 issues the products of x, warp 14 (Algorithm 2) those of rho, so that the T rho
+    // products of a tile start as soon as its rho is written, not after the next tile's x products.
+    // Warp-uniform schedules (descriptors stay in uniform registers); one elected lane issues.
     if (mbar_wait_warp(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
       const uint32_t idesc = idesc_f16_f32(128, NV);
       const uint32_t a0 = smem_u32(smem + Lo.off_a[0]), a1 = smem_u32(smem + Lo.off_a[1]);
@@ -228,6 +232,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         return true;
       };
       bool ok = true;
+      if (ALG2 && warp == 14) {
+        for (int j = 0; j < my_tiles && ok; ++j) ok = issue_T(j);
+        ok = false;                                  // the x products are warp 1's
+      }
       for (int k = 0; k < my_tiles && ok; ++k) {
         const int a = k & 1, s = k & 1;
         if (!mbar_wait_warp(&bar[ACC_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
@@ -249,9 +257,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
           mma_commit(&bar[ACC_FULL + a]);
         }
         __syncwarp();
-        if (ALG2 && k >= 1) ok = issue_T(k - 1);
       }
-      if (ALG2 && ok && my_tiles >= 1 && !*abort_flag) issue_T(my_tiles - 1);
     }
   } else if (warp < 6) {
     // ---------------- converters: one thread per vector (TPV threads when NV < 128) -------------
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[STAGE_READY + s]);
     }
-  } else {
+  } else if (warp < 14) {
     // ---------------- epilogue: quantise, ballot-pack, residual, signs -------------------------
     const int e = warp - 6;                 // 0..7
     const int q = warp & 3;                 // TMEM lane quarter = packing group
@@ -522,7 +528,7 @@ tq_status launch_encode(EncodeParams& p, const void* x, cudaStream_t st) {
   if (e != cudaSuccess) return cuda_fail(e, "encode: shared memory attribute");
   p.ntiles = (int)((p.n + NV - 1) / NV);
   const int grid = std::min(p.ntiles, sm_count());
-  kern<<<grid, kEncThreads, Lo.total, st>>>(p, tmap);
+  kern<<<grid, enc_threads(ALG2), Lo.total, st>>>(p, tmap);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "encode: launch");
   return TQ_OK;
 }
