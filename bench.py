@@ -466,6 +466,44 @@ def run_ours(args):
     return 0
 
 
+def run_only_block(args):
+    """Times the block kernels alone (encode K, encode V, decode K, decode V) on the llama8b block shape
+    (a profiling entry point; prints one JSON line with the mean time of each call)."""
+    import torch
+    import kv_cache_vector_encode_b200 as tq
+    import workloads as W
+    dev = torch.device("cuda")
+    Pi, S = W.rotation(D), W.jl_matrix(D)
+    rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    cbk, cbv = tq.tq_codebook_init(D, K_BITS), tq.tq_codebook_init(D, V_BITS_BLOCK - 1)
+    nblk = BLK_HEADS * BLK_TOKENS
+    Kb = gen_kv(BLK_HEADS, BLK_TOKENS, D, 3, 20.0, 0.5, 7, dev)
+    Vb = gen_kv(BLK_HEADS, BLK_TOKENS, D, 3, 20.0, 0.5, 8, dev)
+    kc, kn = tq.empty_mse(nblk, D, K_BITS, dev)
+    vc, vs, vn, vg = tq.empty_prod(nblk, D, V_BITS_BLOCK, dev)
+    outk = torch.empty((nblk, D), dtype=torch.float32, device=dev)
+    outv = torch.empty((nblk, D), dtype=torch.float32, device=dev)
+    calls = {"encode_k": lambda: tq.tq_encode_mse(cbk, Kb, rot, kc, kn),
+             "encode_v": lambda: tq.tq_encode_prod(cbv, Vb, rot, vc, vs, vn, vg),
+             "decode_k": lambda: tq.tq_decode(cbk, rot, kc, kn, outk),
+             "decode_v": lambda: tq.tq_decode(cbv, rot, vc, vn, outv, signs=vs, gammas=vg)}
+    res = {}
+    for name, f in calls.items():
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            f()
+        b2.record()
+        torch.cuda.synchronize()
+        res[name + "_us"] = a.elapsed_time(b2) / args.steps * 1e3
+    tq.tq_sync_check()
+    print(json.dumps({"only": "block", "vectors": nblk, **res}), flush=True)
+    return 0
+
+
 def run_only_attend(args):
     """Times tq_attend_decode alone on the decode-attention shape with `--att-tokens` cached tokens
     (a profiling entry point; prints one JSON line with the mean time of a call)."""
@@ -519,7 +557,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["attend"], default=None,
+    ap.add_argument("--only", choices=["attend", "block"], default=None,
                     help="profiling entry point: time one path alone (not a bench line)")
     ap.add_argument("--att-tokens", type=int, default=ATT_T)
     args = ap.parse_args()
@@ -529,6 +567,8 @@ def main():
         return run_reference(args)
     if args.only == "attend":
         return run_only_attend(args)
+    if args.only == "block":
+        return run_only_block(args)
     return run_ours(args)
 
 
