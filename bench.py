@@ -255,6 +255,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     import kv_cache_vector_encode_b200 as tq
+    from kv_cache_vector_encode_b200 import shard
     import workloads as W
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -343,10 +344,7 @@ def run_ours(args):
     total_ms = e_start.elapsed_time(e_end)
     parts = {name: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
              for i, name in enumerate(["encode_k", "encode_v", "decode_k", "decode_v", "attend"])}
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = shard.max_over_ranks(total_ms, device=dev)      # device time, max over ranks
     ms_step = total_ms / args.steps
     value = world * vectors_per_step() / (ms_step * 1e-3)
 
@@ -409,10 +407,7 @@ def run_ours(args):
     e2e_run(e2e_steps, a, b2)
     barrier()
     e2e_ms = a.elapsed_time(b2) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = shard.max_over_ranks(e2e_ms, device=dev)
     e2e_value = world * vectors_per_step() / (e2e_ms * 1e-3)
 
     peak, peak_kind = peaks()
