@@ -4,8 +4,12 @@
 // estimates; ai-navigate-news page: keys by Algorithm 1, values by Algorithm 2):
 //   out[b][h] = sum_t softmax_t(scale <q, k_hat_t>) v_hat_t,   k_hat_t = n_t Pi^T c_K[idx_t],
 //   v_hat_t = m_t (Pi^T c_V[jdx_t] + alpha gamma_t S^T (2 z_t - 1)).
+// Keys may also be Algorithm 2: k_hat_t = n_t (Pi^T c_K[idx_t] + alpha g_t S^T (2 y_t - 1)), whose
+// extra score term alpha g_t <S q, 2 y_t - 1> is one more 0 / 2^s plane (the key sign bits) against
+// the fixed-point digits of q'' = S q, accumulated into score columns of its own.
 // Evaluated from the codes, never materialising k_hat or v_hat:
-//   * the query is rotated once, q' = Pi q (prep kernel);
+//   * the query is rotated once, q' = Pi q (and projected, q'' = S q, for Algorithm 2 keys) (prep
+//     kernel);
 //   * the codebook is an odd function of the index bits (exact symmetry), so c[idx] =
 //     sum_S beta_S prod_{p in S} (1 - 2 bit_p) over the odd subsets S of the bit planes
 //     (Walsh expansion). With b_S = XOR of the planes in S,
@@ -27,21 +31,21 @@
 // and the 2^s factor is divided out of the query limbs (scores) or of the output rows (values).
 //
 // Online softmax: a running maximum per head and running maxima of the value weights (which fix
-// the fixed-point scales). A chunk needs the four softmax warps to exchange maxima only when some
+// the fixed-point scales). A chunk needs a group's four softmax warps to exchange maxima only when some
 // token exceeds a running maximum; one barrier with an OR-reduction decides that, so after the
 // first chunks of a segment most chunks take no exchange at all.
 //
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
 // (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
-// Main-kernel roles (19 warps, 23 with separate value expanders): 0 bulk-copies packed chunks; 1
-// owns TMEM and issues the key MMAs;
-// 2-9 softmax (thread = token; two groups of four warps, each group owning half of the query
-// heads); 10-13 expand K into TMEM and (19 warps) V into shared memory (thread = token); 14-17
-// accumulate the value products (thread = coordinate); 18 issues the value MMAs; 19-22 (at most
-// four query heads per KV head) expand V, so that key and value expansion run side by side.
+// Main-kernel roles (19 warps; 23 with at most four query heads per KV head): 0 bulk-copies packed
+// chunks; 1 owns TMEM and issues the key MMAs; 2-9 softmax (thread = token; two groups of four
+// warps, each group owning half of the query heads); 10-13 expand the key planes into TMEM (thread
+// = token), and with 19 warps also the value planes into shared memory; 14-17 accumulate the value
+// products (thread = coordinate); 18 issues the value MMAs; 19-22 (23 warps) expand the value
+// planes, so that key and value expansion run side by side.
 // All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
-// same number of times by all four warps (their loop never exits early).
+// same number of times by the four warps of a group (their loop never exits early).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -252,16 +256,16 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
 
 enum ABars {
   ST_FULL = 0,                         // [kMaxStages]
-  ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (expander warps: 4)
+  ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (key and value expander warps: 4 or 8)
   BQ_FULL = ST_EMPTY + kMaxStages,     // [2]
   BQ_EMPTY = BQ_FULL + 2,              // [2]
-  AK_FULL = BQ_EMPTY + 2,              // [2]  expanders -> key MMA warp: key planes in TMEM (4 warps)
+  AK_FULL = BQ_EMPTY + 2,              // [2]  key expanders -> key MMA warp: key planes in TMEM (4 warps)
   SC_DONE = AK_FULL + 2,               // [2]  scores MMA complete (commit)
   BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA warps (8 warps)
-  AV_FULL = BW_FULL + 2,               // [3]  expanders -> value MMA warp: value planes (4 warps)
+  AV_FULL = BW_FULL + 2,               // [3]  value expanders -> value MMA warp: value planes (4 warps)
   V_DONE = AV_FULL + 3,                // [6]  value MMA of chunk c complete (commit), slot c % 6
   DV_EMPTY = V_DONE + 6,               // [2]  accumulators -> value MMA warp (4 warps)
-  SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (4 warps)
+  SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (8 warps)
   ANBARS = SCAL_FULL + 4
 };
 
