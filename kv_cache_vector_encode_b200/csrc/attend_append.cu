@@ -88,6 +88,16 @@ extern "C" TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_c
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(TQ_ERR_INVALID_ARG, f + ": bad B / Hq / Hkv");
   if (T_cur < 0 || T_max < T_cur + 1) return fail(TQ_ERR_INVALID_ARG, f + ": need 0 <= T_cur < T_max");
   if (cb_k->d != d || cb_v->d != d) return fail(TQ_ERR_INVALID_ARG, f + ": codebook d mismatch");
+  // the attention's limits, checked before anything is written to the cache
+  if (d != 128) return fail(TQ_ERR_UNSUPPORTED, f + ": this build supports d = 128");
+  if (Hq / Hkv > 8) return fail(TQ_ERR_UNSUPPORTED, f + ": at most 8 query heads per KV head");
+  if (T_cur + 1 > ((int64_t)1 << 31)) return fail(TQ_ERR_UNSUPPORTED, f + ": T too large");
+  if (cb_k->bits < 1 || cb_k->bits > 3 || cb_v->bits < 1 || cb_v->bits > 2)
+    return fail(TQ_ERR_UNSUPPORTED, f + ": key codebooks of 1..3 bits, value codebooks of 1..2 bits");
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, f + ": q dtype");
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(v_signs) || !aligned16(ws) || !aligned16(out) ||
+      !aligned16(rot))
+    return fail(TQ_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
   const AppendWs w = append_ws(B, Hq, Hkv, T_cur, d, cb_k->bits, cb_v->bits);
   if (ws_bytes < w.total) return fail(TQ_ERR_WORKSPACE, f + ": workspace too small");
   uint8_t* base = (uint8_t*)ws;

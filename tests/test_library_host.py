@@ -109,3 +109,11 @@ def test_attend_append_rejects_bad_arguments_on_host(L):
     assert L.tq_attend_append(*args(-1, 10, need)) == tq.TQ_ERR_INVALID_ARG
     assert L.tq_attend_append(*args(10, 20, need, vs=None)) == tq.TQ_ERR_INVALID_ARG   # values are Algorithm 2
     assert L.tq_attend_append(*args(10, 20, need - 1)) == tq.TQ_ERR_WORKSPACE
+    # the attention's own limits are checked before the encoders touch the cache
+    cb64 = tq.tq_codebook_init(64, 3)
+    bad_d = (ctypes.byref(cb64), ctypes.byref(tq.tq_codebook_init(64, 1)), 2, 8, 2, 10, 20, 64, g, tq.TQ_BF16, g, g,
+             tq.TQ_BF16, g, g, g, g, g, g, g, ctypes.c_float(0.1), g, g, need, None)
+    assert L.tq_attend_append(*bad_d) == tq.TQ_ERR_UNSUPPORTED
+    bad_q = list(args(10, 20, need))
+    bad_q[9] = tq.TQ_F16
+    assert L.tq_attend_append(*bad_q) == tq.TQ_ERR_UNSUPPORTED
