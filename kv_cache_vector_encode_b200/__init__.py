@@ -279,6 +279,10 @@ def tq_attend_append(cb_k: Codebook, cb_v: Codebook, q, rot, k_new, v_new, T_cur
     import torch
     B, Hq, d = q.shape
     Hkv, T_max = k_norms.shape[1], k_norms.shape[2]
+    if k_new.dtype != v_new.dtype:
+        raise TypeError("tq_attend_append: k_new and v_new must have the same dtype (one x_dtype for both)")
+    if tuple(k_new.shape) != (B, Hkv, d) or tuple(v_new.shape) != (B, Hkv, d):
+        raise ValueError(f"tq_attend_append: k_new / v_new must be [B, Hkv, d] = {(B, Hkv, d)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     wsb = tq_attend_append_workspace_bytes(B, Hq, Hkv, T_cur, d, cb_k.bits, cb_v.bits)
