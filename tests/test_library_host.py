@@ -117,3 +117,16 @@ def test_attend_append_rejects_bad_arguments_on_host(L):
     bad_q = list(args(10, 20, need))
     bad_q[9] = tq.TQ_F16
     assert L.tq_attend_append(*bad_q) == tq.TQ_ERR_UNSUPPORTED
+
+
+def test_binding_signatures_match_the_header(L):
+    # every function the binding declares has as many arguments as its prototype in tq.h
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"TQ_API\s+[\w\s\*]+?\b(tq_\w+)\s*\(([^;]*?)\)\s*;", src, flags=re.S):
+        params = m.group(2).strip()
+        protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    for name, (_res, args) in tq._SIGNATURES.items():
+        assert name in protos, name
+        assert len(args) == protos[name], (name, len(args), protos[name])
