@@ -12,7 +12,9 @@ Plain definitions, deliberately not the code-domain route of the CUDA path:
 * attention    = softmax_t(<q, k_hat_t> * scale) weighted sum of v_hat_t, per
   (batch, query head), query head h reading KV head h // (Hq / Hkv);
   no causal mask (one decode query sees the whole cache);
-* top-k        = the k largest scores, ties to the lower id, descending.
+* top-k        = the k largest scores, ties to the lower id, descending;
+* prefill      = causal multi-query attention: the last Q cached tokens are the queries' own
+  tokens, and query j attends the tokens up to and including its own position.
 """
 from __future__ import annotations
 
@@ -31,6 +33,19 @@ def softmax_attend(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, scale: flo
     p = np.exp(logits)
     p /= p.sum(axis=1, keepdims=True)
     return p @ np.asarray(vhat, dtype=np.float64)
+
+
+def prefill_attend(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, scale: float) -> np.ndarray:
+    """Causal multi-query attention of one KV head: q [Q, H, d] are the queries of the last Q of the
+    T cached tokens (khat, vhat [T, d]); query j sits at position T - Q + j and attends the tokens
+    t <= T - Q + j. Returns [Q, H, d] (fp64)."""
+    q = np.asarray(q, dtype=np.float64)
+    Qn, T = q.shape[0], np.asarray(khat).shape[0]
+    out = np.empty(q.shape, dtype=np.float64)
+    for j in range(Qn):
+        n = T - Qn + j + 1
+        out[j] = softmax_attend(q[j], khat[:n], vhat[:n], scale)
+    return out
 
 
 def decode_attention(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, scale: float) -> np.ndarray:

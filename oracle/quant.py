@@ -29,6 +29,12 @@ Readings where the pages are silent (each also listed in the design notes):
   QJL bit is z_j = [ (S r)_j >= 0 ] (sign(0) -> +1).
 * Zero vector: n = 0 gives u = 0, y = 0, idx_j = L/2 - 1; for Algorithm 2 the
   residual is taken as 0 (gamma = 0, all sign bits 1). Decode returns 0.
+* Non-finite input (the pages are silent; a policy of this library): a row with
+  a NaN entry stores n = NaN, a row with an infinite entry and no NaN stores
+  n = +Inf (the IEEE sum of squares), and either row is otherwise encoded as the
+  zero vector (idx_j = L/2 - 1; gamma = 0 and all sign bits 1). Decode then
+  returns non-finite values for it. A finite row whose norm exceeds the fp16
+  range stores n = +Inf (round to nearest) with its ordinary codes.
 * Packed layout (bit planes, one 32-bit word per 32 coordinates and plane):
   bit l of codes[v][g][p] is bit p of idx[v][32 g + l]; bit l of signs[v][g]
   is z[v][32 g + l]. Words are little-endian uint32.
@@ -96,12 +102,17 @@ def unpack_signs(words: np.ndarray) -> np.ndarray:
 # ---- encode -----------------------------------------------------------------------------------
 
 def normalise(x: np.ndarray):
-    """n = ||x|| (fp64), fp16 copy of n (RNE), u = x / n (0 for the zero vector)."""
+    """n = ||x|| (fp64), fp16 copy of n (RNE), u = x / n; u = 0 for the zero vector and for a row
+    with a non-finite entry (whose n is then NaN, or +Inf when no entry is NaN)."""
     x = np.asarray(x, dtype=np.float64)
-    n = np.sqrt(np.sum(x * x, axis=1))
-    safe = np.where(n > 0, n, 1.0)
-    u = np.where(n[:, None] > 0, x / safe[:, None], 0.0)
-    return n, n.astype(np.float16), u
+    with np.errstate(invalid="ignore", over="ignore"):
+        n = np.sqrt(np.sum(x * x, axis=1))
+    ok = np.isfinite(n) & (n > 0)
+    safe = np.where(ok, n, 1.0)
+    with np.errstate(invalid="ignore", over="ignore"):
+        u = np.where(ok[:, None], x / safe[:, None], 0.0)
+        n16 = n.astype(np.float16)                       # above the fp16 range: +Inf
+    return n, n16, u
 
 
 def rotate(u: np.ndarray, Pi: np.ndarray) -> np.ndarray:
@@ -131,7 +142,8 @@ def residual_signs(u: np.ndarray, idx: np.ndarray, n: np.ndarray, Pi: np.ndarray
     chat = c[idx]                                        # rotated-domain reconstruction
     Pi64 = np.asarray(Pi, dtype=np.float64)
     r = u - chat @ Pi64                                  # u - Pi^T c[idx], original domain
-    r[np.asarray(n) == 0] = 0.0
+    nn = np.asarray(n)
+    r[~(np.isfinite(nn) & (nn > 0))] = 0.0               # zero and non-finite rows: no residual
     gamma = np.sqrt(np.sum(r * r, axis=1))
     s = r @ np.asarray(S, dtype=np.float64).T            # S r
     z = s >= 0

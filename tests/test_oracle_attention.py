@@ -76,3 +76,38 @@ def test_topk_brute_force_with_ties():
     ids, _ = A.topk(s, 10)
     for r in range(5):
         assert list(ids[r]) == sorted(range(200), key=lambda j: (-s[r, j], j))[:10]
+
+
+def test_prefill_brute_force_mask():
+    """Causal multi-query attention against explicit loops with a mask matrix (tiny sizes)."""
+    g = np.random.default_rng(3)
+    T, Qn, H, d = 7, 4, 2, 5
+    q = g.standard_normal((Qn, H, d))
+    k = g.standard_normal((T, d))
+    v = g.standard_normal((T, d))
+    scale = 0.7
+    got = A.prefill_attend(q, k, v, scale)
+    for j in range(Qn):
+        pos = T - Qn + j
+        for h in range(H):
+            logit = [sum(q[j, h, i] * k[t, i] for i in range(d)) * scale if t <= pos else -math.inf
+                     for t in range(T)]
+            m = max(logit)
+            w = [math.exp(x - m) if x > -math.inf else 0.0 for x in logit]
+            z = sum(w)
+            want = [sum(w[t] * v[t, i] for t in range(T)) / z for i in range(d)]
+            assert np.allclose(got[j, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_special_cases():
+    """One query is decode attention over the whole cache; with T = Q the first query sees only its
+    own token (its output is that token's value); the last query always sees the whole cache."""
+    g = np.random.default_rng(4)
+    T, H, d = 9, 3, 6
+    k, v = g.standard_normal((T, d)), g.standard_normal((T, d))
+    q1 = g.standard_normal((1, H, d))
+    assert np.allclose(A.prefill_attend(q1, k, v, 0.3)[0], A.softmax_attend(q1[0], k, v, 0.3), rtol=1e-14)
+    qs = g.standard_normal((T, H, d))
+    out = A.prefill_attend(qs, k, v, 0.3)
+    assert np.allclose(out[0], np.broadcast_to(v[0], (H, d)), rtol=1e-14)
+    assert np.allclose(out[-1], A.softmax_attend(qs[-1], k, v, 0.3), rtol=1e-14)

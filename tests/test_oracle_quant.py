@@ -135,6 +135,35 @@ def test_zero_vector_convention():
     assert np.all(xh[0] == 0)
 
 
+def test_nonfinite_rows_policy():
+    """A row with a NaN entry stores n = NaN, one with an infinite entry (no NaN) n = +Inf; both are
+    otherwise the zero vector's record. Finite rows beside them are unaffected, and a finite row whose
+    norm overflows fp16 keeps its codes with n = +Inf."""
+    d, bits = 64, 3
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    cb = lloyd_max(d, bits - 1)
+    x = W.gaussian(6, d)
+    x[1, 5] = np.nan
+    x[2, 7] = np.inf
+    x[3, 0] = -np.inf
+    x[3, 9] = np.nan                              # NaN wins over Inf
+    x[4] *= np.float32(1e4)                       # |x| about 8e4 > 65504
+    e = Q.encode_prod(x, Pi, S, cb)
+    ref = Q.encode_prod(x[[0, 5]], Pi, S, cb)
+    L = 1 << (bits - 1)
+    assert np.isnan(e["norms"][1]) and np.isnan(e["norms"][3])
+    assert e["norms"][2] == np.inf and e["norms"][4] == np.inf
+    for r in (1, 2, 3):
+        assert np.all(e["idx"][r] == L // 2 - 1)
+        assert e["gammas"][r] == 0 and np.all(e["signs"][r] == 0xFFFFFFFF)
+    fin = Q.encode_prod(x[4:5] / np.float32(1e4), Pi, S, cb)
+    assert np.array_equal(e["codes"][4], fin["codes"][0])
+    for k in ("codes", "signs", "norms", "gammas"):
+        assert np.array_equal(e[k][[0, 5]], ref[k])
+    xh = Q.decode(e["codes"], e["norms"], Pi, cb, e["signs"], e["gammas"], S)
+    assert np.all(np.isnan(xh[1])) and np.all(~np.isfinite(xh[2])) and np.all(np.isfinite(xh[[0, 5]]))
+
+
 def test_scale_invariance_of_codes():
     d = 128
     Pi = W.rotation(d)
