@@ -35,6 +35,12 @@
  *   gammas fp16           gamma = ||r||, r = x/n - Pi^T c[idx]            (Algorithm 2)
  *   idx_j = #{k : t_k < y_j} for y = Pi x / n (ties to the lower index); the zero vector stores
  *   n = 0, idx_j = L/2 - 1, and for Algorithm 2 gamma = 0 with all sign bits 1.
+ *   Non-finite input (a policy of this library; the method is stated for finite vectors): a row
+ *   with a NaN entry stores n = NaN, a row with an infinite entry and no NaN stores n = +Inf, and
+ *   either row is otherwise stored as the zero vector (idx_j = L/2 - 1; gamma = 0, all sign bits
+ *   1); other rows of the call are unaffected. Decoding such a record gives non-finite values;
+ *   attention and scores over it are not specified. A finite row whose norm exceeds the fp16 range
+ *   (65504) stores n = +Inf with its ordinary codes.
  *   Bytes per vector: b d/8 + 2 (Algorithm 1); (b-1) d/8 + d/8 + 4 (Algorithm 2 at b bits).
  *   Arrays of vectors are the per-vector records above, back to back: codes [n][G][b],
  *   signs [n][G], norms [n], gammas [n].
@@ -148,6 +154,30 @@ TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t d, const vo
                     const uint32_t* signs, const uint16_t* norms, const uint16_t* gammas, void* out,
                     int32_t out_dtype, void* stream);
 
+/* Mixed widths per channel group (Algorithm 1). The d rotated coordinates form d/32 groups of 32
+ * (the packing groups of the layout); group g is quantised with its own width b_g = group_bits[g]
+ * (1..4) and the b_g-bit Lloyd-Max codebook of the same coordinate law (after the rotation every
+ * coordinate has that law), so fractional average rates such as 2.5 bits per coordinate, or more
+ * bits where a caller wants them, keep the per-coordinate optimality of each group. (The scope of
+ * this library's "mixed / fractional bit widths"; the techblog-plum page's compression table quotes
+ * an average of 2.5 bits, which is keys at 3 bits with values at 2, and the aigentlab page advises
+ * choosing the width per task.)
+ *   cbs         HOST array of 4 codebooks for d: cbs[b - 1] has b bits (entries for widths that
+ *               group_bits does not use are not read)
+ *   group_bits  HOST array of d/32 widths
+ *   codes       [n][W] words, W = sum_g b_g: group g's b_g bit-plane words (bit l of word p = bit p
+ *               of idx[32 g + l]) at word sum_{g' < g} b_g' of the record; norms [n] as tq_encode_mse
+ * d <= 128 (one fused kernel; 32, 64, 96 or 128). Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+TQ_API tq_status tq_encode_mse_mixed(const tq_codebook* cbs, const int32_t* group_bits, int64_t n, int32_t d,
+                                     const void* x, int32_t x_dtype, const void* rot, uint32_t* codes,
+                                     uint16_t* norms, void* stream);
+
+/* Dequantise the mixed-width format of tq_encode_mse_mixed: x_hat = n Pi^T c_g[idx] with each group's
+ * codebook, into out [n][d] of out_dtype (TQ_F32 or TQ_BF16). Arguments as tq_encode_mse_mixed. */
+TQ_API tq_status tq_decode_mixed(const tq_codebook* cbs, const int32_t* group_bits, int64_t n, int32_t d,
+                                 const void* rot, const uint32_t* codes, const uint16_t* norms, void* out,
+                                 int32_t out_dtype, void* stream);
+
 /* Workspace bytes tq_scores needs for these sizes. */
 TQ_API size_t tq_scores_workspace_bytes(int64_t nq, int64_t n, int32_t d, int32_t k);
 
@@ -189,6 +219,7 @@ TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int6
  *   values  Algorithm 2 with cb_v the (b_v-1)-bit codebook: v_codes [B][Hkv][T][d/32][b_v-1],
  *           v_signs [B][Hkv][T][d/32], v_norms, v_gammas [B][Hkv][T];
  *           or Algorithm 1 (v_signs and v_gammas NULL, cb_v the b_v-bit codebook)
+ *   scale   the softmax scale; 0 (or any value that is not > 0) selects 1/sqrt(d)
  *   out     [B][Hq][d] fp32
  * Supported: d = 128, Hq a multiple of Hkv with Hq/Hkv <= 8, T >= 1, key codebooks of 1..3 bits,
  * value codebooks of 1..2 bits (Algorithm 2 values at 2..3 bits, Algorithm 1 values at 1..2 bits).
@@ -199,6 +230,30 @@ TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_codebook* cb
                            const uint16_t* k_gammas, const uint32_t* v_codes,
                            const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas, float scale,
                            float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes tq_attend_prefill needs for these sizes (0 for invalid sizes). */
+TQ_API size_t tq_attend_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Qn, int64_t T, int32_t d);
+
+/* Multi-query (prefill) attention over a packed KV cache with a causal mask (techblog-plum page,
+ * notes: the rotation / QJL overhead shows once many queries share the cache; aiboss88 page:
+ * attention on the quantised cache). The last Qn of the T cached tokens of every slice are the new
+ * tokens themselves; query token j (0 <= j < Qn) sits at cache position T - Qn + j and attends the
+ * tokens t <= T - Qn + j:
+ *   out[b][j][h] = sum_{t <= T-Qn+j} softmax_t(scale <q[b][j][h], k_hat[b][g][t]>) v_hat[b][g][t],
+ *   g = h / (Hq/Hkv).
+ *   q    [B][Qn][Hq][d]  TQ_BF16 or TQ_F32;  out [B][Qn][Hq][d] fp32
+ *   cache, codebooks, rot, scale: as tq_attend_decode (keys Algorithm 1 or 2, values Algorithm 1
+ *   or 2), with the same limits; 1 <= Qn <= T. Qn = 1 is tq_attend_decode.
+ * The kernels evaluate up to 8 (query token, query head) pairs per KV head in one pass over the
+ * cache (8 / (Hq/Hkv) query tokens per pass); longer prefills take several passes, each over the
+ * tokens its queries can see. ws: caller device workspace of at least
+ * tq_attend_prefill_workspace_bytes(B, Hq, Hkv, Qn, T, d) bytes. */
+TQ_API tq_status tq_attend_prefill(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                   int32_t Hkv, int32_t Qn, int64_t T, int32_t d, const void* q, int32_t q_dtype,
+                                   const void* rot, const uint32_t* k_codes, const uint16_t* k_norms,
+                                   const uint32_t* k_signs, const uint16_t* k_gammas, const uint32_t* v_codes,
+                                   const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas,
+                                   float scale, float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Workspace bytes of tq_attend_append for these sizes (k_bits: the key codebook's bits;
  * v_codebook_bits: the value codebook's bits, b_v - 1); 0 for invalid sizes. */
@@ -250,6 +305,15 @@ TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, const tq_code
                                    const uint32_t* k_signs, const uint16_t* k_gammas, const uint32_t* v_codes,
                                    const uint32_t* v_signs, const uint16_t* v_norms, const uint16_t* v_gammas,
                                    float scale, float* out, void* stream);
+
+/* Self-test of the failure-detection path; no counterpart in the TurboQuant write-ups. Every
+ * hand-off between the warps of a libtq kernel is a wait bounded in time: one that runs out records
+ * an error and lets the kernel return, so a lost arrival is reported instead of hanging the GPU.
+ * This call enqueues one small kernel that makes such a wait run out on purpose (an mbarrier that
+ * nothing arrives on, limit `limit_ns` nanoseconds, 1000 <= limit_ns <= 1e9); the next
+ * tq_sync_check then returns TQ_ERR_DEVICE_TIMEOUT once and clears it, and later calls work as
+ * before. Nothing faults and nothing hangs. Errors: INVALID_ARG (limit), CUDA. */
+TQ_API tq_status tq_selftest_wait(uint64_t limit_ns, void* stream);
 
 /* Synchronises `stream`, then reports a pending CUDA error (TQ_ERR_CUDA) or a device-side
  * timeout recorded by any libtq kernel since the last check (TQ_ERR_DEVICE_TIMEOUT, which this

@@ -67,6 +67,8 @@ _SIGNATURES = {
     "tq_encode_prod": (_I32, [_CB, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tq_encode_workspace_bytes": (_SZ, [_I64, _I32, _I32]),
     "tq_decode": (_I32, [_CB, _I64, _I32, _P, _P, _P, _P, _P, _P, _I32, _P]),
+    "tq_encode_mse_mixed": (_I32, [_CB, _P, _I64, _I32, _P, _I32, _P, _P, _P, _P]),
+    "tq_decode_mixed": (_I32, [_CB, _P, _I64, _I32, _P, _P, _P, _P, _I32, _P]),
     "tq_scores_workspace_bytes": (_SZ, [_I64, _I64, _I32, _I32]),
     "tq_scores": (_I32, [_CB, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tq_attend_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
@@ -74,9 +76,13 @@ _SIGNATURES = {
                                 _P, _F, _P, _P, _SZ, _P]),
     "tq_attend_decode_noalloc": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P,
                                         _P, _P, _P, _F, _P, _P]),
+    "tq_attend_prefill_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I64, _I32]),
+    "tq_attend_prefill": (_I32, [_CB, _CB, _I32, _I32, _I32, _I32, _I64, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P,
+                                 _P, _P, _F, _P, _P, _SZ, _P]),
     "tq_attend_append_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32, _I32, _I32]),
     "tq_attend_append": (_I32, [_CB, _CB, _I32, _I32, _I32, _I64, _I64, _I32, _P, _I32, _P, _P, _I32, _P, _P, _P,
                                 _P, _P, _P, _P, _F, _P, _P, _SZ, _P]),
+    "tq_selftest_wait": (_I32, [ctypes.c_uint64, _P]),
     "tq_sync_check": (_I32, [_P]),
 }
 
@@ -192,6 +198,38 @@ def tq_decode(cb: Codebook, rot, codes, norms, out, signs=None, gammas=None, str
                            _ptr(out, "out", [torch.float32, torch.bfloat16]), _xdtype(out), _stream(stream)))
 
 
+def _mixed_args(d: int, group_bits):
+    """Host arrays of the mixed-width calls: the 4 codebooks of d (1..4 bits) and the group widths."""
+    G = d // 32
+    if len(group_bits) != G:
+        raise ValueError(f"group_bits needs {G} entries for d = {d}")
+    cbs = (Codebook * 4)()
+    for b in sorted(set(int(x) for x in group_bits)):
+        if 1 <= b <= 4:
+            cbs[b - 1] = tq_codebook_init(d, b)
+    gb = (ctypes.c_int32 * G)(*[int(x) for x in group_bits])
+    return cbs, gb
+
+
+def tq_encode_mse_mixed(group_bits, x, rot, codes, norms, stream=None):
+    """Algorithm 1 with a width per group of 32 rotated coordinates; codes [n, sum(group_bits)] int32."""
+    import torch
+    n, d = x.shape
+    cbs, gb = _mixed_args(d, group_bits)
+    _check(lib().tq_encode_mse_mixed(cbs, gb, n, d, _ptr(x, "x", [torch.float32, torch.bfloat16]), _xdtype(x),
+                                     _ptr(rot, "rot"), _ptr(codes, "codes", [torch.int32]),
+                                     _ptr(norms, "norms", [torch.float16]), _stream(stream)))
+
+
+def tq_decode_mixed(group_bits, rot, codes, norms, out, stream=None):
+    import torch
+    n, d = out.shape
+    cbs, gb = _mixed_args(d, group_bits)
+    _check(lib().tq_decode_mixed(cbs, gb, n, d, _ptr(rot, "rot"), _ptr(codes, "codes", [torch.int32]),
+                                 _ptr(norms, "norms", [torch.float16]),
+                                 _ptr(out, "out", [torch.float32, torch.bfloat16]), _xdtype(out), _stream(stream)))
+
+
 def tq_scores_workspace_bytes(nq: int, n: int, d: int, k: int) -> int:
     return int(lib().tq_scores_workspace_bytes(nq, n, d, k))
 
@@ -220,12 +258,11 @@ def tq_attend_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int) -> int:
 
 def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
                      v_signs=None, v_gammas=None, scale=None, ws=None, stream=None, k_signs=None, k_gammas=None):
-    import math
     import torch
     B, Hq, d = q.shape
     Hkv, T = k_norms.shape[1], k_norms.shape[2]
     if scale is None:
-        scale = 1.0 / math.sqrt(d)
+        scale = 0.0                   # the library's default, 1/sqrt(d)
     wsb = tq_attend_workspace_bytes(B, Hq, Hkv, T, d)
     if ws is None:
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
@@ -244,12 +281,11 @@ def tq_attend_decode(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v
 def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
                              v_signs=None, v_gammas=None, scale=None, stream=None, k_signs=None, k_gammas=None):
     """tq_attend_decode with the library's fixed scratch array (no workspace, no allocation)."""
-    import math
     import torch
     B, Hq, d = q.shape
     Hkv, T = k_norms.shape[1], k_norms.shape[2]
     if scale is None:
-        scale = 1.0 / math.sqrt(d)
+        scale = 0.0                   # the library's default, 1/sqrt(d)
     _check(lib().tq_attend_decode_noalloc(ctypes.byref(cb_k), ctypes.byref(cb_v), B, Hq, Hkv, T, d,
                                           _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q), _ptr(rot, "rot"),
                                           _ptr(k_codes, "k_codes", [torch.int32]),
@@ -261,6 +297,34 @@ def tq_attend_decode_noalloc(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_
                                           _ptr(v_norms, "v_norms", [torch.float16]),
                                           _ptr(v_gammas, "v_gammas", [torch.float16], True), float(scale),
                                           _ptr(out, "out", [torch.float32]), _stream(stream)))
+
+
+def tq_attend_prefill_workspace_bytes(B: int, Hq: int, Hkv: int, Qn: int, T: int, d: int) -> int:
+    return int(lib().tq_attend_prefill_workspace_bytes(B, Hq, Hkv, Qn, T, d))
+
+
+def tq_attend_prefill(cb_k: Codebook, cb_v: Codebook, q, rot, k_codes, k_norms, v_codes, v_norms, out,
+                      v_signs=None, v_gammas=None, scale=None, ws=None, stream=None, k_signs=None, k_gammas=None):
+    """Causal multi-query attention: q, out [B, Qn, Hq, d]; the cache [B][Hkv][T] holds the Qn new
+    tokens in its last Qn slots (query j attends slots t <= T - Qn + j)."""
+    import torch
+    B, Qn, Hq, d = q.shape
+    Hkv, T = k_norms.shape[1], k_norms.shape[2]
+    if scale is None:
+        scale = 0.0                   # the library's default, 1/sqrt(d)
+    wsb = tq_attend_prefill_workspace_bytes(B, Hq, Hkv, Qn, T, d)
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().tq_attend_prefill(ctypes.byref(cb_k), ctypes.byref(cb_v), B, Hq, Hkv, Qn, T, d,
+                                   _ptr(q, "q", [torch.float32, torch.bfloat16]), _xdtype(q), _ptr(rot, "rot"),
+                                   _ptr(k_codes, "k_codes", [torch.int32]), _ptr(k_norms, "k_norms", [torch.float16]),
+                                   _ptr(k_signs, "k_signs", [torch.int32], True),
+                                   _ptr(k_gammas, "k_gammas", [torch.float16], True),
+                                   _ptr(v_codes, "v_codes", [torch.int32]),
+                                   _ptr(v_signs, "v_signs", [torch.int32], True),
+                                   _ptr(v_norms, "v_norms", [torch.float16]),
+                                   _ptr(v_gammas, "v_gammas", [torch.float16], True), float(scale),
+                                   _ptr(out, "out", [torch.float32]), _ptr(ws, "ws"), ws.numel(), _stream(stream)))
 
 
 TQ_ATTEND_NOALLOC_MAX_BYTES = 8 << 20
@@ -275,7 +339,6 @@ def tq_attend_append(cb_k: Codebook, cb_v: Codebook, q, rot, k_new, v_new, T_cur
                      v_signs, v_norms, v_gammas, out, scale=None, ws=None, stream=None):
     """Encode the new token's K / V of every slice into slot T_cur of the cache, then attend over slots
     [0, T_cur]. The cache tensors are [B][Hkv][T_max]... as for tq_attend_decode; k_new, v_new [B][Hkv][d]."""
-    import math
     import torch
     B, Hq, d = q.shape
     Hkv, T_max = k_norms.shape[1], k_norms.shape[2]
@@ -284,7 +347,7 @@ def tq_attend_append(cb_k: Codebook, cb_v: Codebook, q, rot, k_new, v_new, T_cur
     if tuple(k_new.shape) != (B, Hkv, d) or tuple(v_new.shape) != (B, Hkv, d):
         raise ValueError(f"tq_attend_append: k_new / v_new must be [B, Hkv, d] = {(B, Hkv, d)}")
     if scale is None:
-        scale = 1.0 / math.sqrt(d)
+        scale = 0.0                   # the library's default, 1/sqrt(d)
     wsb = tq_attend_append_workspace_bytes(B, Hq, Hkv, T_cur, d, cb_k.bits, cb_v.bits)
     if ws is None:
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
@@ -301,6 +364,12 @@ def tq_attend_append(cb_k: Codebook, cb_v: Codebook, q, rot, k_new, v_new, T_cur
 
 def tq_sync_check(stream=None):
     _check(lib().tq_sync_check(_stream(stream)))
+
+
+def tq_selftest_wait(limit_ns: int = 1_000_000, stream=None):
+    """Enqueue the failure-detection self-test: a bounded device wait that runs out on purpose; the
+    next tq_sync_check raises TQError with status TQ_ERR_DEVICE_TIMEOUT once."""
+    _check(lib().tq_selftest_wait(int(limit_ns), _stream(stream)))
 
 
 # ---- allocation helpers (torch device memory) --------------------------------------------------

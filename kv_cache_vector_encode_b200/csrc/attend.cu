@@ -71,11 +71,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Parameters shared by the three kernels
 // ------------------------------------------------------------------------------------------------
 struct AttParams {
-  int B, Hq, Hkv, Hg, d, G;
+  int B, Hq, Hkv, d, G;
+  // Virtual heads: a pass attends Hg = nqry x Hgr (query token, query head) pairs per slice; query
+  // token j of the pass and head h are virtual head j * Hgr + h. Decode has nqry = 1 (Hg = Hgr).
+  int Hg, Hgr, nqry;
+  int64_t q_bs, q_js;            // element strides of q and out: batch, query token (head stride d)
+  int64_t tlim0;                 // query token j of the pass attends the tokens t < tlim0 + j
   int64_t T;                     // tokens attended per slice
   int64_t tstride;               // token slots per slice in the cache arrays (>= T)
   int slices, nchunk, per_cta, maxseg;
   int nst;                       // depth of the packed-chunk ring
+  int norm_bulk;                 // 1: the norm arrays are bulk-copied into the stage with the codes
+                                 // (slot stride a multiple of 8 tokens, 16-byte aligned arrays)
   int bk, mk, ksign;             // key codebook bits, key Walsh planes, key sign plane (Algorithm 2 keys)?
   int bv, mv, vsign, np;         // value codebook bits, value Walsh planes, sign plane?, planes
   int nq;                        // MMA N of the scores / of one value weight kind (16 or 32)
@@ -93,6 +100,19 @@ struct AttParams {
   const uint32_t* v_signs;
   const uint16_t* v_norms;
   const uint16_t* v_gammas;
+  // append (tq_attend_append): the prep kernel encodes each slice's new key (Algorithm 1) and value
+  // (Algorithm 2) into slot t_new of the cache before the main kernel reads it; NULL otherwise
+  const void* k_new;
+  const void* v_new;             // [slices][d], x_bf16 ? bf16 : fp32
+  int x_bf16;
+  int64_t t_new;
+  uint32_t* kw_codes;
+  uint16_t* kw_norms;
+  uint32_t* vw_codes;
+  uint32_t* vw_signs;
+  uint16_t* vw_norms;
+  uint16_t* vw_gammas;
+  float ck[8], tk[8], cv[8], tv[8];   // fp32 centroids / boundaries of the key and value codebooks
   uint8_t* bq_img;               // [slices][nq rows x (mk + ksign) d bytes] K-major SW128 image
   float* head_c;                 // [slices][8][4]: 2^-F, Q_h * sum beta, 2^-F'', Q''_h
   float* partial;                // [slices][maxseg][Hg][att_rec(d)]
@@ -105,6 +125,64 @@ struct AttParams {
 __host__ __device__ inline int att_rec(int d) { return 4 + 3 * d; }
 
 // ------------------------------------------------------------------------------------------------
+// append: encode one new vector of a slice into its cache slot, in fp64 on the SIMT cores (thread =
+// coordinate, 128 threads). The steps are Algorithm 1 / 2 as the encoders compute them (ai-navigate-
+// news page, "how it works (technical)"): n = |x| (fp16 record), u = x / n (zero and non-finite rows:
+// u = 0), y = Pi u, idx_j = #{k : t_k < y_j}, bit planes by ballot; Algorithm 2 adds
+// r = u - Pi^T c[idx], gamma = |r| and the sign bits of S r.
+// ------------------------------------------------------------------------------------------------
+__device__ double prep_block_sum(double v, double* red4) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red4[warp] = v;
+  __syncthreads();
+  return (red4[0] + red4[1]) + (red4[2] + red4[3]);
+}
+
+__device__ void append_encode(const AttParams& p, int slice, const void* xsrc, bool alg2, int bits, const float* c,
+                              const float* t, uint32_t* codes, uint16_t* norms, uint32_t* signs, uint16_t* gammas,
+                              double* sh, double* red4) {
+  const int d = p.d, i = threadIdx.x, g = i >> 5, lane = i & 31;
+  const int L = 1 << bits;
+  const size_t xo = (size_t)slice * d + i;
+  const double xi = p.x_bf16 ? (double)__uint_as_float((uint32_t)((const uint16_t*)xsrc)[xo] << 16)
+                             : (double)((const float*)xsrc)[xo];
+  const double n = sqrt(prep_block_sum(xi * xi, red4));
+  const bool ok = isfinite(n) && n > 0.0;
+  double* u = sh;                                     // [128]
+  double* cs = sh + 128;                              // [128]
+  u[i] = ok ? xi / n : 0.0;
+  __syncthreads();
+  double y = 0.0;                                     // y_i = sum_j Pi[i][j] u_j
+  for (int j = 0; j < d; ++j) y = fma((double)__ldg(p.Pi + (size_t)i * d + j), u[j], y);
+  int idx = 0;
+  for (int k = 0; k < L - 1; ++k) idx += (double)t[k] < y ? 1 : 0;
+  const int64_t rec = (int64_t)slice * p.tstride + p.t_new;
+  for (int pl = 0; pl < bits; ++pl) {
+    const uint32_t w = __ballot_sync(0xffffffffu, (idx >> pl) & 1);
+    if (lane == 0) codes[(rec * p.G + g) * bits + pl] = w;
+  }
+  if (i == 0) norms[rec] = __half_as_ushort(__double2half(n));
+  if (!alg2) return;
+  cs[i] = (double)c[idx];
+  __syncthreads();
+  double a = 0.0;                                     // (Pi^T c)_i = sum_j Pi[j][i] c_j
+  for (int j = 0; j < d; ++j) a = fma((double)__ldg(p.Pi + (size_t)j * d + i), cs[j], a);
+  const double r = ok ? u[i] - a : 0.0;
+  const double gam = sqrt(prep_block_sum(r * r, red4));
+  cs[i] = r;                                          // (the sums above synchronised the block)
+  __syncthreads();
+  double sv = 0.0;                                    // (S r)_i
+  for (int j = 0; j < d; ++j) sv = fma((double)__ldg(p.S + (size_t)i * d + j), cs[j], sv);
+  const uint32_t w = __ballot_sync(0xffffffffu, sv >= 0.0);
+  if (lane == 0) signs[rec * p.G + g] = w;
+  if (i == 0) gammas[rec] = __half_as_ushort(__double2half(gam));
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------------------------------------
 // prep: q' = Pi q per query head, fixed-point limbs of beta_S q' (scaled by 2^-s), constants
 // ------------------------------------------------------------------------------------------------
 __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
@@ -114,11 +192,19 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   const int warp = i >> 5, lane = i & 31;
   __shared__ __align__(16) float sq[8][128];
   __shared__ double red[4][8][4];
+  if (p.kw_codes) {
+    // append: this slice's new key and value go into slot t_new before anything reads the cache
+    __shared__ double esh[256];
+    __shared__ double ered[4];
+    append_encode(p, slice, p.k_new, false, p.bk, p.ck, p.tk, p.kw_codes, p.kw_norms, nullptr, nullptr, esh, ered);
+    append_encode(p, slice, p.v_new, true, p.bv, p.cv, p.tv, p.vw_codes, p.vw_norms, p.vw_signs, p.vw_gammas, esh,
+                  ered);
+  }
   const int kbytes = (p.mk + p.ksign) * d;
   uint8_t* img = p.bq_img + (size_t)slice * p.nq * kbytes;
   for (int o = i; o < p.nq * kbytes / 16; o += blockDim.x) ((uint4*)img)[o] = make_uint4(0, 0, 0, 0);
   for (int h = 0; h < p.Hg; ++h) {
-    const size_t qoff = ((size_t)b * p.Hq + hk * p.Hg + h) * d;
+    const size_t qoff = (size_t)b * p.q_bs + (size_t)(h / p.Hgr) * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * d;
     sq[h][i] = p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
                         : ((const float*)p.q)[qoff + i];
   }
@@ -222,10 +308,20 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
 // ------------------------------------------------------------------------------------------------
 // main kernel
 // ------------------------------------------------------------------------------------------------
+// A run is a stretch of consecutive chunks of one slice over which no running maximum and no
+// fixed-point scale of the softmax changes: the value MMAs accumulate its chunks in one TMEM buffer
+// (exact int32 limb sums) and the accumulator warps fold it once. Runs stop at 256 chunks, which
+// keeps every limb sum below 2^30. Run record (kRunRec bytes): [0, 32) running maxima of the 8
+// heads, [32] 1/sw, [36] 1/sw', [40] flags (1 = last run of its segment, 2 = last run of the CTA),
+// [44] segment ordinal, [48] slice, [64, 256) exact run sums (uint64) of the weight kinds
+// w, w gamma, p (2^22 fixed point) for the 8 heads.
+constexpr int kRunRec = 256;
+constexpr int kMaxRun = 256;
+
 struct AttLayout {
-  uint32_t kc_bytes, vc_bytes, sg_off, ks_off, stage_bytes;
+  uint32_t kc_bytes, vc_bytes, sg_off, ks_off, nrm_off, stage_bytes;
   uint32_t off_stage, av_bytes, off_av, bw_kind, bw_buf, off_bw, bq_bytes, off_bq, off_sc, off_red, off_sum,
-      off_bar, total;
+      off_run, off_bar, total;
 };
 
 __host__ __device__ inline uint32_t aru(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -236,7 +332,9 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.sg_off = L.kc_bytes + kChunk * p.G * p.bv * 4;     // sign words of the chunk
   L.vc_bytes = kChunk * p.G * (p.bv + (p.vsign ? 1 : 0)) * 4;
   L.ks_off = L.kc_bytes + L.vc_bytes;                 // key sign words (Algorithm 2 keys)
-  L.stage_bytes = aru(L.ks_off + (p.ksign ? kChunk * p.G * 4 : 0), 1024);
+  // fp16 key norms, value norms, value gammas, key gammas of the chunk: [4][128]
+  L.nrm_off = aru(L.ks_off + (p.ksign ? kChunk * p.G * 4 : 0), 16);
+  L.stage_bytes = aru(L.nrm_off + (p.norm_bulk ? 4 * kChunk * 2 : 0), 1024);
   uint32_t off = 0;
   L.off_stage = off; off += nst * L.stage_bytes;
   L.av_bytes = kChunk * 128;                       // one plane: 128 tokens x 128 coordinates
@@ -249,14 +347,17 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.off_sc = off; off += 4 * 64 * 4;               // chunk scalars, 4-deep ring of 64 floats
   L.off_red = off; off += 2 * 4 * 16 * 4;          // max exchange of the softmax warps: [group][warp][16]
   L.off_sum = off; off += 4 * 4 * 24 * 4;          // chunk sums of the weights: [ring][warp][kind][head]
+  L.off_run = aru(off, 16); off = L.off_run + 2 * kRunRec;   // records of the two runs in flight
   L.off_bar = aru(off, 8); off = L.off_bar + 64 * 8;
   L.total = off + 1024;
   return L;
 }
 
+
 enum ABars {
   ST_FULL = 0,                         // [kMaxStages]
-  ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (key and value expander warps: 4 or 8)
+  ST_EMPTY = ST_FULL + kMaxStages,     // [kMaxStages] (key and value expander warps, 4 or 8, and the
+                                       //  8 softmax warps, which read the stage's norms)
   BQ_FULL = ST_EMPTY + kMaxStages,     // [2]
   BQ_EMPTY = BQ_FULL + 2,              // [2]
   AK_FULL = BQ_EMPTY + 2,              // [2]  key expanders -> key MMA warp: key planes in TMEM (4 warps)
@@ -264,9 +365,10 @@ enum ABars {
   BW_FULL = SC_DONE + 2,               // [2]  softmax -> MMA warps (8 warps)
   AV_FULL = BW_FULL + 2,               // [3]  value expanders -> value MMA warp: value planes (4 warps)
   V_DONE = AV_FULL + 3,                // [6]  value MMA of chunk c complete (commit), slot c % 6
-  DV_EMPTY = V_DONE + 6,               // [2]  accumulators -> value MMA warp (4 warps)
-  SCAL_FULL = DV_EMPTY + 2,            // [4]  softmax -> accumulators: chunk scalars (8 warps)
-  ANBARS = SCAL_FULL + 4
+  RUN_DONE = V_DONE + 6,               // [2]  value MMA warp -> accumulators: a run's MMAs complete (commit)
+                                       //      and its record written (arrive): 2 arrivals
+  RUN_FREE = RUN_DONE + 2,             // [2]  accumulators -> value MMA warp: run buffer drained (4 warps)
+  ANBARS = RUN_FREE + 2
 };
 
 // TMEM columns: A_K [2][32 (mk + ksign)] at 0, scores [2][nq (1 + ksign)] after them, value
@@ -288,6 +390,19 @@ struct ChunkIter {
       cis = 0;
       ++slice;
       ++seg;
+    }
+  }
+};
+
+// Position in a ring of n slots walked one step per chunk: slot and the parity of the pass over the
+// ring (the mbarrier phase), kept incrementally instead of by division.
+struct RingPos {
+  int slot, n;
+  uint32_t par;
+  __device__ __forceinline__ void next() {
+    if (++slot == n) {
+      slot = 0;
+      par ^= 1u;
     }
   }
 };
@@ -401,7 +516,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&bar[ST_FULL + s], 1);
-      mbar_init(&bar[ST_EMPTY + s], SPLITV ? 8 : 4);   // key (and value) expanders
+      mbar_init(&bar[ST_EMPTY + s], (SPLITV ? 8 : 4) + 8);   // key (and value) expanders, softmax
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
@@ -409,11 +524,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       mbar_init(&bar[AK_FULL + s], 4);
       mbar_init(&bar[SC_DONE + s], 1);
       mbar_init(&bar[BW_FULL + s], 8);
-      mbar_init(&bar[DV_EMPTY + s], 4);
+      mbar_init(&bar[RUN_DONE + s], 2);
+      mbar_init(&bar[RUN_FREE + s], 4);
     }
     for (int s = 0; s < 3; ++s) mbar_init(&bar[AV_FULL + s], 4);
     for (int s = 0; s < 6; ++s) mbar_init(&bar[V_DONE + s], 1);
-    for (int s = 0; s < 4; ++s) mbar_init(&bar[SCAL_FULL + s], 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -433,7 +548,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     // ------------------------------------ producer -------------------------------------------------
     // warp-uniform schedule; one elected lane issues the copies
     const uint32_t nb = (uint32_t)(NQ * MKT * d);
-    for (int c = 0; c < nmy; ++c, it.next()) {
+    RingPos rs{0, nst, 0u};
+    for (int c = 0; c < nmy; ++c, it.next(), rs.next()) {
       if (c == 0 || it.cis == 0) {
         const int sg = it.seg;
         if (!mbar_wait_warp(&bar[BQ_EMPTY + (sg & 1)], ((sg >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
@@ -444,17 +560,28 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         }
         __syncwarp();
       }
-      const int st = c % nst;
-      if (!mbar_wait_warp(&bar[ST_EMPTY + st], ((c / nst) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
+      const int st = rs.slot;
+      if (!mbar_wait_warp(&bar[ST_EMPTY + st], rs.par ^ 1u, p.err, kDevTimeoutSync, abort_flag)) break;
       const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
       const int64_t vec0 = (int64_t)it.slice * TS + (int64_t)it.cis * kChunk;  // record of the first token
       const uint32_t kb = (uint32_t)tc * G * BK * 4;
       const uint32_t vb = (uint32_t)tc * G * BV * 4;
       const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
       const uint32_t kgb = KS ? (uint32_t)tc * G * 4 : 0u;
+      // norms of the first tc & ~7 tokens (whole 16-byte pieces; a ragged remainder is read by the
+      // softmax warps themselves)
+      const uint32_t nb2 = p.norm_bulk ? (uint32_t)(tc & ~7) * 2u : 0u;
+      const uint32_t nrmb = nb2 * (2u + (VS ? 1u : 0u) + (KS ? 1u : 0u));
       uint8_t* stg = smem + Lo.off_stage + st * Lo.stage_bytes;
       if (elect_one_sync()) {
-        mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb + kgb);
+        mbar_arrive_expect_tx(&bar[ST_FULL + st], kb + vb + sb + kgb + nrmb);
+        if (nb2) {
+          uint8_t* sn = stg + Lo.nrm_off;
+          bulk_g2s(sn, p.k_norms + vec0, nb2, &bar[ST_FULL + st]);
+          bulk_g2s(sn + 2 * kChunk, p.v_norms + vec0, nb2, &bar[ST_FULL + st]);
+          if (VS) bulk_g2s(sn + 4 * kChunk, p.v_gammas + vec0, nb2, &bar[ST_FULL + st]);
+          if (KS) bulk_g2s(sn + 6 * kChunk, p.k_gammas + vec0, nb2, &bar[ST_FULL + st]);
+        }
         bulk_g2s(stg, p.k_codes + vec0 * G * BK, kb, &bar[ST_FULL + st]);
         bulk_g2s(stg + Lo.kc_bytes, p.v_codes + vec0 * G * BV, vb, &bar[ST_FULL + st]);
         if (VS) bulk_g2s(stg + Lo.sg_off, p.v_signs + vec0 * G, sb, &bar[ST_FULL + st]);
@@ -511,33 +638,36 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     const int Hg = p.Hg;
     float* rgrp = red + gq * 64;
     float mrun[HH], ha[HH], hb[HH], hs[HH], hq[HH];
+    int hlim[HH];                                   // each head sees the slice's tokens t < hlim (causal)
     float vmax_run = 0.0f, gmax_run = 0.0f, sw = 1.0f, sw2 = 1.0f, isw = 1.0f, isw2 = 1.0f;
     bool ok = true;
-    // fp16 norms of the next chunk, loaded one chunk ahead and converted only when used (dead
-    // tokens read as zero)
-    uint16_t nk_n = 0, nv_n = 0, gm_n = 0, gk_n = 0;
-    ChunkIter nx = it;                              // position of the chunk whose norms are prefetched
-    auto load_norms = [&]() {
-      nk_n = nv_n = gm_n = gk_n = 0;
-      if (t < (nx.cis == p.nchunk - 1 ? tail : kChunk)) {
-        const int64_t rec = (int64_t)nx.slice * TS + (int64_t)nx.cis * kChunk + t;
+    // fp16 norms of the chunk's tokens: from the stage (bulk-copied with the codes) where possible,
+    // else from global memory (dead tokens read as zero)
+    RingPos rs{0, nst, 0u};
+    for (int c = 0; c < nmy; ++c, it.next(), rs.next()) {     // no early exit: the named barriers must match
+      const int b = c & 1;
+      const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
+      const bool live = t < tc;
+      uint16_t nk_n = 0, nv_n = 0, gm_n = 0, gk_n = 0;
+      ok = mbar_wait_warp(&bar[ST_FULL + rs.slot], rs.par, p.err, kDevTimeoutLoad, abort_flag) && ok;
+      if (p.norm_bulk && t < (tc & ~7)) {
+        const uint16_t* sn = (const uint16_t*)(smem + Lo.off_stage + rs.slot * Lo.stage_bytes + Lo.nrm_off);
+        nk_n = sn[t];
+        nv_n = sn[kChunk + t];
+        if (VS) gm_n = sn[2 * kChunk + t];
+        if (KS) gk_n = sn[3 * kChunk + t];
+      } else if (live) {
+        const int64_t rec = (int64_t)it.slice * TS + (int64_t)it.cis * kChunk + t;
         nk_n = __ldg(p.k_norms + rec);
         nv_n = __ldg(p.v_norms + rec);
         if (VS) gm_n = __ldg(p.v_gammas + rec);
         if (KS) gk_n = __ldg(p.k_gammas + rec);
       }
-    };
-    if (nmy > 0) load_norms();
-    for (int c = 0; c < nmy; ++c, it.next()) {     // no early exit: the named barriers must match
-      const int b = c & 1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[ST_EMPTY + rs.slot]);   // done with the stage
       const float nk = __half2float(__ushort_as_half(nk_n)), nv = __half2float(__ushort_as_half(nv_n));
       const float gm = VS ? __half2float(__ushort_as_half(gm_n)) : 0.0f;
       const float gk = KS ? __half2float(__ushort_as_half(gk_n)) : 0.0f;
-      const bool live = t < (it.cis == p.nchunk - 1 ? tail : kChunk);
-      if (c + 1 < nmy) {
-        nx.next();
-        load_norms();
-      }
       if (c == 0 || it.cis == 0) {
         vmax_run = gmax_run = 0.0f;
         const float4* hc = (const float4*)(p.head_c + it.slice * 32);
@@ -550,8 +680,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
           // key sign term alpha gamma <q'', 2z - 1> = alpha gamma (2 2^-F'' D_z - Q'')
           hs[i] = 2.0f * p.alpha * x.z * p.scale_log2e;
           hq[i] = -p.alpha * x.w * p.scale_log2e;
+          // virtual head h0 + i is query token (h0 + i) / Hgr of the pass
+          hlim[i] = (int)(p.tlim0 + (h0 + i) / p.Hgr);
         }
       }
+      const int tg = it.cis * kChunk + t;           // this thread's token, counted in the slice
       ok = mbar_wait_warp(&bar[SC_DONE + b], (c >> 1) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
       tc_fence_after();
       uint32_t dsr[4 * HH], dzr[KS ? 4 * HH : 1];
@@ -579,12 +712,13 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
                                 256.0f, small_i2f((int)dzr[4 * i]));
           sc = fmaf(gk, fmaf(hs[i], dz, hq[i]), sc);
         }
-        lg[i] = (h0 + i < Hg && live) ? nk * sc : -INFINITY;
+        lg[i] = (h0 + i < Hg && live && tg < hlim[i]) ? nk * sc : -INFINITY;
         up = up || lg[i] > mrun[i];
       }
       float corr[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) corr[i] = 1.0f;
+      bool changed = false;                         // a running maximum or a fixed-point scale moved
       if (bar_red_or(1 + 2 * gq, 128, up)) {
         // some token raised a running maximum: exchange the chunk maxima of the group's warps
         float* rb = rgrp + q * 16;
@@ -604,6 +738,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
           const float cm = fmaxf(fmaxf(rgrp[i], rgrp[16 + i]), fmaxf(rgrp[32 + i], rgrp[48 + i]));
           const float mn = fmaxf(mrun[i], cm);
           corr[i] = (mn == -INFINITY) ? 1.0f : fast_exp2(mrun[i] - mn);
+          changed = changed || mn != mrun[i];
           mrun[i] = mn;
         }
         vmax_run = fmaxf(vmax_run, fmaxf(fmaxf(rgrp[8], rgrp[24]), fmaxf(rgrp[40], rgrp[56])));
@@ -613,10 +748,12 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         frexpf(fmaxf(gmax_run, 1e-30f), &E2);
         E1 = max(E1, -80);
         E2 = max(E2, -80);
+        const float nisw = ldexpf(1.0f, E1 - 23), nisw2 = ldexpf(1.0f, E2 - 23);
+        changed = changed || nisw != isw || nisw2 != isw2;
         sw = ldexpf(1.0f, 23 - E1);                // w * sw <= 2^23 for every w <= vmax_run
         sw2 = ldexpf(1.0f, 23 - E2);               // likewise for w * gamma
-        isw = ldexpf(1.0f, E1 - 23);
-        isw2 = ldexpf(1.0f, E2 - 23);
+        isw = nisw;
+        isw2 = nisw2;
       }
       // weights: p = 2^(lg - m) <= 1, w = p |v|, w' = w gamma, as 24-bit unsigned fixed point
       uint32_t wv[HH], wz[HH], pv[HH];
@@ -655,23 +792,19 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       }
       fence_proxy_async_smem();
       if (q == 0 && lane == 0) {
-        // chunk scalars for the accumulators (4-deep ring): rescale factors, running maxima, scales
+        // chunk scalars for the value MMA warp (4-deep ring): running maxima, scales, and whether this
+        // group's maxima or scales moved (the chunk then starts a new run)
         float* sc = scal + (c & 3) * 64;
 #pragma unroll
-        for (int i = 0; i < HH; ++i) {
-          sc[h0 + i] = corr[i];
-          sc[16 + h0 + i] = mrun[i];
-        }
+        for (int i = 0; i < HH; ++i) sc[16 + h0 + i] = mrun[i];
         if (gq == 0) {
           sc[32] = isw;
           sc[33] = isw2;
         }
+        sc[34 + gq] = changed ? 1.0f : 0.0f;
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[BW_FULL + b]);
-        mbar_arrive(&bar[SCAL_FULL + (c & 3)]);
-      }
+      if (lane == 0) mbar_arrive(&bar[BW_FULL + b]);
     }
     (void)ok;
   } else if (warp < 14) {
@@ -685,9 +818,10 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       voff[2 * g] = sw128_offset(t, g * 32, 128);
       voff[2 * g + 1] = sw128_offset(t, g * 32 + 16, 128);
     }
-    for (int c = 0; c < nmy; ++c) {
-      const int st = c % nst, b = c & 1;
-      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / nst) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+    RingPos rs{0, nst, 0u};
+    for (int c = 0; c < nmy; ++c, rs.next()) {
+      const int st = rs.slot, b = c & 1;
+      if (!mbar_wait_warp(&bar[ST_FULL + st], rs.par, p.err, kDevTimeoutLoad, abort_flag)) break;
       if (c >= 2 && !mbar_wait_warp(&bar[SC_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
         break;
       tc_fence_after();
@@ -755,76 +889,72 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     }
   } else if (warp < 18) {
     // ------------------------------------ accumulators (thread = coordinate row) -------------------
+    // One pass per run: the run's limb sums from TMEM and its exact weight sums are folded in int64,
+    //   O_P = 2^s W - 2 Y_P (Walsh planes),  O_z = 2 Y_z - 2^s W' (sign plane),
+    // then added to the running state with the rescale from the previous run's maxima.
     const int q = warp & 3;
     const int m = q * 32 + lane;                 // TMEM lane = M index of the value MMA
     const int g = m >> 5, r = m & 31, s = r >> 2, jj = r & 3;
     const int coord = 32 * g + 8 * jj + s;       // coordinate this row holds
     const float rowscale = ldexpf(1.0f, -s);
-    const float two_s = ldexpf(1.0f, s);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int Hg = p.Hg;
     float acc[NP][HG];                           // folded planes O_P per head
     float Lr[HG];                                // sum of p
-    for (int c = 0; c < nmy; ++c, it.next()) {
-      const int b = c & 1;
-      if (c == 0 || it.cis == 0) {
+    float macc[HG];                              // maxima the state refers to
+    bool fresh = true;                           // the next run starts a segment
+    for (int R = 0; nmy > 0; ++R) {
+      const int nb = R & 1;
+      if (!mbar_wait_warp(&bar[RUN_DONE + nb], (R >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t col = tbase + lane_base + dv0 + nb * dv_cols;
+      const uint8_t* rr = smem + Lo.off_run + nb * kRunRec;
+      const float* rm = (const float*)rr;
+      const unsigned long long* rs = (const unsigned long long*)(rr + 64);
+      const int flags = *(const int*)(rr + 40);
+      const int seg = *(const int*)(rr + 44);
+      const int sgs = *(const int*)(rr + 48);
+      const float fw = rm[8] * rowscale, fz = rm[9] * rowscale;
+      if (fresh) {
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
           Lr[h] = 0.0f;
+          macc[h] = -INFINITY;
 #pragma unroll
           for (int P = 0; P < NP; ++P) acc[P][h] = 0.0f;
         }
       }
-      if (!mbar_wait_warp(&bar[SCAL_FULL + (c & 3)], (c >> 2) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      if (!mbar_wait_warp(&bar[V_DONE + c % 6], (c / 6) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t col = tbase + lane_base + dv0 + b * dv_cols;
-      uint32_t dv[NP][NQ];
-#pragma unroll
-      for (int P = 0; P < NP; ++P) {
-        tmem_ld16(col + P * NQ, *(uint32_t(*)[16]) & dv[P][0]);
-        if (NQ > 16) tmem_ld16(col + P * NQ + 16, *(uint32_t(*)[16]) & dv[P][NQ > 16 ? 16 : 0]);
-      }
-      // chunk sums of the weight kinds (four warp partials each), rescale factors, scales
-      const float* sc = scal + (c & 3) * 64;
-      const uint32_t* su = sums + (c & 3) * 96;
-      float corr[HG], Ws[HG], Zs[HG];
+      float corr[HG];
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
-        corr[h] = sc[h];
-        const uint32_t W = su[h] + su[24 + h] + su[48 + h] + su[72 + h];   // < 2^31
-        Ws[h] = (float)W * two_s;
-        if (VS) Zs[h] = (float)(su[8 + h] + su[32 + h] + su[56 + h] + su[80 + h]) * two_s;
-        if (m == 0) {
-          const uint32_t Lq = su[16 + h] + su[40 + h] + su[64 + h] + su[88 + h];
-          Lr[h] = fmaf(Lr[h], corr[h], (float)Lq * (1.0f / 4194304.0f));
-        }
+        const float mr = rm[h];
+        corr[h] = macc[h] == -INFINITY ? 0.0f : fast_exp2(macc[h] - mr);
+        macc[h] = mr;
+        if (m == 0) Lr[h] = fmaf(Lr[h], corr[h], (float)rs[16 + h] * (1.0f / 4194304.0f));
       }
-      const float fw = sc[32] * rowscale, fz = sc[33] * rowscale;
-      const bool last = c == nmy - 1 || it.cis == p.nchunk - 1;
-      float mseg[HG];                            // running maxima, read before the ring slot is released
-#pragma unroll
-      for (int h = 0; h < HG; ++h) mseg[h] = last ? sc[16 + h] : 0.0f;
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[DV_EMPTY + b]);
+      // one plane at a time (keeps the TMEM columns of a single plane in registers)
 #pragma unroll
       for (int P = 0; P < NP; ++P) {
         const bool sgn = VS && P == NP - 1;
+        uint32_t dv[NQ];
+        tmem_ld16(col + P * NQ, *(uint32_t(*)[16]) & dv[0]);
+        if (NQ > 16) tmem_ld16(col + P * NQ + 16, *(uint32_t(*)[16]) & dv[NQ > 16 ? 16 : 0]);
+        tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-          // Y = sum_t 2^s b w (limb sums below 2^22: exact), then the fold 2^s W - 2 Y (or 2 Y - 2^s W')
-          const float y = fmaf(fmaf(small_i2f((int)dv[P][4 * h + 2]), 256.0f, small_i2f((int)dv[P][4 * h + 1])), 256.0f,
-                               small_i2f((int)dv[P][4 * h]));
-          const float o = sgn ? fmaf(2.0f, y, -Zs[h]) : fmaf(-2.0f, y, Ws[h]);
-          acc[P][h] = fmaf(acc[P][h], corr[h], o * (sgn ? fz : fw));
+          // Y = sum over the run of 2^s b w (three 8-bit limb columns), exact in int64
+          const long long y = (long long)dv[4 * h] + ((long long)dv[4 * h + 1] << 8) + ((long long)dv[4 * h + 2] << 16);
+          const long long o = sgn ? 2 * y - ((long long)rs[8 + h] << s) : ((long long)rs[h] << s) - 2 * y;
+          acc[P][h] = fmaf(acc[P][h], corr[h], (float)o * (sgn ? fz : fw));
         }
       }
-      if (last) {
-        // this segment's partial state
-        const int sgs = it.slice;
-        const int seg = (c_begin + c) / p.per_cta - (sgs * p.nchunk) / p.per_cta;   // CTA ordinal inside the slice
+      // the buffer and the record may now be reused by the run after next
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[RUN_FREE + nb]);
+      fresh = (flags & 1) != 0;
+      if (fresh) {
+        // the last run of a segment: write the segment's partial state
         float* rec = p.partial + ((size_t)sgs * p.maxseg + seg) * Hg * att_rec(d);
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
@@ -833,7 +963,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 #pragma unroll
             for (int P = 0; P < NP; ++P) rh[4 + P * d + coord] = acc[P][h];
             if (m == 0) {
-              rh[0] = mseg[h];
+              rh[0] = macc[h];
               rh[1] = Lr[h];
               rh[2] = 1.0f;
               rh[3] = 0.0f;
@@ -841,22 +971,60 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
           }
         }
       }
+      if (flags & 2) break;
     }
   } else if (warp == 18) {
     // ------------------------------------ value MMA issuer (warp 18) ------------------------------
     // Runs beside the key MMA warp so that neither warp's barrier waits and commits sit behind the
-    // other's tensor-core work. Warp-uniform schedule, one elected lane issues.
+    // other's tensor-core work. Warp-uniform schedule, one elected lane issues. It also keeps the
+    // runs: a chunk whose softmax scalars moved starts a new run in the other TMEM buffer; lanes
+    // 0..23 add up the chunk weight sums of the run (kind lane / 8, head lane % 8) in 64 bits.
     const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
     const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
     const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
-    for (int c = 0; c < nmy; ++c) {
+    int R = -1, runlen = 0;
+    bool open = false;
+    unsigned long long rsum = 0;
+    auto close_run = [&](int flags, int seg) {
+      uint8_t* rr = smem + Lo.off_run + (R & 1) * kRunRec;
+      if (lane < 24) ((unsigned long long*)(rr + 64))[lane] = rsum;
+      if (lane == 0) {
+        *(int*)(rr + 40) = flags;
+        *(int*)(rr + 44) = seg;
+      }
+      __syncwarp();
+      if (elect_one_sync()) {
+        mma_commit(&bar[RUN_DONE + (R & 1)]);     // the run's MMAs are complete
+        mbar_arrive(&bar[RUN_DONE + (R & 1)]);    // and its record is written
+      }
+      __syncwarp();
+      open = false;
+    };
+    for (int c = 0; c < nmy; ++c, it.next()) {
       const int b = c & 1, c3 = c % 3;
       if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
       if (!mbar_wait_warp(&bar[AV_FULL + c3], (c / 3) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      if (c >= 2 && !mbar_wait_warp(&bar[DV_EMPTY + b], ((c >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
-        break;
+      const float* sc = scal + (c & 3) * 64;
+      const bool newrun = !open || sc[34] != 0.0f || sc[35] != 0.0f || runlen == kMaxRun;
+      if (newrun) {
+        if (open) close_run(0, 0);
+        ++R;
+        runlen = 0;
+        rsum = 0;
+        // the other buffer's previous run must have been drained by the accumulators
+        if (R >= 2 && !mbar_wait_warp(&bar[RUN_FREE + (R & 1)], ((R >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
+          break;
+        uint8_t* rr = smem + Lo.off_run + (R & 1) * kRunRec;
+        if (lane < 10) ((float*)rr)[lane] = lane < 8 ? sc[16 + lane] : sc[32 + lane - 8];
+        if (lane == 10) *(int*)(rr + 48) = it.slice;
+        open = true;
+      }
+      if (lane < 24) {
+        const uint32_t* su = sums + (c & 3) * 96 + lane;
+        rsum += (unsigned long long)((su[0] + su[24]) + (su[48] + su[72]));   // four warp partials, < 2^31
+      }
       tc_fence_after();
-      const uint32_t dcol = tbase + dv0 + b * dv_cols;
+      const uint32_t dcol = tbase + dv0 + (R & 1) * dv_cols;
       const uint64_t da = da0 + ((c3 * NP * Lo.av_bytes) >> 4);
       const uint64_t db = db0 + ((b * Lo.bw_buf) >> 4);
       if (elect_one_sync()) {
@@ -866,11 +1034,16 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 #pragma unroll
           for (int ks = 0; ks < kChunk / 32; ++ks)
             mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
-                      db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, ks > 0);
+                      db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, (ks > 0 || !newrun) ? 1u : 0u);
         }
         mma_commit(&bar[V_DONE + c % 6]);
       }
       __syncwarp();
+      ++runlen;
+      if (c == nmy - 1 || it.cis == p.nchunk - 1) {
+        const int seg = (c_begin + c) / p.per_cta - (it.slice * p.nchunk) / p.per_cta;   // CTA ordinal in the slice
+        close_run(1 | (c == nmy - 1 ? 2 : 0), seg);
+      }
     }
   } else if (SPLITV) {
     // ------------------------------------ value expanders (warps 19-22, thread = token) -----------
@@ -882,9 +1055,10 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       voff[2 * g] = sw128_offset(t, g * 32, 128);
       voff[2 * g + 1] = sw128_offset(t, g * 32 + 16, 128);
     }
-    for (int c = 0; c < nmy; ++c) {
-      const int st = c % nst, c3 = c % 3;
-      if (!mbar_wait_warp(&bar[ST_FULL + st], (c / nst) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
+    RingPos rs{0, nst, 0u};
+    for (int c = 0; c < nmy; ++c, rs.next()) {
+      const int st = rs.slot, c3 = c % 3;
+      if (!mbar_wait_warp(&bar[ST_FULL + st], rs.par, p.err, kDevTimeoutLoad, abort_flag)) break;
       // the planes of chunk c - 3 (same buffer) must have been consumed
       if (c >= 3 && !mbar_wait_warp(&bar[V_DONE + (c - 3) % 6], ((c - 3) / 6) & 1, p.err, kDevTimeoutMma, abort_flag))
         break;
@@ -911,10 +1085,10 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 // combine: merge the partial states of a slice, apply Pi^T and alpha S^T once per query head
 // ------------------------------------------------------------------------------------------------
 __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
-  const int bh = blockIdx.x;                 // b * Hq + hq
-  const int b = bh / p.Hq, hq = bh % p.Hq;
-  const int hk = hq / p.Hg, h = hq % p.Hg;
-  const int slice = b * p.Hkv + hk;
+  const int slice = blockIdx.x / p.Hg;       // one block per (slice, virtual head)
+  const int h = blockIdx.x % p.Hg;
+  const int b = slice / p.Hkv, hk = slice % p.Hkv;
+  const size_t ooff = (size_t)b * p.q_bs + (size_t)(h / p.Hgr) * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * p.d;
   const int d = p.d, i = threadIdx.x;
   __shared__ float orot[128], osgn[128];
   __shared__ float mmax, linv;
@@ -969,7 +1143,7 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
       }
       acc = fmaf(p.alpha, (z[0] + z[1]) + (z[2] + z[3]), acc);
     }
-    p.out[(size_t)bh * d + i] = acc;
+    p.out[ooff + i] = acc;
   }
 }
 
@@ -996,13 +1170,20 @@ struct AttPlan {
   size_t bq_bytes, hc_bytes, part_bytes, total;
 };
 
-bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl) {
+// Plan of one pass over T tokens of every slice with nqry query tokens per slice (Hg = nqry x Hq/Hkv
+// virtual heads, at most 8).
+bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl, int nqry = 1) {
   AttParams& p = pl.p;
   p = AttParams{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.Hg = Hq / Hkv;
+  p.Hgr = Hq / Hkv;
+  p.nqry = nqry;
+  p.Hg = nqry * p.Hgr;
+  p.q_bs = (int64_t)Hq * d;
+  p.q_js = 0;
+  p.tlim0 = T;
   p.d = d;
   p.G = d / 32;
   p.T = T;
@@ -1013,9 +1194,9 @@ bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl) {
   const int ncta = (int)std::min<long long>(nsm, totalc);
   p.per_cta = (int)((totalc + ncta - 1) / ncta);
   p.maxseg = (p.nchunk + p.per_cta - 1) / p.per_cta + 1;
-  p.nq = p.Hg <= 4 ? 16 : 32;      // the kernel is built for 4 or 8 heads per KV head
+  p.nq = p.Hg <= 4 ? 16 : 32;      // the kernel is built for 4 or 8 (virtual) heads per KV head
   pl.bq_bytes = (size_t)p.slices * p.nq * 4 * d;       // mk <= 4
-  pl.hc_bytes = (size_t)p.slices * 16 * sizeof(float);
+  pl.hc_bytes = (size_t)p.slices * 8 * 4 * sizeof(float);   // head_c [slices][8 heads][4]
   pl.part_bytes = (size_t)p.slices * p.maxseg * p.Hg * att_rec(d) * sizeof(float);
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   pl.total = al(pl.bq_bytes) + al(pl.hc_bytes) + al(pl.part_bytes);
@@ -1042,13 +1223,35 @@ extern "C" TQ_API size_t tq_attend_workspace_bytes(int32_t B, int32_t Hq, int32_
 }
 
 namespace tq {
-// Decode attention over T tokens of every slice, whose records lie tstride apart (tstride >= T).
-tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
-                      int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
-                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
-                      const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
-                      const uint16_t* v_norms, const uint16_t* v_gammas, float scale, float* out, void* ws,
-                      size_t ws_bytes, void* stream) {
+namespace {
+// Geometry of one attention pass: nqry query tokens per slice, q / out strides, causal limit.
+struct PassGeom {
+  int nqry;                      // query tokens per slice in this pass (1 for decode)
+  int64_t q_bs, q_js;            // element strides of q / out: batch, query token
+  int64_t q_off;                 // element offset of the pass's first query token
+  int64_t tlim0;                 // query token j of the pass attends t < tlim0 + j
+};
+
+// The new token of every slice for tq_attend_append (written into slot t_new by the prep kernel).
+struct AppendArgs {
+  const void* k_new;
+  const void* v_new;
+  int x_dtype;
+  int64_t t_new;
+  uint32_t* k_codes;
+  uint16_t* k_norms;
+  uint32_t* v_codes;
+  uint32_t* v_signs;
+  uint16_t* v_norms;
+  uint16_t* v_gammas;
+};
+
+// Argument checks shared by the attention entry points (no work is enqueued on failure).
+tq_status attend_check(const std::string& f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                       int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
+                       const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                       const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
+                       const uint16_t* v_norms, const uint16_t* v_gammas, const float* out, const void* ws) {
   if (!cb_k || !cb_v || !q || !rot || !k_codes || !k_norms || !v_codes || !v_norms || !out || !ws)
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": NULL pointer");
   if ((v_signs == nullptr) != (v_gammas == nullptr))
@@ -1081,12 +1284,29 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
       !aligned16(ws) ||
       !aligned16(rot) || !aligned16(out))
     return fail(TQ_ERR_INVALID_ARG, std::string(f) + ": pointers must be 16-byte aligned");
+  return TQ_OK;
+}
+
+// One pass: prep, main and combine kernels over the first T tokens of every slice.
+tq_status attend_pass(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                      int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
+                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                      const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
+                      const uint16_t* v_norms, const uint16_t* v_gammas, float scale, float* out, void* ws,
+                      size_t ws_bytes, void* stream, const PassGeom& g, const AppendArgs* app = nullptr) {
+  const bool ksign = k_signs != nullptr;
+  const bool vsign = v_signs != nullptr;
   AttPlan pl;
-  att_plan(B, Hq, Hkv, T, d, sm_count(), pl);
-  if (ws_bytes < pl.total || ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
-    return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
+  att_plan(B, Hq, Hkv, T, d, sm_count(), pl, g.nqry);
+  if (ws_bytes < pl.total) return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
   AttParams& p = pl.p;
   p.tstride = tstride;
+  p.q_bs = g.q_bs;
+  p.q_js = g.q_js;
+  p.tlim0 = g.tlim0;
+  const size_t esz = q_dtype == TQ_BF16 ? 2 : 4;
+  q = (const uint8_t*)q + (size_t)g.q_off * esz;
+  out += g.q_off;
   int kmask[8], vmask[8];
   float kbeta[8], vbeta[8];
   p.bk = cb_k->bits;
@@ -1098,6 +1318,8 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   for (int i = 0; i < p.mv; ++i) p.beta_v[i] = vbeta[i];
   p.vsign = vsign ? 1 : 0;
   p.np = p.mv + p.vsign;
+  // scale <= 0 (or NaN) selects the plain attention scale 1/sqrt(d)
+  if (!(scale > 0.0f)) scale = (float)(1.0 / std::sqrt((double)d));
   p.scale_log2e = scale * kLog2e;
   p.alpha = (float)(std::sqrt(M_PI / 2.0) / d);
   p.q = q;
@@ -1119,6 +1341,26 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   p.head_c = (float*)(w + al(pl.bq_bytes));
   p.partial = (float*)(w + al(pl.bq_bytes) + al(pl.hc_bytes));
   p.out = out;
+  p.norm_bulk = (tstride % 8 == 0) && aligned16(k_norms) && aligned16(v_norms) && (!v_gammas || aligned16(v_gammas)) &&
+                (!k_gammas || aligned16(k_gammas));
+  if (app) {
+    p.k_new = app->k_new;
+    p.v_new = app->v_new;
+    p.x_bf16 = app->x_dtype == TQ_BF16;
+    p.t_new = app->t_new;
+    p.kw_codes = app->k_codes;
+    p.kw_norms = app->k_norms;
+    p.vw_codes = app->v_codes;
+    p.vw_signs = app->v_signs;
+    p.vw_norms = app->v_norms;
+    p.vw_gammas = app->v_gammas;
+    for (int k = 0; k < 8; ++k) {
+      p.ck[k] = k < cb_k->levels ? cb_k->c[k] : 0.0f;
+      p.tk[k] = k < cb_k->levels - 1 ? cb_k->t[k] : 0.0f;
+      p.cv[k] = k < cb_v->levels ? cb_v->c[k] : 0.0f;
+      p.tv[k] = k < cb_v->levels - 1 ? cb_v->t[k] : 0.0f;
+    }
+  }
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, std::string(f) + ": no device error word");
   const AttLayout L0 = att_layout(p, 0);
@@ -1131,13 +1373,46 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   const AttLayout Lo = att_layout(p, nst);
   const MainKernel kern = pick_main(p.Hg, p.bk, p.bv, p.vsign, p.ksign);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode: shared memory attribute");
+  if (e != cudaSuccess) return cuda_fail(e, (std::string(f) + ": shared memory attribute").c_str());
   const long long totalc = (long long)p.slices * p.nchunk;
   const int grid = (int)((totalc + p.per_cta - 1) / p.per_cta);
   kern<<<grid, 32 * att_warps(p.Hg <= 4 ? 4 : 8), Lo.total, st>>>(p);
-  attend_combine_kernel<<<B * Hq, 128, 0, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tq_attend_decode: launch");
+  attend_combine_kernel<<<p.slices * p.Hg, 128, 0, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, (std::string(f) + ": launch").c_str());
   return TQ_OK;
+}
+
+// Query tokens per pass of a prefill: as many as keep the virtual heads at 8 or fewer.
+int prefill_qpass(int Hg) { return std::max(1, 8 / Hg); }
+
+size_t prefill_ws(int32_t B, int32_t Hq, int32_t Hkv, int32_t Qn, int64_t T, int32_t d, int nsm) {
+  const int qp = prefill_qpass(Hq / Hkv);
+  size_t need = 0;
+  for (int j0 = 0; j0 < Qn; j0 += qp) {
+    const int nq = std::min(qp, Qn - j0);
+    AttPlan pl;
+    att_plan(B, Hq, Hkv, T - Qn + j0 + nq, d, nsm, pl, nq);
+    need = std::max(need, pl.total);
+  }
+  return need;
+}
+}  // namespace
+
+// Decode attention over T tokens of every slice, whose records lie tstride apart (tstride >= T).
+tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                      int32_t Hkv, int64_t T, int64_t tstride, int32_t d, const void* q, int32_t q_dtype,
+                      const void* rot, const uint32_t* k_codes, const uint16_t* k_norms, const uint32_t* k_signs,
+                      const uint16_t* k_gammas, const uint32_t* v_codes, const uint32_t* v_signs,
+                      const uint16_t* v_norms, const uint16_t* v_gammas, float scale, float* out, void* ws,
+                      size_t ws_bytes, void* stream) {
+  tq_status st = attend_check(f, cb_k, cb_v, B, Hq, Hkv, T, tstride, d, q, q_dtype, rot, k_codes, k_norms, k_signs,
+                              k_gammas, v_codes, v_signs, v_norms, v_gammas, out, ws);
+  if (st != TQ_OK) return st;
+  if (ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
+    return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
+  PassGeom g{1, (int64_t)Hq * d, 0, 0, T};
+  return attend_pass(f, cb_k, cb_v, B, Hq, Hkv, T, tstride, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas,
+                     v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g);
 }
 }  // namespace tq
 
@@ -1151,4 +1426,83 @@ extern "C" TQ_API tq_status tq_attend_decode(const tq_codebook* cb_k, const tq_c
   clear_error();
   return attend_impl("tq_attend_decode", cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs,
                      k_gammas, v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream);
+}
+
+extern "C" TQ_API size_t tq_attend_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Qn, int64_t T,
+                                                           int32_t d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Qn <= 0 || T < Qn || d <= 0 || Hq % Hkv) return 0;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      nsm <= 0) {
+    cudaGetLastError();
+    nsm = 148;
+  }
+  return prefill_ws(B, Hq, Hkv, Qn, T, d, nsm);
+}
+
+extern "C" TQ_API tq_status tq_attend_prefill(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                              int32_t Hkv, int32_t Qn, int64_t T, int32_t d, const void* q,
+                                              int32_t q_dtype, const void* rot, const uint32_t* k_codes,
+                                              const uint16_t* k_norms, const uint32_t* k_signs,
+                                              const uint16_t* k_gammas, const uint32_t* v_codes,
+                                              const uint32_t* v_signs, const uint16_t* v_norms,
+                                              const uint16_t* v_gammas, float scale, float* out, void* ws,
+                                              size_t ws_bytes, void* stream) {
+  clear_error();
+  const char* f = "tq_attend_prefill";
+  if (Qn <= 0 || T < Qn) return fail(TQ_ERR_INVALID_ARG, "tq_attend_prefill: need 1 <= Qn <= T");
+  tq_status st = attend_check(f, cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas,
+                              v_codes, v_signs, v_norms, v_gammas, out, ws);
+  if (st != TQ_OK) return st;
+  if (ws_bytes < tq_attend_prefill_workspace_bytes(B, Hq, Hkv, Qn, T, d))
+    return fail(TQ_ERR_WORKSPACE, "tq_attend_prefill: workspace too small");
+  const int qp = prefill_qpass(Hq / Hkv);
+  for (int j0 = 0; j0 < Qn; j0 += qp) {
+    const int nq = std::min(qp, Qn - j0);
+    // query token j (0-based among the Qn new tokens) sits at cache position T - Qn + j and sees
+    // the tokens t <= T - Qn + j; the pass covers exactly the tokens its last query sees
+    const int64_t Tp = T - Qn + j0 + nq;
+    PassGeom g{nq, (int64_t)Qn * Hq * d, (int64_t)Hq * d, (int64_t)j0 * Hq * d, T - Qn + j0 + 1};
+    st = attend_pass(f, cb_k, cb_v, B, Hq, Hkv, Tp, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas, v_codes,
+                     v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g);
+    if (st != TQ_OK) return st;
+  }
+  return TQ_OK;
+}
+
+extern "C" TQ_API size_t tq_attend_append_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t T_cur, int32_t d,
+                                                          int32_t k_bits, int32_t v_codebook_bits) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || T_cur < 0 || d <= 0 || d % 32 || Hq % Hkv || k_bits < 1 || k_bits > 4 ||
+      v_codebook_bits < 1 || v_codebook_bits > 4)
+    return 0;
+  return tq_attend_workspace_bytes(B, Hq, Hkv, T_cur + 1, d);
+}
+
+// tq_attend_append: one decode step on a packed KV cache with room to grow. The prep kernel encodes
+// each slice's new key (Algorithm 1) and value (Algorithm 2) into slot T_cur (ai-navigate-news page:
+// keys by Algorithm 1, values by Algorithm 2, appended as tokens are generated), then the main and
+// combine kernels attend over the T_cur + 1 filled slots: three launches in all.
+extern "C" TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_codebook* cb_v, int32_t B, int32_t Hq,
+                                             int32_t Hkv, int64_t T_cur, int64_t T_max, int32_t d, const void* q,
+                                             int32_t q_dtype, const void* k_new, const void* v_new, int32_t x_dtype,
+                                             const void* rot, uint32_t* k_codes, uint16_t* k_norms,
+                                             uint32_t* v_codes, uint32_t* v_signs, uint16_t* v_norms,
+                                             uint16_t* v_gammas, float scale, float* out, void* ws, size_t ws_bytes,
+                                             void* stream) {
+  clear_error();
+  const char* f = "tq_attend_append";
+  if (!k_new || !v_new || !v_signs || !v_gammas)
+    return fail(TQ_ERR_INVALID_ARG, "tq_attend_append: NULL pointer (values are Algorithm 2: signs and gammas are required)");
+  if (T_cur < 0 || T_max < T_cur + 1) return fail(TQ_ERR_INVALID_ARG, "tq_attend_append: need 0 <= T_cur < T_max");
+  if (x_dtype != TQ_F32 && x_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, "tq_attend_append: k_new / v_new dtype");
+  const int64_t T = T_cur + 1;
+  tq_status st = attend_check(f, cb_k, cb_v, B, Hq, Hkv, T, T_max, d, q, q_dtype, rot, k_codes, k_norms, nullptr,
+                              nullptr, v_codes, v_signs, v_norms, v_gammas, out, ws);
+  if (st != TQ_OK) return st;
+  if (ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
+    return fail(TQ_ERR_WORKSPACE, "tq_attend_append: workspace too small");
+  const AppendArgs app{k_new, v_new, x_dtype, T_cur, k_codes, k_norms, v_codes, v_signs, v_norms, v_gammas};
+  PassGeom g{1, (int64_t)Hq * d, 0, 0, T};
+  return attend_pass(f, cb_k, cb_v, B, Hq, Hkv, T, T_max, d, q, q_dtype, rot, k_codes, k_norms, nullptr, nullptr,
+                     v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g, &app);
 }

@@ -2,10 +2,13 @@
 
 A compact cache of T_cur + 1 tokens is encoded with the plain encoders; its first T_cur tokens are
 copied into a larger cache of T_max slots per slice whose other slots hold a sentinel, and
-tq_attend_append appends the last token's raw K / V. Checked:
-  * the appended slot holds exactly the records the plain encoders made for that token, earlier
-    slots are unchanged and later slots still hold the sentinel;
-  * the output equals tq_attend_decode over the compact cache bit for bit (same kernels, same
+tq_attend_append appends the last token's raw K / V (its prep kernel encodes them in fp64).
+Checked:
+  * the appended slot holds the oracle's encoding of that token (keys Algorithm 1, values
+    Algorithm 2): codes and signs exact outside the 1e-5 band of a decision, fp16 norms / gammas
+    exact up to the 2^-20 midpoint rule; earlier slots are unchanged and later slots still hold the
+    sentinel;
+  * the output equals tq_attend_decode over the first T_cur + 1 slots bit for bit (same kernels, same
     split of the chunks, the cache read with a slot stride);
   * the output matches the oracle's fp64 attention over the dequantised cache (1e-3 normwise).
 """
@@ -13,7 +16,9 @@ import numpy as np
 import pytest
 
 import workloads as W
-from parity import normwise_rel
+from oracle import quant as Q
+from oracle.codebook import lloyd_max
+from parity import check_codes, check_fp16, check_signs, normwise_rel, np_f16, np_u32
 from test_gpu_attend import make_cache, oracle_attention
 
 pytestmark = pytest.mark.gpu
@@ -68,27 +73,41 @@ def test_append_then_attend(dev, B, Hq, Hkv, T_cur, T_max):
                         vn, vg, out)
     tq.tq_sync_check()
 
-    # records: slot T_cur equals the compact cache's last token, the rest is as before
-    compact = [cache["kc"].view(B, Hkv, T, G, kb), cache["vc"].view(B, Hkv, T, G, vb - 1),
-               cache["vs"].view(B, Hkv, T, G), cache["kn"].view(B, Hkv, T), cache["vn"].view(B, Hkv, T),
-               cache["vg"].view(B, Hkv, T)]
-    for now, was, c in zip((kc, vc, vs, kn, vn, vg), before, compact):
+    # records: slot T_cur holds the oracle's encoding of the new token, the rest is as before
+    Pi, S = cache["Pi"], cache["S"]
+    kx = K[:, :, T_cur].reshape(B * Hkv, d)
+    vx = V[:, :, T_cur].reshape(B * Hkv, d)
+    okb, ovb = lloyd_max(d, kb), lloyd_max(d, vb - 1)
+    ek = Q.encode_mse(kx, Pi, okb)
+    ev = Q.encode_prod(vx, Pi, S, ovb)
+    gk = np_u32(kc[:, :, T_cur].contiguous()).reshape(B * Hkv, G, kb)
+    gv = np_u32(vc[:, :, T_cur].contiguous()).reshape(B * Hkv, G, vb - 1)
+    check_codes(gk, ek["idx"], ek["y"], okb.t32, kb, d)
+    check_codes(gv, ev["idx"], ev["y"], ovb.t32, vb - 1, d)
+    gidx = Q.unpack_planes(gv, vb - 1)
+    ev2 = Q.residual_signs(ev["u"], gidx, ev["n"], Pi, S, ovb)
+    check_signs(np_u32(vs[:, :, T_cur].contiguous()).reshape(B * Hkv, G), ev2["z"], ev2["s"], ev2["gamma"], d)
+    check_fp16(np_f16(kn[:, :, T_cur].contiguous()).reshape(-1), ek["n"], "key norms")
+    check_fp16(np_f16(vn[:, :, T_cur].contiguous()).reshape(-1), ev["n"], "value norms")
+    check_fp16(np_f16(vg[:, :, T_cur].contiguous()).reshape(-1), ev2["gamma"], "gammas")
+    for now, was in zip((kc, vc, vs, kn, vn, vg), before):
         a = now.view(torch.int16) if now.dtype == torch.float16 else now
         b_ = was.view(torch.int16) if was.dtype == torch.float16 else was
-        cc = c.view(torch.int16) if c.dtype == torch.float16 else c
-        assert torch.equal(a[:, :, T_cur], cc[:, :, T_cur])
         assert torch.equal(a[:, :, :T_cur], b_[:, :, :T_cur])
         assert torch.equal(a[:, :, T_cur + 1:], b_[:, :, T_cur + 1:])
 
-    # the same attention over the compact cache, bit for bit
+    # the same attention over the first T_cur + 1 slots as a compact cache, bit for bit
+    cut = lambda t: t[:, :, :T].contiguous()
+    ckc, ckn, cvc, cvs, cvn, cvg = (cut(t) for t in (kc, kn, vc, vs, vn, vg))
     ref = torch.empty_like(out)
-    tq.tq_attend_decode(cache["cbk"], cache["cbv"], q, cache["rot"], cache["kc"], cache["kn"].view(B, Hkv, T),
-                        cache["vc"], cache["vn"].view(B, Hkv, T), ref, v_signs=cache["vs"],
-                        v_gammas=cache["vg"].view(B, Hkv, T))
+    tq.tq_attend_decode(cache["cbk"], cache["cbv"], q, cache["rot"], ckc.view(-1, G, kb), ckn, cvc.view(-1, G, vb - 1),
+                        cvn, ref, v_signs=cvs.view(-1, G), v_gammas=cvg)
     tq.tq_sync_check()
     assert torch.equal(out, ref)
 
-    want = oracle_attention(cache, q_np, B, Hq, Hkv, T, d)
+    # the oracle over the cache as the GPU wrote it
+    grown = dict(cache, kc=ckc, kn=ckn, vc=cvc, vs=cvs, vn=cvn, vg=cvg)
+    want = oracle_attention(grown, q_np, B, Hq, Hkv, T, d)
     got = out.cpu().numpy()
     rel = np.array([normwise_rel(got[b, h], want[(b, h)]) for (b, h) in want])
     print("append", (B, Hq, Hkv, T_cur, T_max), "max rel", rel.max())

@@ -103,13 +103,13 @@ def test_attend_append_rejects_bad_arguments_on_host(L):
                                                 tq.TQ_BF16, g, g, tq.TQ_BF16, g, g, g, g, vs, g, g, ctypes.c_float(0.1), g,
                                                 g, ws_bytes, None)
     need = L.tq_attend_append_workspace_bytes(2, 8, 2, 10, 128, 3, 1)
-    assert need > L.tq_attend_workspace_bytes(2, 8, 2, 11, 128)
+    assert need == L.tq_attend_workspace_bytes(2, 8, 2, 11, 128)      # the attention's own workspace
     assert L.tq_attend_append_workspace_bytes(2, 8, 2, -1, 128, 3, 1) == 0
     assert L.tq_attend_append(*args(10, 10, need)) == tq.TQ_ERR_INVALID_ARG        # no free slot
     assert L.tq_attend_append(*args(-1, 10, need)) == tq.TQ_ERR_INVALID_ARG
     assert L.tq_attend_append(*args(10, 20, need, vs=None)) == tq.TQ_ERR_INVALID_ARG   # values are Algorithm 2
     assert L.tq_attend_append(*args(10, 20, need - 1)) == tq.TQ_ERR_WORKSPACE
-    # the attention's own limits are checked before the encoders touch the cache
+    # the attention's limits are checked before anything touches the cache
     cb64 = tq.tq_codebook_init(64, 3)
     bad_d = (ctypes.byref(cb64), ctypes.byref(tq.tq_codebook_init(64, 1)), 2, 8, 2, 10, 20, 64, g, tq.TQ_BF16, g, g,
              tq.TQ_BF16, g, g, g, g, g, g, g, ctypes.c_float(0.1), g, g, need, None)
@@ -130,3 +130,46 @@ def test_binding_signatures_match_the_header(L):
     for name, (_res, args) in tq._SIGNATURES.items():
         assert name in protos, name
         assert len(args) == protos[name], (name, len(args), protos[name])
+
+
+def test_selftest_wait_rejects_bad_limits_on_host(L):
+    for lim in (0, 999, 2_000_000_000):
+        assert L.tq_selftest_wait(lim, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_attend_prefill_rejects_bad_arguments_on_host(L):
+    cbk, cbv = tq.tq_codebook_init(128, 3), tq.tq_codebook_init(128, 1)
+    P = ctypes.c_void_p
+    g = P(1 << 20)
+    need = L.tq_attend_prefill_workspace_bytes(2, 8, 2, 5, 700, 128)
+    assert need >= L.tq_attend_workspace_bytes(2, 8, 2, 700, 128) > 0
+    assert L.tq_attend_prefill_workspace_bytes(2, 8, 2, 0, 700, 128) == 0
+    assert L.tq_attend_prefill_workspace_bytes(2, 8, 2, 701, 700, 128) == 0
+    args = lambda Qn, T, ws_bytes: (ctypes.byref(cbk), ctypes.byref(cbv), 2, 8, 2, Qn, T, 128, g, tq.TQ_BF16, g, g, g,
+                                    None, None, g, g, g, g, ctypes.c_float(0.0), g, g, ws_bytes, None)
+    assert L.tq_attend_prefill(*args(0, 700, need)) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_attend_prefill(*args(701, 700, need)) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_attend_prefill(*args(5, 700, need - 1)) == tq.TQ_ERR_WORKSPACE
+
+
+def test_mixed_width_calls_reject_bad_arguments_on_host(L):
+    d = 128
+    cbs = (tq.Codebook * 4)()
+    for b in (1, 2, 3, 4):
+        cbs[b - 1] = tq.tq_codebook_init(d, b)
+    P = ctypes.c_void_p
+    g = P(1 << 20)
+    gb = lambda *w: (ctypes.c_int32 * len(w))(*w)
+    ok = gb(3, 3, 2, 2)
+    assert L.tq_encode_mse_mixed(cbs, gb(3, 3, 2, 5), 10, d, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse_mixed(cbs, gb(3, 3, 0, 2), 10, d, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse_mixed(cbs, ok, 10, 256, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse_mixed(cbs, ok, -1, d, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_encode_mse_mixed(cbs, ok, 10, d, P((1 << 20) + 4), tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_INVALID_ARG
+    wrong = (tq.Codebook * 4)()
+    wrong[2] = tq.tq_codebook_init(d, 2)                  # a 2-bit codebook where the 3-bit one belongs
+    wrong[1] = tq.tq_codebook_init(d, 2)
+    assert L.tq_encode_mse_mixed(wrong, ok, 10, d, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_decode_mixed(cbs, gb(3, 3, 2, 9), 10, d, g, g, g, g, tq.TQ_F32, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_decode_mixed(cbs, ok, 10, d, g, g, g, g, tq.TQ_F16, None) == tq.TQ_ERR_UNSUPPORTED
+    assert L.tq_encode_mse_mixed(cbs, ok, 0, d, g, tq.TQ_BF16, g, g, g, None) == tq.TQ_OK      # n = 0: no work
