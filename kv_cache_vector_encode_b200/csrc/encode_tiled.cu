@@ -19,7 +19,11 @@
 // Precision: products exact in the tensor core, fp32 accumulation over K = d. For large d the
 // accumulated rounding approaches the parity band, so a decision whose value lies within 20x the
 // band of a boundary (a quantiser boundary, or zero for a sign) is recomputed exactly in fp64 from
-// the fp32 matrices -- rare (about 1e-4 of the coordinates) and off the fast path.
+// the fp32 matrices -- rare (about 1e-4 of the coordinates) and off the fast path. The same holds
+// for the fp16 rounding of gamma = |r|: a gamma within 2^-15 (relative) of an fp16 rounding
+// midpoint, far wider than the fp32 accumulation error, is flagged, and a fix-up kernel recomputes
+// r = x / |x| - Pi^T c[idx] for that vector in fp64 from x, the fp32 Pi and the vector's own codes,
+// and rewrites gamma (a few percent of the vectors; about d^2 fp64 operations each).
 //
 // Roles (10 warps): 0 TMA / bulk copies; 1 TMEM owner and MMA issuer; 2-5 converters (thread =
 // vector: fp64 norm, fp16 split of x, copies of the rho images); 6-9 epilogue (thread = vector).
@@ -57,6 +61,7 @@ struct TEParams {
   uint16_t* gammas;
   uint8_t* rho;              // per-CTA slots of slot_bytes: [KB][hi, lo][kBlk]
   size_t slot_bytes;
+  uint32_t* gflag;           // one bit per vector: gamma next to an fp16 rounding midpoint (Algorithm 2)
   const void* x;             // the input (exact recomputation of decisions next to a boundary)
   const float* pi32;         // fp32 Pi, row-major
   const float* t32;          // fp32 T = S Pi^T, row-major
@@ -135,6 +140,84 @@ __device__ __noinline__ double exact_sign_value(const float* srow, const float* 
     tc = fma((double)trow[k], neg ? -(double)cm : (double)cm, tc);
   }
   return sx - tc;
+}
+
+constexpr double kGammaFixTol = 1.0 / 32768.0;   // 2^-15: flag gamma this close to an fp16 midpoint
+
+// True when x > 0 lies within tol (relative) of the midpoint between its fp16 rounding and the
+// neighbouring fp16 value on x's side, i.e. where a small error in x could flip the rounding.
+__device__ __forceinline__ bool near_f16_midpoint(double x, double tol) {
+  const __half h = __double2half(x);
+  const double hd = (double)__half2float(h);
+  const unsigned short hb = __half_as_ushort(h);
+  if (hb >= 0x7BFFu) return false;                       // at or past the largest finite value
+  const unsigned short nb = (x >= hd) ? (unsigned short)(hb + 1u) : (hb == 0u ? hb : (unsigned short)(hb - 1u));
+  const double mid = 0.5 * (hd + (double)__half2float(__ushort_as_half(nb)));
+  return fabs(x - mid) <= tol * x;
+}
+
+// Exact gamma for the flagged vectors: r = x / |x| - Pi^T c[idx] in fp64 (original domain, the
+// vector's own codes), gamma = |r| rounded to fp16. One block of 256 threads per flagged vector.
+template <bool F32, int BITS>
+__global__ void __launch_bounds__(256) gamma_fixup_kernel(const __grid_constant__ TEParams p, int nwords) {
+  extern __shared__ double fx[];                      // [d] x (fp64), [d] c[idx] (fp64)
+  __shared__ double red[8];
+  const int d = p.d, G = p.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  double* xs = fx;
+  double* cs = fx + d;
+  constexpr int H = 1 << (BITS - 1);
+  auto block_sum = [&](double v) -> double {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w];
+    return t;
+  };
+  for (int wi = blockIdx.x; wi < nwords; wi += gridDim.x) {
+    uint32_t bits = p.gflag[wi];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      const int64_t v = (int64_t)wi * 32 + b;
+      double ss = 0.0;
+      for (int j = tid; j < d; j += 256) {
+        const double xj = F32 ? (double)((const float*)p.x)[v * d + j]
+                              : (double)__uint_as_float((uint32_t)((const uint16_t*)p.x)[v * d + j] << 16);
+        xs[j] = xj;
+        ss = fma(xj, xj, ss);
+      }
+      const double nrm = sqrt(block_sum(ss));
+      const uint32_t* vc = p.codes + (size_t)v * G * BITS;
+      for (int i = tid; i < d; i += 256) {
+        const uint32_t* wk = vc + (i >> 5) * BITS;
+        const int l = i & 31;
+        const bool neg = ((wk[BITS - 1] >> l) & 1u) == 0u;
+        int m = 0;
+        for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> l) & 1u) << pl;
+        if (neg) m ^= H - 1;
+        float cm = p.C[0];
+#pragma unroll
+        for (int q = 1; q < H; ++q)
+          if (q == m) cm = p.C[q];
+        cs[i] = neg ? -(double)cm : (double)cm;
+      }
+      __syncthreads();
+      double g2 = 0.0;
+      for (int j = tid; j < d; j += 256) {
+        double a = 0.0;                                  // (Pi^T c)_j = sum_i Pi[i][j] c_i
+        for (int i = 0; i < d; ++i) a = fma((double)__ldg(p.pi32 + (size_t)i * d + j), cs[i], a);
+        const double r = xs[j] / nrm - a;
+        g2 = fma(r, r, g2);
+      }
+      g2 = block_sum(g2);
+      if (tid == 0) p.gammas[v] = __half_as_ushort(__double2half(sqrt(g2)));
+      __syncthreads();
+    }
+  }
 }
 
 template <bool F32, bool ALG2, int BITS>
@@ -576,7 +659,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
           if (live) *(uint4*)(p.signs + (size_t)v * G + 4 * nb) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
         }
         if (!ok) break;
-        if (live) p.gammas[v] = __half_as_ushort(__double2half(sqrt(g2)));
+        if (live) {
+          const double gam = sqrt(g2);
+          p.gammas[v] = __half_as_ushort(__double2half(gam));
+          if (gam > 0.0 && near_f16_midpoint(gam, kGammaFixTol)) atomicOr(p.gflag + (v >> 5), 1u << (v & 31));
+        }
       }
     }
   }
@@ -599,7 +686,17 @@ tq_status launch_tiled(TEParams& p, const void* x, int grid, cudaStream_t st) {
   const TLayout Lo = t_layout();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "encode: shared memory attribute");
+  const int nwords = (int)((p.n + 31) / 32);
+  if (ALG2 && (e = cudaMemsetAsync(p.gflag, 0, (size_t)nwords * 4, st)) != cudaSuccess)
+    return cuda_fail(e, "encode: clear the gamma flags");
   kern<<<grid, kTThreads, Lo.total, st>>>(p, tmap);
+  if (ALG2) {
+    auto fix = gamma_fixup_kernel<F32, BITS>;
+    const int fsm = 2 * p.d * (int)sizeof(double);
+    if (fsm > 48 * 1024 && (e = cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm)) != cudaSuccess)
+      return cuda_fail(e, "encode: gamma fix-up shared memory attribute");
+    fix<<<std::max(1, std::min(nwords, 4 * grid)), 256, fsm, st>>>(p, nwords);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "encode: launch");
   return TQ_OK;
 }
@@ -616,11 +713,17 @@ tq_status launch_tiled_bits(TEParams& p, int bits, const void* x, int grid, cuda
 
 }  // namespace
 
-size_t encode_tiled_ws_bytes(int64_t n, int d, bool alg2, int nsm) {
-  if (!alg2 || d <= 128 || n <= 0) return 0;
+// Algorithm 2 workspace: the residual slots of the tiles in flight (one per CTA), then one flag bit
+// per vector (gamma next to an fp16 rounding midpoint).
+size_t tiled_rho_bytes(int64_t n, int d, int nsm) {
   const int64_t ntiles = (n + 127) / 128;
   const int64_t grid = std::min<int64_t>(ntiles, nsm);
   return (size_t)grid * (size_t)(d / 64) * 2 * kBlk;
+}
+
+size_t encode_tiled_ws_bytes(int64_t n, int d, bool alg2, int nsm) {
+  if (!alg2 || d <= 128 || n <= 0) return 0;
+  return tiled_rho_bytes(n, d, nsm) + (size_t)((n + 31) / 32) * 4;
 }
 
 tq_status encode_tiled(const tq_codebook* cb, int64_t n, int d, const void* x, int xt, const void* rot,
@@ -651,6 +754,7 @@ tq_status encode_tiled(const tq_codebook* cb, int64_t n, int d, const void* x, i
   p.norms = norms;
   p.gammas = gammas;
   p.rho = alg2 ? (uint8_t*)ws : nullptr;
+  p.gflag = alg2 ? (uint32_t*)((uint8_t*)ws + tiled_rho_bytes(n, d, nsm)) : nullptr;
   p.x = x;
   p.pi32 = (const float*)(base + RL.pi32);
   p.t32 = (const float*)(base + RL.t32);

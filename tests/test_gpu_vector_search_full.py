@@ -77,7 +77,7 @@ def test_vector_search_full_size(dev):
     ora2 = Q.residual_signs(ora["u"], gidx, ora["n"], Pi, S, ocb)
     st["signs"] = check_signs(signs_h[sample], ora2["z"], ora2["s"], ora2["gamma"], D)
     check_fp16(norms_h[sample], ora["n"], "norms")
-    check_fp16(gammas_h[sample], ora2["gamma"], "gammas", 2.0 ** -20 * D / 128)
+    check_fp16(gammas_h[sample], ora2["gamma"], "gammas")
     print("sampled encode parity", st)
 
     # top-10 of sampled queries against the oracle's explicit scores over the whole database
