@@ -82,17 +82,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // one second per wait
 
-// Bounded wait for the phase with the given parity. Gives up (returns false) after about one
-// second, or as soon as *abort is non-zero; on its own timeout it records `code` in *err and sets
-// *abort so that the other roles of the block stop waiting too.
+// Bounded wait for the phase with the given parity. Gives up (returns false) after `limit_ns`
+// (about one second unless a caller passes less), or as soon as *abort is non-zero; on its own
+// timeout it records `code` in *err and sets *abort so that the other roles of the block stop
+// waiting too.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
-                                            volatile uint32_t* abort) {
+                                            volatile uint32_t* abort, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1; i < (1u << 30); ++i) {
     if (mbar_try_wait_sleep(bar, phase, 2000u)) return true;
     if ((i & 31u) == 0) {
       if (abort && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (globaltimer_ns() - t0 > limit_ns) break;
     }
   }
   if (err) atomicCAS(err, 0u, code);
@@ -100,15 +101,15 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t phase
   return false;
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
-                                          volatile uint32_t* abort) {
-  return mbar_try_wait(bar, phase) || mbar_wait_slow(bar, phase, err, code, abort);
+                                          volatile uint32_t* abort, uint64_t limit_ns = kWaitLimitNs) {
+  return mbar_try_wait(bar, phase) || mbar_wait_slow(bar, phase, err, code, abort, limit_ns);
 }
 
 // Bounded wait made by every lane of a warp with a warp-uniform result, so a warp that arrives on
 // barriers as a unit also leaves its loop as a unit.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t phase, uint32_t* err, uint32_t code,
-                                               volatile uint32_t* abort) {
-  const bool ok = mbar_wait(bar, phase, err, code, abort);
+                                               volatile uint32_t* abort, uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, phase, err, code, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
