@@ -8,14 +8,16 @@
 // this entry point allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
 //
 // The scratch is one file-scope __device__ array per device (each device that uses the library
-// holds its own copy). Its device address is looked up once per device and cached. The array is
+// holds its own copy). Its device address is looked up on every call, with the caller's device
+// current: a cached address would go stale if the device's context were torn down and created
+// again (the module, and with it the array, may then load elsewhere). The lookup is a host-side
+// table read of the loaded module, cheap next to the launches. The array is
 // shared by every call on that device, so calls whose GPU work overlaps (two streams, two host
 // threads) race on it: callers must order such calls themselves (one stream, or events).
 // Nothing in the array has to start at zero or survive between calls: every byte the attention
 // kernels read from their scratch is written earlier in the same call.
 #include <cuda_runtime.h>
 
-#include <mutex>
 #include <string>
 
 #include "tq_internal.h"
@@ -24,22 +26,14 @@ namespace {
 
 __device__ __align__(256) uint8_t g_attend_scratch[TQ_ATTEND_NOALLOC_MAX_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of this device's scratch array; the current device must be `dev`.
-tq_status scratch_for(int dev, void** out) {
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return tq::cuda_fail(e != cudaSuccess ? (int)e : (int)cudaErrorInvalidSymbol,
-                           "tq_attend_decode_noalloc: scratch address");
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+// Device address of the current device's scratch array.
+tq_status scratch_address(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return tq::cuda_fail(e != cudaSuccess ? (int)e : (int)cudaErrorInvalidSymbol,
+                         "tq_attend_decode_noalloc: scratch address");
+  *out = p;
   return TQ_OK;
 }
 
@@ -60,14 +54,8 @@ extern "C" TQ_API tq_status tq_attend_decode_noalloc(const tq_codebook* cb_k, co
                     "tq_attend_decode_noalloc: these sizes need " + std::to_string(need) +
                         " bytes of scratch, more than the fixed " + std::to_string(TQ_ATTEND_NOALLOC_MAX_BYTES) +
                         "-byte array; call tq_attend_decode with a workspace instead");
-  int dev = 0;
-  const cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return tq::cuda_fail(e, "tq_attend_decode_noalloc: current device");
-  if (dev < 0 || dev >= kMaxDevices)
-    return tq::fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode_noalloc: device ordinal beyond " +
-                                            std::to_string(kMaxDevices - 1));
   void* scratch = nullptr;
-  const tq_status s = scratch_for(dev, &scratch);
+  const tq_status s = scratch_address(&scratch);
   if (s != TQ_OK) return s;
   // sizes too small to be valid (need == 0) are reported by tq_attend_decode's own checks
   return tq_attend_decode(cb_k, cb_v, B, Hq, Hkv, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas,

@@ -84,3 +84,36 @@ def test_noalloc_rejects_oversize():
     assert st == tq.TQ_ERR_WORKSPACE
     msg = L.tq_last_error().decode()
     assert str(need) in msg
+
+
+@pytest.mark.gpu
+def test_noalloc_many_chunks_per_cta(gpu_required):
+    """A size where every CTA walks many chunks (B=2, Hq=32, Hkv=8, T=16384: 2048 chunks over the SMs),
+    noalloc against the workspace entry point, twice in a row."""
+    dev = torch.device("cuda")
+    B, Hkv, T, d = 2, 8, 16384, 128
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    n = B * Hkv * T
+    cbk, cbv = tq.tq_codebook_init(d, 3), tq.tq_codebook_init(d, 1)
+    kc, kn = tq.empty_mse(n, d, 3)
+    vc, vs, vn, vg = tq.empty_prod(n, d, 2)
+    tq.tq_encode_mse(cbk, W.kv_slices_device(B * Hkv, T, d, 3, 20.0, 0.5, 21, dev), rot, kc, kn)
+    tq.tq_encode_prod(cbv, W.kv_slices_device(B * Hkv, T, d, 3, 20.0, 0.5, 22, dev), rot, vc, vs, vn, vg)
+    q = torch.from_numpy(W.queries_bf16((B, 32, d), seed=4)).to(dev).to(torch.bfloat16)
+    c = dict(B=B, Hkv=Hkv, T=T, d=d, rot=rot, cbk=cbk, cbv=cbv, kc=kc, kn=kn.view(B, Hkv, T), vc=vc, vs=vs,
+             vn=vn.view(B, Hkv, T), vg=vg.view(B, Hkv, T), q=q)
+    got1 = _attend(c, tq.tq_attend_decode_noalloc)
+    got2 = _attend(c, tq.tq_attend_decode_noalloc)
+    want = _attend(c, tq.tq_attend_decode)
+    tq.tq_sync_check()
+    for got in (got1, got2):
+        assert torch.isfinite(got).all()
+        assert _rel(got, want) <= TOL
+
+
+def test_noalloc_array_covers_the_decode_attention_workload():
+    """The fixed array is sized for the decode-attention workload (B=16, Hq=32, Hkv=8, T=131072,
+    d=128) with room to spare; a change to the workspace plan that outgrew it would fail here."""
+    need = tq.tq_attend_workspace_bytes(16, 32, 8, 131072, 128)
+    assert 0 < need <= tq.TQ_ATTEND_NOALLOC_MAX_BYTES
