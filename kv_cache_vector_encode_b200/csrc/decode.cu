@@ -47,6 +47,10 @@ struct DecodeParams {
   void* out;
   float alpha;
   uint32_t tab[8];                 // level bytes: [0,1] low / [2,3] high bytes of c_hi, [4,5] / [6,7] of c_lo
+  // mixed widths per channel group (BITS == 0): group g's width, its first word in the record, the
+  // record's words, and the level tables of the codebooks of 1..4 bits
+  int gbits[4], goff[4], wv;
+  uint32_t tabs[4][8];
   uint32_t* err;
 };
 
@@ -77,6 +81,9 @@ enum DBars { A_FULL = 0, B_FULL = 1, B_EMPTY = 3, ACC_FULL = 5, ACC_EMPTY = 7, I
 
 template <bool ALG2, int NV, bool OUT_BF16, int BITS>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr bool MIX = BITS == 0;          // widths per channel group (Algorithm 1 codes)
+  constexpr int BMAX = MIX ? 4 : BITS;
+  static_assert(!(MIX && ALG2), "mixed widths are an Algorithm 1 format");
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;
   constexpr uint32_t NCOLS = 2 * COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -165,17 +172,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     constexpr int UPT = NV * 4 / 128;        // units per thread (gp <= 4)
     // The code words of a tile are fetched one tile ahead, all loads of a tile issued together,
     // so the unpack does not wait on one global load after another.
-    uint32_t cw[UPT][BITS], cs[UPT];
+    uint32_t cw[UPT][BMAX], cs[UPT];
     uint16_t cn = 0, cg = 0;
-    auto fetch = [&](int k, uint32_t (&W)[UPT][BITS], uint32_t (&SGW)[UPT], uint16_t& nn, uint16_t& gg) {
+    auto fetch = [&](int k, uint32_t (&W)[UPT][BMAX], uint32_t (&SGW)[UPT], uint16_t& nn, uint16_t& gg) {
       const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
 #pragma unroll
       for (int j = 0; j < UPT; ++j) {
         const int u = ut + 128 * j, v = u / gp, g = u % gp;
         const bool live = u < units && v < rows && g < G;
+        const int gb = MIX ? p.gbits[g < G ? g : 0] : BITS;
+        const int64_t wbase = MIX ? (v0 + v) * p.wv + p.goff[g < G ? g : 0] : ((v0 + v) * G + g) * BITS;
 #pragma unroll
-        for (int pl = 0; pl < BITS; ++pl) W[j][pl] = live ? __ldg(p.codes + ((v0 + v) * G + g) * BITS + pl) : 0u;
+        for (int pl = 0; pl < BMAX; ++pl) W[j][pl] = (live && pl < gb) ? __ldg(p.codes + wbase + pl) : 0u;
         SGW[j] = (ALG2 && live) ? __ldg(p.signs + (v0 + v) * G + g) : 0u;
       }
       nn = gg = 0;
@@ -189,7 +198,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       const int a = k & 1;
       const int64_t v0 = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * NV;
       const int rows = (int)min((int64_t)NV, p.n - v0);
-      uint32_t nw[UPT][BITS], ns[UPT];
+      uint32_t nw[UPT][BMAX], ns[UPT];
       uint16_t nn = 0, ngm = 0;
       if (k + 1 < my_tiles) fetch(k + 1, nw, ns, nn, ngm);
       if (!mbar_wait_warp(&bar[INFO_EMPTY + a], ((k >> 1) & 1) ^ 1, p.err, kDevTimeoutSync, abort_flag)) break;
@@ -209,22 +218,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         const bool live = v < rows && g < G;
         const uint32_t* w = cw[j];
         const uint32_t sg = cs[j];
+        // this unit's width and level table (a group's own codebook in the mixed format)
+        const int gb = MIX ? p.gbits[g < G ? g : 0] : BITS;
+        if (MIX) {
+#pragma unroll
+          for (int t8 = 0; t8 < 8; ++t8) tab[t8] = p.tabs[gb - 1][t8];
+        }
         // selector planes: the index bits (up to 3), or for 16 levels the magnitude bits
         // (low bits ^ ~top bit) with the sign taken from the top bit
-        constexpr int SB = BITS < 4 ? BITS : 3;
-        const uint32_t flip = BITS == 4 ? ~w[BITS == 4 ? 3 : 0] : 0u;
+        const int SB = gb < 4 ? gb : 3;
+        const uint32_t flip = gb == 4 ? ~w[BMAX == 4 ? 3 : 0] : 0u;
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) {
           uint32_t x = 0;
 #pragma unroll
-          for (int pl = 0; pl < SB; ++pl) x |= (((w[pl] ^ flip) >> s4) & 0x11111111u) << pl;
-          const uint32_t fl = BITS == 4 ? (flip >> s4) & 0x11111111u : 0u;
+          for (int pl = 0; pl < (BMAX < 4 ? BMAX : 3); ++pl)
+            if (pl < SB) x |= (((w[pl] ^ flip) >> s4) & 0x11111111u) << pl;
+          const uint32_t fl = gb == 4 ? (flip >> s4) & 0x11111111u : 0u;
           uint32_t o_hi[4], o_lo[4], o_s[4];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const uint32_t sel = half ? x >> 16 : x;
             uint32_t hb = __byte_perm(tab[2], tab[3], sel), hl = __byte_perm(tab[6], tab[7], sel);
-            if (BITS == 4) {
+            if (gb == 4) {
               const uint32_t sb = __byte_perm(0x8000u, 0u, half ? fl >> 16 : fl);   // 0x80 where negative
               hb ^= sb;
               hl ^= sb;
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < UPT; ++j) {
 #pragma unroll
-        for (int pl = 0; pl < BITS; ++pl) cw[j][pl] = nw[j][pl];
+        for (int pl = 0; pl < BMAX; ++pl) cw[j][pl] = nw[j][pl];
         cs[j] = ns[j];
       }
       cn = nn;
@@ -333,6 +349,28 @@ tq_status launch_decode(DecodeParams& p, cudaStream_t st) {
   return TQ_OK;
 }
 
+// Byte tables of the fp16 hi / lo parts of a codebook's levels for the byte-permute lookup: up to
+// eight levels are looked up directly; sixteen by magnitude (the positive half c[8 + m]).
+void level_tables(const tq_codebook* cb, uint32_t (&tab)[8]) {
+  const int L = cb->levels;
+  const int base_level = L > 8 ? L / 2 : 0, nt = L > 8 ? 8 : L;
+  uint8_t hl[4][8] = {};                       // [low c_hi, high c_hi, low c_lo, high c_lo][entry]
+  for (int m = 0; m < nt; ++m) {
+    const float c = cb->c[base_level + m];
+    const __half h = __float2half_rn(c);
+    const __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
+    const uint16_t hu = __half_as_ushort(h), lu = __half_as_ushort(l);
+    hl[0][m] = (uint8_t)(hu & 0xFF);
+    hl[1][m] = (uint8_t)(hu >> 8);
+    hl[2][m] = (uint8_t)(lu & 0xFF);
+    hl[3][m] = (uint8_t)(lu >> 8);
+  }
+  for (int t = 0; t < 4; ++t)
+    for (int w = 0; w < 2; ++w)
+      tab[2 * t + w] = (uint32_t)hl[t][4 * w] | (uint32_t)hl[t][4 * w + 1] << 8 | (uint32_t)hl[t][4 * w + 2] << 16 |
+                       (uint32_t)hl[t][4 * w + 3] << 24;
+}
+
 template <bool ALG2, int NV, bool BF16>
 tq_status decode_bits(DecodeParams& p, int bits, cudaStream_t st) {
   switch (bits) {
@@ -386,27 +424,63 @@ extern "C" TQ_API tq_status tq_decode(const tq_codebook* cb, int64_t n, int32_t 
   const int L = cb->levels;
   for (int k = 0; k < L; ++k)
     if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, "tq_decode: codebook is not symmetric");
-  // up to eight levels are looked up directly; sixteen by magnitude (the positive half c[8 + m])
-  const int base_level = L > 8 ? L / 2 : 0, nt = L > 8 ? 8 : L;
-  uint8_t hl[4][8] = {};                       // [low c_hi, high c_hi, low c_lo, high c_lo][entry]
-  for (int m = 0; m < nt; ++m) {
-    const float c = cb->c[base_level + m];
-    const __half h = __float2half_rn(c);
-    const __half l = __float2half_rn((c - __half2float(h)) * kSplitScale);
-    const uint16_t hu = __half_as_ushort(h), lu = __half_as_ushort(l);
-    hl[0][m] = (uint8_t)(hu & 0xFF);
-    hl[1][m] = (uint8_t)(hu >> 8);
-    hl[2][m] = (uint8_t)(lu & 0xFF);
-    hl[3][m] = (uint8_t)(lu >> 8);
-  }
-  for (int t = 0; t < 4; ++t)
-    for (int w = 0; w < 2; ++w)
-      p.tab[2 * t + w] = (uint32_t)hl[t][4 * w] | (uint32_t)hl[t][4 * w + 1] << 8 | (uint32_t)hl[t][4 * w + 2] << 16 |
-                         (uint32_t)hl[t][4 * w + 3] << 24;
+  level_tables(cb, p.tab);
   p.err = device_error_word();
   if (!p.err) return fail(TQ_ERR_CUDA, "tq_decode: no device error word (is a CUDA device present?)");
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf = out_dtype == TQ_BF16;
   if (signs) return bf ? decode_bits<true, 64, true>(p, cb->bits, st) : decode_bits<true, 64, false>(p, cb->bits, st);
   return bf ? decode_bits<false, 128, true>(p, cb->bits, st) : decode_bits<false, 128, false>(p, cb->bits, st);
+}
+
+// Decode of the mixed-width format of tq_encode_mse_mixed (d <= 128): each unpacking thread expands
+// its (vector, group) unit with the group's own codebook.
+extern "C" TQ_API tq_status tq_decode_mixed(const tq_codebook* cbs, const int32_t* group_bits, int64_t n, int32_t d,
+                                            const void* rot, const uint32_t* codes, const uint16_t* norms, void* out,
+                                            int32_t out_dtype, void* stream) {
+  clear_error();
+  const char* f = "tq_decode_mixed";
+  if (!cbs || !group_bits || !rot || !codes || !norms || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode_mixed: NULL pointer");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, "tq_decode_mixed: n < 0");
+  if (!valid_dim(d) || d > 128) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_mixed: d must be 32, 64, 96 or 128");
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_mixed: out_dtype");
+  DecodeParams p{};
+  const int G = d / 32;
+  int wv = 0;
+  for (int g = 0; g < G; ++g) {
+    const int b = group_bits[g];
+    if (b < 1 || b > 4) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_mixed: group widths must be 1..4 bits");
+    const tq_codebook* cb = &cbs[b - 1];
+    if (cb->d != d || cb->bits != b || cb->levels != (1 << b))
+      return fail(TQ_ERR_INVALID_ARG, "tq_decode_mixed: cbs[b - 1] must be the b-bit codebook for this d");
+    const int L = cb->levels;
+    for (int k = 0; k < L; ++k)
+      if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, "tq_decode_mixed: codebook is not symmetric");
+    p.gbits[g] = b;
+    p.goff[g] = wv;
+    wv += b;
+    level_tables(cb, p.tabs[b - 1]);
+  }
+  p.wv = wv;
+  if (!aligned16(rot) || !aligned16(codes) || !aligned16(norms) || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "tq_decode_mixed: pointers must be 16-byte aligned");
+  if (n == 0) return TQ_OK;
+  RotLayout RL = rot_layout(d);
+  const uint8_t* base = (const uint8_t*)rot;
+  p.n = n;
+  p.d = d;
+  p.G = G;
+  p.KP = d <= 64 ? 64 : 128;
+  p.img[0] = base + RL.pit_hi;
+  p.img[1] = base + RL.pit_lo;
+  p.img[2] = base + RL.st_hi;
+  p.img[3] = base + RL.st_lo;
+  p.img_bytes = 128u * p.KP * 2;
+  p.codes = codes;
+  p.norms = norms;
+  p.out = out;
+  p.err = device_error_word();
+  if (!p.err) return fail(TQ_ERR_CUDA, std::string(f) + ": no device error word");
+  cudaStream_t st = (cudaStream_t)stream;
+  return out_dtype == TQ_BF16 ? launch_decode<false, 128, true, 0>(p, st) : launch_decode<false, 128, false, 0>(p, st);
 }

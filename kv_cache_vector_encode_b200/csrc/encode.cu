@@ -61,6 +61,10 @@ struct EncodeParams {
   uint16_t* gammas;
   float P[8];                // positive boundaries t_{L/2} .. t_{L-2}
   float C[8];                // positive centroids c_{L/2} .. c_{L-1}
+  // mixed widths per channel group (BITS == 0): group g's width, its first word in the record,
+  // the record's words, and the group's positive boundaries
+  int gbits[4], goff[4], wv;
+  float Pm[4][8];
   uint32_t* err;
 };
 
@@ -125,13 +129,16 @@ template <int XT, bool ALG2, int NV, int BITS>
 __global__ void __launch_bounds__(enc_threads(ALG2), 1)
     encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmap) {
   constexpr bool F32 = XT == TQ_F32;
+  constexpr bool MIX = BITS == 0;                          // widths per channel group (Algorithm 1)
+  constexpr int BMAX = MIX ? 4 : BITS;                     // planes of the widest group
+  static_assert(!(MIX && ALG2), "mixed widths are an Algorithm 1 format");
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;       // TMEM columns per accumulator buffer
   constexpr uint32_t NCOLS = 2 * COLS;
   constexpr int TPV = 128 / NV;                            // converter threads per vector
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int d = p.d, KP = p.KP, G = p.G;
-  const EncLayout Lo = enc_layout<XT, ALG2, NV, BITS>(d, KP, G);
+  const EncLayout Lo = enc_layout<XT, ALG2, NV, BMAX>(d, KP, G);
   uint64_t* bar = (uint64_t*)(smem + Lo.off_bar);
   uint32_t* tmem_slot = (uint32_t*)(bar + NBARS);
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + NBARS) + 1;
@@ -362,9 +369,13 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
     const int cbeg = (e >> 2) * (NV / 2), cend = cbeg + NV / 2;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     float P[8], C[8];
+    const int gq = q < G ? q : 0;
+    const int gbw = MIX ? p.gbits[gq] : BITS;   // this warp's group width (warp-uniform)
+    const int wrec = MIX ? p.wv : G * BITS;     // words of a vector's codes
+    const int woff = MIX ? p.goff[gq] : q * BITS;
 #pragma unroll
     for (int kq = 0; kq < 8; ++kq) {
-      P[kq] = p.P[kq];
+      P[kq] = MIX ? p.Pm[gq][kq] : p.P[kq];
       C[kq] = p.C[kq];
     }
     uint32_t epi_uses = 0;
@@ -389,9 +400,9 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
         tmem_ld16(dhi + c0, hi);
         tmem_ld16(dlo + c0, lo);
         tmem_ld_wait();
-        uint32_t myw[BITS];
+        uint32_t myw[BMAX];
 #pragma unroll
-        for (int pl = 0; pl < BITS; ++pl) myw[pl] = 0u;
+        for (int pl = 0; pl < BMAX; ++pl) myw[pl] = 0u;
         float r2[16];                       // rho * 2^14 of the 16 vectors (Algorithm 2)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -399,15 +410,16 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
           const float inv = info[a * NV + v];
           const float y = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j])) * inv;
           const bool neg = !(y > 0.0f);
-          const int m = sym_m<BITS>(fabsf(y), P);
+          const int m = MIX ? sym_m_rt(fabsf(y), P, gbw) : sym_m<BMAX>(fabsf(y), P);
 #pragma unroll
-          for (int pl = 0; pl < BITS; ++pl) {
-            const bool bit = pl == BITS - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
+          for (int pl = 0; pl < BMAX; ++pl) {
+            if (MIX && pl >= gbw) break;            // warp-uniform
+            const bool bit = pl == gbw - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
             const uint32_t w = __ballot_sync(0xffffffffu, active && bit);
             if (lane == j) myw[pl] = w;
           }
           if (ALG2) {
-            const float cm = sym_c<BITS>(m, C);
+            const float cm = sym_c<BMAX>(m, C);
             float rho = neg ? y + cm : y - cm;
             if (!active || inv == 0.0f) rho = 0.0f;
             if (NV == 64) {
@@ -452,7 +464,8 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
         }
         if (q < G && lane < 16) {
 #pragma unroll
-          for (int pl = 0; pl < BITS; ++pl) codes_stage[((c0 + lane) * G + q) * BITS + pl] = myw[pl];
+          for (int pl = 0; pl < BMAX; ++pl)
+            if (!MIX || pl < gbw) codes_stage[(c0 + lane) * wrec + woff + pl] = myw[pl];
         }
         if (ALG2) {
           const float tot = transpose_reduce16(r2, lane);
@@ -466,8 +479,8 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
       }
       if (!epi_sync()) break;
       {
-        uint32_t* dst = p.codes + v0 * G * BITS;
-        const int nw = rows * G * BITS;
+        uint32_t* dst = p.codes + v0 * wrec;
+        const int nw = rows * wrec;
         for (int w = te; w < nw; w += 256) dst[w] = codes_stage[w];
       }
       if (ALG2) {
@@ -519,7 +532,7 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
 template <int XT, bool ALG2, int NV, int BITS>
 tq_status launch_encode(EncodeParams& p, const void* x, cudaStream_t st) {
   constexpr int ES = XT == TQ_BF16 ? 2 : 4;
-  const EncLayout Lo = enc_layout<XT, ALG2, NV, BITS>(p.d, p.KP, p.G);
+  const EncLayout Lo = enc_layout<XT, ALG2, NV, BITS == 0 ? 4 : BITS>(p.d, p.KP, p.G);
   alignas(64) CUtensorMap tmap;
   if (!make_tmap_2d_sw128(&tmap, x, ES, (uint64_t)p.d, (uint64_t)p.n, 128 / ES, NV))
     return fail(TQ_ERR_CUDA, "encode: could not create the TMA tensor map of x");
@@ -623,4 +636,57 @@ extern "C" TQ_API tq_status tq_encode_prod(const tq_codebook* cb_bm1, int64_t n,
                                     uint16_t* gammas, void* ws, size_t ws_bytes, void* stream) {
   return encode_common("tq_encode_prod", cb_bm1, n, d, x, x_dtype, rot, codes, signs, norms, gammas, true, ws, ws_bytes,
                        stream);
+}
+
+// Algorithm 1 with a bit width per group of 32 rotated coordinates (d <= 128): each epilogue warp
+// quantises one group with that group's codebook and writes its planes at the group's offset in the
+// record.
+extern "C" TQ_API tq_status tq_encode_mse_mixed(const tq_codebook* cbs, const int32_t* group_bits, int64_t n,
+                                                int32_t d, const void* x, int32_t x_dtype, const void* rot,
+                                                uint32_t* codes, uint16_t* norms, void* stream) {
+  clear_error();
+  const std::string f = "tq_encode_mse_mixed";
+  if (!cbs || !group_bits || !rot || !codes || !norms || (n > 0 && !x)) return fail(TQ_ERR_INVALID_ARG, f + ": NULL pointer");
+  if (n < 0) return fail(TQ_ERR_INVALID_ARG, f + ": n < 0");
+  if (!valid_dim(d) || d > 128) return fail(TQ_ERR_UNSUPPORTED, f + ": d must be 32, 64, 96 or 128");
+  const int G = d / 32;
+  EncodeParams p{};
+  int wv = 0;
+  for (int g = 0; g < G; ++g) {
+    const int b = group_bits[g];
+    if (b < 1 || b > 4) return fail(TQ_ERR_UNSUPPORTED, f + ": group widths must be 1..4 bits");
+    const tq_codebook* cb = &cbs[b - 1];
+    if (cb->d != d || cb->bits != b || cb->levels != (1 << b))
+      return fail(TQ_ERR_INVALID_ARG, f + ": cbs[b - 1] must be the b-bit codebook for this d");
+    const int L = cb->levels, H = L / 2;
+    for (int k = 0; k < L; ++k)
+      if (cb->c[L - 1 - k] != -cb->c[k]) return fail(TQ_ERR_INVALID_ARG, f + ": codebook is not symmetric");
+    p.gbits[g] = b;
+    p.goff[g] = wv;
+    wv += b;
+    for (int k = 0; k < 8; ++k) p.Pm[g][k] = k < H - 1 ? cb->t[H + k] : 0.0f;
+  }
+  p.wv = wv;
+  if (x_dtype != TQ_F32 && x_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, f + ": x_dtype must be TQ_F32 or TQ_BF16");
+  if (!aligned16(x) || !aligned16(rot) || !aligned16(codes) || !aligned16(norms))
+    return fail(TQ_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
+  if (n == 0) return TQ_OK;
+  if (n > ((int64_t)1 << 31) - 256) return fail(TQ_ERR_UNSUPPORTED, f + ": n >= 2^31");
+  RotLayout RL = rot_layout(d);
+  const uint8_t* base = (const uint8_t*)rot;
+  p.n = n;
+  p.d = d;
+  p.G = G;
+  p.KP = d <= 64 ? 64 : 128;
+  p.img[0] = base + RL.pi_hi;
+  p.img[1] = base + RL.pi_lo;
+  p.img[2] = base + RL.t_hi;
+  p.img[3] = base + RL.t_lo;
+  p.img_bytes = 128u * p.KP * 2;
+  p.codes = codes;
+  p.norms = norms;
+  p.err = device_error_word();
+  if (!p.err) return fail(TQ_ERR_CUDA, f + ": no device error word (is a CUDA device present?)");
+  cudaStream_t st = (cudaStream_t)stream;
+  return x_dtype == TQ_BF16 ? launch_encode<TQ_BF16, false, 128, 0>(p, x, st) : launch_encode<TQ_F32, false, 64, 0>(p, x, st);
 }

@@ -25,6 +25,16 @@ __device__ __forceinline__ int sym_m(float a, const float (&P)[8]) {
   return 4 * m2 + 2 * m1 + m0;
 }
 
+// sym_m for a width known only at run time (warp-uniform where it is used)
+__device__ __forceinline__ int sym_m_rt(float a, const float (&P)[8], int bits) {
+  switch (bits) {
+    case 1: return sym_m<1>(a, P);
+    case 2: return sym_m<2>(a, P);
+    case 3: return sym_m<3>(a, P);
+    default: return sym_m<4>(a, P);
+  }
+}
+
 template <int BITS>
 __device__ __forceinline__ float sym_c(int m, const float (&C)[8]) {
   if (BITS == 1) return C[0];

@@ -160,6 +160,50 @@ def encode_prod(x: np.ndarray, Pi: np.ndarray, S: np.ndarray, cb_bm1: Codebook) 
     return e
 
 
+# ---- mixed widths per channel group ----------------------------------------------------------
+# Reading (the scope table's "mixed / fractional bit widths per channel group"; the pages' only
+# fractional figure, techblog-plum's "average 2.5 bit", is keys at 3 bits and values at 2): the d
+# rotated coordinates form d/32 groups of 32 (the packing groups), and group g is quantised with
+# the b_g-bit Lloyd-Max codebook of the same coordinate law f_d (after the rotation every coordinate
+# has that law, so each group's own codebook is optimal for it). The record holds, group by group,
+# that group's b_g bit-plane words, then the fp16 norm: 4 sum_g b_g + 2 bytes. Algorithm 1 only.
+
+def pack_mixed(idx: np.ndarray, group_bits) -> np.ndarray:
+    """idx [N, d] -> uint32 [N, sum(group_bits)]: group g's planes (pack_planes of its 32 columns)."""
+    idx = np.asarray(idx, dtype=np.int64)
+    parts = [pack_planes(idx[:, 32 * g:32 * g + 32], b).reshape(idx.shape[0], b) for g, b in enumerate(group_bits)]
+    return np.concatenate(parts, axis=1)
+
+
+def unpack_mixed(words: np.ndarray, group_bits) -> np.ndarray:
+    """uint32 [N, sum(group_bits)] -> idx [N, 32 len(group_bits)]."""
+    w = np.asarray(words, dtype=np.uint32)
+    out, o = [], 0
+    for b in group_bits:
+        out.append(unpack_planes(w[:, o:o + b].reshape(w.shape[0], 1, b), b))
+        o += b
+    return np.concatenate(out, axis=1)
+
+
+def encode_mse_mixed(x: np.ndarray, Pi: np.ndarray, cbs: dict, group_bits) -> dict:
+    """Algorithm 1 with a bit width per group of 32 rotated coordinates (cbs: bits -> codebook)."""
+    n, n16, u = normalise(x)
+    y = rotate(u, Pi)
+    idx = np.empty(y.shape, dtype=np.int64)
+    for g, b in enumerate(group_bits):
+        idx[:, 32 * g:32 * g + 32] = quantise(y[:, 32 * g:32 * g + 32], cbs[b])
+    return dict(codes=pack_mixed(idx, group_bits), norms=n16, n=n, u=u, y=y, idx=idx)
+
+
+def decode_mixed(codes: np.ndarray, norms16: np.ndarray, Pi: np.ndarray, cbs: dict, group_bits) -> np.ndarray:
+    """x_hat = n Pi^T c_g[idx] with each group's own codebook."""
+    idx = unpack_mixed(codes, group_bits)
+    chat = np.empty(idx.shape, dtype=np.float64)
+    for g, b in enumerate(group_bits):
+        chat[:, 32 * g:32 * g + 32] = cbs[b].c32.astype(np.float64)[idx[:, 32 * g:32 * g + 32]]
+    return np.asarray(norms16, dtype=np.float64)[:, None] * (chat @ np.asarray(Pi, dtype=np.float64))
+
+
 # ---- decode -----------------------------------------------------------------------------------
 
 def decode(codes: np.ndarray, norms16: np.ndarray, Pi: np.ndarray, cb: Codebook,

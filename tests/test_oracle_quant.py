@@ -271,3 +271,59 @@ def test_planted_alpha_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(Q, "qjl_alpha", lambda d: math.sqrt(2 / math.pi) / d)
     mean, se = _qjl_bias(Q.qjl_alpha)
     assert abs(mean) > 8 * se
+
+
+# ---- mixed widths per channel group ------------------------------------------------------------
+
+def test_mixed_uniform_map_is_algorithm_1():
+    """A map with one width everywhere is plain Algorithm 1: the same words, the same decode."""
+    d = 128
+    Pi = W.rotation(d)
+    x = W.gaussian(300, d, seed=5)
+    for b in (1, 2, 3, 4):
+        cb = lloyd_max(d, b)
+        e = Q.encode_mse(x, Pi, cb)
+        m = Q.encode_mse_mixed(x, Pi, {b: cb}, [b] * (d // 32))
+        assert np.array_equal(m["codes"], e["codes"].reshape(len(x), -1))
+        assert np.array_equal(Q.decode_mixed(m["codes"], m["norms"], Pi, {b: cb}, [b] * (d // 32)),
+                              Q.decode(e["codes"], e["norms"], Pi, cb))
+
+
+def test_mixed_packing_bit_by_bit():
+    """Brute force at d = 64 with widths (1, 4) and (4, 2): every index value at every coordinate
+    round-trips, and an independent reader finds bit p of idx[32 g + l] at bit l of word
+    sum_{g' < g} b_g' + p."""
+    g = np.random.default_rng(8)
+    for gb in ([1, 4], [4, 2], [3, 3]):
+        idx = np.concatenate([g.integers(0, 1 << b, size=(40, 32)) for b in gb], axis=1)
+        words = Q.pack_mixed(idx, gb)
+        assert words.shape == (40, sum(gb))
+        assert np.array_equal(Q.unpack_mixed(words, gb), idx)
+        off = np.concatenate([[0], np.cumsum(gb)[:-1]])
+        for v in range(0, 40, 7):
+            for j in range(64):
+                gg, lane = divmod(j, 32)
+                for p in range(gb[gg]):
+                    assert (int(words[v, off[gg] + p]) >> lane) & 1 == (int(idx[v, j]) >> p) & 1
+
+
+@pytest.mark.parametrize("gb", [[3, 3, 2, 2], [4, 2, 2, 2], [1, 2, 3, 4]])
+def test_mixed_distortion_is_the_group_average(gb):
+    """After the rotation every coordinate has the law f_d, so the per-vector distortion of a mixed
+    map is the group-weighted average sum_g (32/d) D_{b_g} of the uniform distortions; the empirical
+    MSE on 4096 vectors matches it within 3 standard errors. A (3,3,2,2) map is a 2.5-bit code
+    between the 2- and 3-bit ones."""
+    d = 128
+    x = W.gaussian(4096, d)
+    Pi = W.rotation(d)
+    cbs = {b: lloyd_max(d, b) for b in set(gb)}
+    m = Q.encode_mse_mixed(x, Pi, cbs, gb)
+    uh = Q.decode_mixed(m["codes"], np.ones(len(x), dtype=np.float16), Pi, cbs, gb)
+    err = np.sum((m["u"] - uh) ** 2, axis=1)
+    D = sum(32.0 / d * distortion_per_vector(cbs[b]) for b in gb)
+    se = err.std(ddof=1) / math.sqrt(len(err))
+    assert abs(err.mean() - D) < 3 * se + 1e-4 * D, (err.mean(), D, se)
+    lo, hi = min(gb), max(gb)
+    assert distortion_per_vector(lloyd_max(d, hi)) <= D <= distortion_per_vector(lloyd_max(d, lo))
+    # record size: the planes of every group plus the fp16 norm
+    assert m["codes"].shape[1] * 4 + 2 == 4 * sum(gb) + 2
