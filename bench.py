@@ -58,59 +58,106 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense fp16 / bf16 tensor peak (TFLOP/s): the measured burst figure, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and throttle-reason samples while the timed region runs: NVML polled every 2 ms from
+    a thread (so a timed region of tens of milliseconds still gets many samples), else nvidia-smi
+    every 20 ms. Reads settings only."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.index = index
+        self.period = period_s
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.stop = threading.Event()
+        self.samples = []          # (sm_mhz, max_mhz, set of reason names)
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll_nvml(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((sm, mx, {k for k, v in bits.items() if r & v}))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _read_smi(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            self.samples.append((sm, mx, {nm for nm, v in zip(self.NAMES, parts[2:6]) if v.lower().startswith("active")}))
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml, every 2 ms"
         except Exception:
-            self.proc = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "20"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._read_smi, daemon=True)
+                self.source = "nvidia-smi, every 20 ms"
+            except Exception:
+                self.thread = None
+        if self.thread is not None:
+            self.thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 6:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[2:6]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [x[0] for x in self.samples]
+        reasons = set().union(*[x[2] for x in self.samples])
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "sm_mhz_min": min(sm), "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -176,11 +223,75 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded Gaussian, outlier channels, log-normal norms)",
         "config": workload_config(),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                         "other_workloads": oracle_per_workload()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def oracle_per_workload():
+    """The oracle on bounded samples of each workload (host cores; vectors or pairs per second)."""
+    import numpy as np
+    import workloads as W
+    from oracle import attention as OA
+    from oracle import quant as Q
+    from oracle.codebook import lloyd_max
+    res = {}
+
+    def clock(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    # tiny: 4096 x 128 fp32, Algorithm 1 encode + decode at b = 1..4 (the whole set)
+    d = 128
+    Pi = W.rotation(d)
+    x = W.gaussian(4096, d)
+    cbs = {b: lloyd_max(d, b) for b in (1, 2, 3, 4)}
+
+    def tiny():
+        for b, cb in cbs.items():
+            e = Q.encode_mse(x, Pi, cb)
+            Q.decode(e["codes"], e["norms"], Pi, cb)
+    el = clock(tiny)
+    res["tiny_4096x128_f32"] = {"vectors_per_s": 4 * 2 * 4096 / el, "sample": "whole set, b = 1..4", "s": el}
+    # TinyLlama-shaped block at d = 64: a 4096-token head of K (Algorithm 1 b=3) and of V (Algorithm 2 b=2)
+    d = 64
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    K = W.kv_slice(4096, d, 4, 20.0, 0.0, 0, W.TAG_K, 0, 0)
+    V = W.kv_slice(4096, d, 4, 20.0, 0.0, 0, W.TAG_V, 0, 0)
+    cbk, cbv = lloyd_max(d, 3), lloyd_max(d, 1)
+
+    def tl():
+        ek = Q.encode_mse(K, Pi, cbk)
+        ev = Q.encode_prod(V, Pi, S, cbv)
+        Q.decode(ek["codes"], ek["norms"], Pi, cbk)
+        Q.decode(ev["codes"], ev["norms"], Pi, cbv, ev["signs"], ev["gammas"], S)
+    el = clock(tl)
+    res["tinyllama_block_32x4096x64"] = {"vectors_per_s": 4 * 4096 / el,
+                                         "sample": "one head: 4096 K and 4096 V encoded and decoded", "s": el}
+    # vector search at d = 1536: 2048 database vectors encoded (Algorithm 2 b=4), 64 queries scored
+    d = 1536
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    X = W.unit_rows(2048, d)
+    qs = W.unit_rows(64, d, tag=W.TAG_Q)
+    cb3 = lloyd_max(d, 3)
+    st = {}
+
+    def enc():
+        st["e"] = Q.encode_prod(X, Pi, S, cb3)
+    el_e = clock(enc)
+
+    def scan():
+        e = st["e"]
+        xh = Q.decode(e["codes"], e["norms"], Pi, cb3, e["signs"], e["gammas"], S)
+        OA.topk(OA.scores(qs, xh), 10)
+    el_s = clock(scan)
+    res["vector_search_1e6x1536"] = {"encode_vectors_per_s": 2048 / el_e, "score_pairs_per_s": 64 * 2048 / el_s,
+                                     "sample": "2048 database vectors, 64 queries", "s": el_e + el_s}
+    return res
 
 
 def cpu_baseline_measure(seconds_cap=20.0):
@@ -209,7 +320,9 @@ def cpu_baseline_measure(seconds_cap=20.0):
         if time.perf_counter() - t0 > seconds_cap or k >= 10:
             break
     el = time.perf_counter() - t0
+    per = oracle_per_workload()
     return {"value": units / el, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "other_workloads": per,
             "sample": f"{k} oracle steps of: encode+decode {n} K and {n} V vectors, attention over one "
                       f"{t}-token KV-head slice (4 query heads); {el:.1f} s"}
 
@@ -304,7 +417,8 @@ def run_ours(args):
     tq.tq_sync_check()
 
     def step(ev=None, bufs=None):
-        Kx, Vx, qx, (ckc, ckn, cvc, cvs, cvn, cvg, cout) = bufs or (Kb, Vb, q, (bkc, bkn, bvc, bvs, bvn, bvg, att_out))
+        Kx, Vx, qx, (ckc, ckn, cvc, cvs, cvn, cvg, cout, cok, cov) = bufs or (
+            Kb, Vb, q, (bkc, bkn, bvc, bvs, bvn, bvg, att_out, outk, outv))
         if ev is not None:
             ev[0].record(stream)
         tq.tq_encode_mse(cbk, Kx, rot, ckc, ckn)
@@ -313,10 +427,10 @@ def run_ours(args):
         tq.tq_encode_prod(cbv, Vx, rot, cvc, cvs, cvn, cvg)
         if ev is not None:
             ev[2].record(stream)
-        tq.tq_decode(cbk, rot, ckc, ckn, outk)
+        tq.tq_decode(cbk, rot, ckc, ckn, cok)
         if ev is not None:
             ev[3].record(stream)
-        tq.tq_decode(cbv, rot, cvc, cvn, outv, signs=cvs, gammas=cvg)
+        tq.tq_decode(cbv, rot, cvc, cvn, cov, signs=cvs, gammas=cvg)
         if ev is not None:
             ev[4].record(stream)
         tq.tq_attend_decode(cbk, cbv2, qx, rot, kc, kn3, vc, vn3, cout, v_signs=vs, v_gammas=vg3, ws=ws)
@@ -349,20 +463,21 @@ def run_ours(args):
     value = world * vectors_per_step() / (ms_step * 1e-3)
 
     # end-to-end through the public API with host buffers: inputs from pinned memory each step,
-    # results (packed block + attention output) read back
+    # every result of the step read back (packed block, both decoded blocks, attention output)
     Kh = Kb.cpu().pin_memory()
     Vh = Vb.cpu().pin_memory()
     qh = q.cpu().pin_memory()
-    res = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (bkc, bkn, bvc, bvs, bvn, bvg, att_out)]
+    outs = (bkc, bkn, bvc, bvs, bvn, bvg, att_out, outk, outv)
+    res = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     h2d = Kh.numel() * 2 + Vh.numel() * 2 + qh.numel() * 2
     d2h = sum(r.numel() * r.element_size() for r in res)
 
     # Two buffer sets: the inputs of step k+1 are copied in (one copy stream) while step k computes,
     # and the results of step k are copied out (a second copy stream) while step k+1 computes.
     # Every step's copies lie inside the timed region, which ends when the last results are home.
-    sets = [(Kb, Vb, q, (bkc, bkn, bvc, bvs, bvn, bvg, att_out))]
+    sets = [(Kb, Vb, q, outs)]
     sets.append((torch.empty_like(Kb), torch.empty_like(Vb), torch.empty_like(q),
-                 tuple(torch.empty_like(t) for t in (bkc, bkn, bvc, bvs, bvn, bvg, att_out))))
+                 tuple(torch.empty_like(t) for t in outs)))
     h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_run(n, start=None, end=None):
@@ -434,6 +549,11 @@ def run_ours(args):
     step_bytes = sum(comp_bytes.values())
     breakdown["step_frac_hbm"] = round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4)
 
+    extra = None
+    if rank == 0 and not args.no_extra:
+        extra = extra_workloads(dev, peak, tensor_peak()[0])
+    if world > 1:
+        dist.barrier()
     if rank == 0:
         cpu = cpu_baseline_measure() if (world == 1 and not args.no_cpu_baseline) else None
         line = {
@@ -447,6 +567,7 @@ def run_ours(args):
                          "frac": round(att_gbs / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": att_bytes},
             "breakdown": breakdown,
+            "other_workloads": extra,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * 7,
@@ -459,6 +580,199 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _timed(fn, iters, warmup=2):
+    """Mean device time (ms) of fn() over `iters` calls on the current stream (CUDA events)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def _graph_timed(fn, reps, iters=20):
+    """Mean device time (ms) of fn() when `reps` calls are captured in one CUDA graph and the graph is
+    replayed `iters` times (removes host launch overhead for the small workloads); None if the calls
+    cannot be captured."""
+    import torch
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / (iters * reps)
+        del g
+        return ms
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+
+
+def extra_workloads(dev, peak_hbm, peak_tensor):
+    """The other workloads measured beside the step (each call timed alone with CUDA events; not part
+    of the step's value): the tiny correctness set (4096 x 128 fp32, Algorithm 1 at b = 1..4), the
+    TinyLlama-shaped block (K, V bf16 [32 x 4096 x 64], K Algorithm 1 b=3, V Algorithm 2 b=2) and
+    the vector-search scan (1e6 x 1536 fp32 unit rows, Algorithm 2 b=4, 1024 queries, top-10)."""
+    import torch
+    import kv_cache_vector_encode_b200 as tq
+    import workloads as W
+    out = {}
+    # -- tiny: 4096 x 128 fp32, Algorithm 1 encode + decode at b = 1..4 (launch-bound)
+    d, n = 128, 4096
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    x = torch.randn((n, d), generator=torch.Generator(device=dev).manual_seed(0), device=dev)
+    xd = torch.empty((n, d), dtype=torch.float32, device=dev)
+    tiny = {}
+    for b in (1, 2, 3, 4):
+        cb = tq.tq_codebook_init(d, b)
+        c, nn = tq.empty_mse(n, d, b, dev)
+        enc = lambda: tq.tq_encode_mse(cb, x, rot, c, nn)
+        dec = lambda: tq.tq_decode(cb, rot, c, nn, xd)
+        both = lambda: (enc(), dec())
+        ms = _timed(both, 50)
+        msg = _graph_timed(both, 50)
+        tiny[f"b{b}"] = {"encode_decode_ms": round(ms, 5), "vectors_per_s": 2 * n / (ms * 1e-3),
+                         "graph_ms": None if msg is None else round(msg, 5),
+                         "graph_vectors_per_s": None if msg is None else 2 * n / (msg * 1e-3)}
+    out["tiny_4096x128_f32"] = tiny
+    # -- TinyLlama-shaped block: K, V bf16 [32 x 4096 x 64]
+    d, heads, tokens = 64, 32, 4096
+    n = heads * tokens
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rot64 = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    K = W.kv_slices_device(heads, tokens, d, 4, 20.0, 0.0, 31, dev)
+    V = W.kv_slices_device(heads, tokens, d, 4, 20.0, 0.0, 32, dev)
+    cbk, cbv = tq.tq_codebook_init(d, 3), tq.tq_codebook_init(d, 1)
+    kc, kn = tq.empty_mse(n, d, 3, dev)
+    vc, vs, vn, vg = tq.empty_prod(n, d, 2, dev)
+    kd = torch.empty((n, d), dtype=torch.float32, device=dev)
+    vd = torch.empty((n, d), dtype=torch.float32, device=dev)
+    calls = {"encode_k": (lambda: tq.tq_encode_mse(cbk, K, rot64, kc, kn), 2 * d + 3 * d // 8 + 2),
+             "encode_v": (lambda: tq.tq_encode_prod(cbv, V, rot64, vc, vs, vn, vg), 2 * d + d // 8 + d // 8 + 4),
+             "decode_k": (lambda: tq.tq_decode(cbk, rot64, kc, kn, kd), 3 * d // 8 + 2 + 4 * d),
+             "decode_v": (lambda: tq.tq_decode(cbv, rot64, vc, vn, vd, signs=vs, gammas=vg), d // 8 + d // 8 + 4 + 4 * d)}
+    blk = {}
+    for name, (fn, bpv) in calls.items():
+        ms = _timed(fn, 50)
+        msg = _graph_timed(fn, 20)
+        best = min(ms, msg) if msg is not None else ms
+        gbs = bpv * n / (best * 1e-3) / 1e9
+        blk[name] = {"ms": round(ms, 5), "graph_ms": None if msg is None else round(msg, 5),
+                     "vectors_per_s": n / (best * 1e-3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peak_hbm, 4)}
+    out["tinyllama_block_32x4096x64"] = blk
+    del K, V, kc, kn, vc, vs, vn, vg, kd, vd
+    # -- mixed widths per channel group: the llama8b-shaped K block at widths (3, 3, 2, 2) = 2.5 bits
+    d = 128
+    nblk = BLK_HEADS * BLK_TOKENS
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rotm = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    gb = [3, 3, 2, 2]
+    Km = W.kv_slices_device(BLK_HEADS, BLK_TOKENS, d, 3, 20.0, 0.5, 51, dev)
+    cm = torch.empty((nblk, sum(gb)), dtype=torch.int32, device=dev)
+    nm = torch.empty((nblk,), dtype=torch.float16, device=dev)
+    xm = torch.empty((nblk, d), dtype=torch.float32, device=dev)
+    ms_me = _timed(lambda: tq.tq_encode_mse_mixed(gb, Km, rotm, cm, nm), 20)
+    ms_md = _timed(lambda: tq.tq_decode_mixed(gb, rotm, cm, nm, xm), 20)
+    be = nblk * (2 * d + 4 * sum(gb) + 2)
+    bd = nblk * (4 * sum(gb) + 2 + 4 * d)
+    out["mixed_widths_3322_llama8b_k_block"] = {
+        "bits_per_coordinate": sum(gb) * 32 / d,
+        "encode_ms": round(ms_me, 4), "encode_GB/s": round(be / (ms_me * 1e-3) / 1e9, 1),
+        "encode_frac_hbm": round(be / (ms_me * 1e-3) / 1e9 / peak_hbm, 4),
+        "decode_ms": round(ms_md, 4), "decode_GB/s": round(bd / (ms_md * 1e-3) / 1e9, 1),
+        "decode_frac_hbm": round(bd / (ms_md * 1e-3) / 1e9 / peak_hbm, 4)}
+    del Km, cm, nm, xm
+    # -- prefill: 128 new query tokens at the end of a 32768-token cache, batch 1, 32 / 8 heads
+    Bp, Hqp, Hkvp, Tp, Qn = 1, 32, 8, 32768, 128
+    cbk, cbv = tq.tq_codebook_init(d, 3), tq.tq_codebook_init(d, 1)
+    npf = Bp * Hkvp * Tp
+    pkc, pkn = tq.empty_mse(npf, d, 3, dev)
+    pvc, pvs, pvn, pvg = tq.empty_prod(npf, d, 2, dev)
+    tq.tq_encode_mse(cbk, W.kv_slices_device(Hkvp, Tp, d, 3, 20.0, 0.5, 61, dev), rotm, pkc, pkn)
+    tq.tq_encode_prod(cbv, W.kv_slices_device(Hkvp, Tp, d, 3, 20.0, 0.5, 62, dev), rotm, pvc, pvs, pvn, pvg)
+    qp = torch.randn((Bp, Qn, Hqp, d), generator=torch.Generator(device=dev).manual_seed(63), device=dev).to(torch.bfloat16)
+    op = torch.empty((Bp, Qn, Hqp, d), dtype=torch.float32, device=dev)
+    wsp = torch.empty(tq.tq_attend_prefill_workspace_bytes(Bp, Hqp, Hkvp, Qn, Tp, d), dtype=torch.uint8, device=dev)
+    sh = (Bp, Hkvp, Tp)
+    ms_pf = _timed(lambda: tq.tq_attend_prefill(cbk, cbv, qp, rotm, pkc, pkn.view(sh), pvc, pvn.view(sh), op,
+                                                 v_signs=pvs, v_gammas=pvg.view(sh), ws=wsp), 5)
+    qpass = max(1, 8 // (Hqp // Hkvp))
+    passes = -(-Qn // qpass)
+    streamed = sum(B_ATT_TOKEN_HEAD * Bp * Hkvp * (Tp - Qn + j0 + min(qpass, Qn - j0)) for j0 in range(0, Qn, qpass))
+    flops = sum(2 * 2 * d * Hqp * (Tp - Qn + j + 1) for j in range(Qn)) * Bp       # q.k and p.v per visible token
+    out["prefill_B1_32x8_T32768_Q128"] = {
+        "ms": round(ms_pf, 3), "query_tokens_per_s": Bp * Qn / (ms_pf * 1e-3), "passes": passes,
+        "cache_bytes_streamed_GB": round(streamed / 1e9, 3),
+        "frac_hbm": round(streamed / (ms_pf * 1e-3) / 1e9 / peak_hbm, 4),
+        "frac_tensor_algorithmic": round(flops / (ms_pf * 1e-3) / 1e12 / peak_tensor, 5)}
+    del pkc, pkn, pvc, pvs, pvn, pvg, wsp
+    # -- vector search: 1e6 x 1536 fp32 unit rows, Algorithm 2 at b = 4, 1024 queries, top-10
+    d, n, nq, k = 1536, 1_000_000, 1024, 10
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rotv = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    g = torch.Generator(device=dev).manual_seed(41)
+    X = torch.empty((n, d), dtype=torch.float32, device=dev)
+    for r0 in range(0, n, 100_000):
+        blkx = torch.randn((min(100_000, n - r0), d), generator=g, device=dev)
+        X[r0:r0 + blkx.shape[0]] = blkx / blkx.norm(dim=1, keepdim=True)
+    qv = torch.randn((nq, d), generator=g, device=dev)
+    qv = qv / qv.norm(dim=1, keepdim=True)
+    cb3 = tq.tq_codebook_init(d, 3)
+    c, sg, nn, gm = tq.empty_prod(n, d, 4, dev)
+    ws = torch.empty(max(16, tq.tq_encode_workspace_bytes(n, d, 2)), dtype=torch.uint8, device=dev)
+    ms_enc = _timed(lambda: tq.tq_encode_prod(cb3, X, rotv, c, sg, nn, gm, ws=ws), 2, warmup=1)
+    ids = torch.empty((nq, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((nq, k), dtype=torch.float32, device=dev)
+    wss = torch.empty(max(16, tq.tq_scores_workspace_bytes(nq, n, d, k)), dtype=torch.uint8, device=dev)
+    ms_sc = _timed(lambda: tq.tq_scores(cb3, qv, rotv, c, nn, signs=sg, gammas=gm, k=k, topk_ids=ids,
+                                        topk_scores=sc, ws=wss), 3, warmup=1)
+    tq.tq_sync_check()
+    # algorithmic flops: encode 2 d^2 (Pi x) + 2 d^2 (T rho) per vector; scores 2 d (<q', c>) + 2 d
+    # (<q'', z>) per (query, vector). Issued: the tiled encoder's split products (2 or 3 for Pi x with
+    # bf16 / fp32 input: 3 here; 3 for T rho); the scores GEMM's K = (Walsh planes + sign plane) d
+    # against two fp16 query parts.
+    enc_alg = 4.0 * d * d * n
+    enc_iss = 2.0 * d * d * (3 + 3) * n
+    mk = 4                                   # Walsh planes of a 3-bit codebook
+    sc_alg = 4.0 * d * n * nq
+    sc_iss = 2.0 * (mk + 1) * d * 2 * n * nq
+    enc_bytes = n * (4 * d + 2 * d // 8 + d // 8 + 4 + d // 8)
+    out["vector_search_1e6x1536"] = {
+        "encode_ms": round(ms_enc, 3), "encode_vectors_per_s": n / (ms_enc * 1e-3),
+        "encode_frac_tensor_algorithmic": round(enc_alg / (ms_enc * 1e-3) / 1e12 / peak_tensor, 4),
+        "encode_frac_tensor_issued": round(enc_iss / (ms_enc * 1e-3) / 1e12 / peak_tensor, 4),
+        "encode_frac_hbm": round(enc_bytes / (ms_enc * 1e-3) / 1e9 / peak_hbm, 4),
+        "scores_topk_ms": round(ms_sc, 3),
+        "scores_frac_tensor_algorithmic": round(sc_alg / (ms_sc * 1e-3) / 1e12 / peak_tensor, 4),
+        "scores_frac_tensor_issued": round(sc_iss / (ms_sc * 1e-3) / 1e12 / peak_tensor, 4),
+        "scores_frac_hbm": round(n * (3 * d // 8 + d // 8 + 4) / (ms_sc * 1e-3) / 1e9 / peak_hbm, 4),
+        "peak_tensor_tflops": peak_tensor,
+    }
+    del X, c, sg, nn, gm, ws, wss
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_only_block(args):
@@ -552,6 +866,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' measurements")
     ap.add_argument("--only", choices=["attend", "block"], default=None,
                     help="profiling entry point: time one path alone (not a bench line)")
     ap.add_argument("--att-tokens", type=int, default=ATT_T)

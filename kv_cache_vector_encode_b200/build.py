@@ -8,6 +8,7 @@ host-only entry points work) on a machine without a GPU.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import hashlib
 import os
@@ -31,31 +32,47 @@ def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
-def _digest():
+def _headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) + \
+        [os.path.join(INCLUDE, "tq.h")]
+
+
+def _digest(files):
     h = hashlib.sha256()
-    for f in _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) \
-            + [os.path.join(INCLUDE, "tq.h"), __file__]:
+    for f in files + _headers() + [__file__]:
         h.update(open(f, "rb").read())
     h.update(" ".join(NVCC_FLAGS).encode())
     return h.hexdigest()
 
 
+def _compile(src, objdir, force, verbose):
+    """Compiles one source unless its object is up to date (same source, headers and flags)."""
+    obj = os.path.join(objdir, os.path.basename(src) + ".o")
+    stamp = obj + ".sha256"
+    dig = _digest([src])
+    if not force and os.path.exists(obj) and os.path.exists(stamp) and open(stamp).read() == dig:
+        return obj
+    cmd = ["nvcc", *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.run(cmd, check=True)
+    with open(stamp, "w") as f:
+        f.write(dig)
+    return obj
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libtq.so unless an up-to-date build is present; returns its path."""
+    """Compile libtq.so unless an up-to-date build is present; returns its path. Sources compile in
+    parallel, each only when it or a header changed."""
     stamp = LIB + ".sha256"
-    dig = _digest()
+    dig = _digest(_sources())
     if not force and os.path.exists(LIB) and os.path.exists(stamp) and open(stamp).read() == dig:
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in _sources():
-        obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = ["nvcc", *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
-        if verbose:
-            print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+    workers = max(1, min(len(_sources()), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        objs = list(ex.map(lambda s: _compile(s, objdir, force, verbose), _sources()))
     tmp = LIB + ".tmp"
     cmd = ["nvcc", "-shared", *NVCC_FLAGS, "-o", tmp, *objs]
     subprocess.run(cmd, check=True)

@@ -35,12 +35,13 @@ def test_product_package_does_not_import_the_oracle():
 
 def test_bench_uses_the_oracle_only_in_its_baseline_legs():
     users = set(_oracle_imports(os.path.join(ROOT, "bench.py"))) - {"<module>"}
-    assert users <= {"oracle_step", "run_reference", "cpu_baseline_measure"}, users
-    # and oracle_step itself is only reached from those legs
+    assert users <= {"oracle_step", "oracle_per_workload", "run_reference", "cpu_baseline_measure"}, users
+    # and the oracle helpers themselves are only reached from those legs
     tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
-    callers = {fn.name for fn in ast.walk(tree) if isinstance(fn, ast.FunctionDef)
-               for c in ast.walk(fn) if isinstance(c, ast.Call) and getattr(c.func, "id", "") == "oracle_step"}
-    assert callers <= {"run_reference", "cpu_baseline_measure"}, callers
+    for helper in ("oracle_step", "oracle_per_workload"):
+        callers = {fn.name for fn in ast.walk(tree) if isinstance(fn, ast.FunctionDef)
+                   for c in ast.walk(fn) if isinstance(c, ast.Call) and getattr(c.func, "id", "") == helper}
+        assert callers <= {"run_reference", "cpu_baseline_measure"}, (helper, callers)
 
 
 def test_missing_native_library_fails_loudly():

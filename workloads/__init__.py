@@ -133,3 +133,24 @@ WORKLOADS = {
                              outlier_scale=20.0, lognormal_sigma=0.5, k_bits=3, v_bits=2),
     "vector_search": dict(n=1_000_000, d=1536, queries=1024, bits=4, topk=10),
 }
+
+
+def kv_slices_device(slices: int, tokens: int, d: int, n_outlier: int, outlier_scale: float,
+                     lognormal_sigma: float, seed: int, device):
+    """The ``kv_block`` recipe drawn on a CUDA device with a torch generator, for caches too large to
+    draw on the host in a test: [slices * tokens, d] bf16, each slice of ``tokens`` rows N(0,1) with
+    ``n_outlier`` channels x ``outlier_scale`` and optional log-normal token norms. Not bit-identical
+    to ``kv_block`` (a different generator); same distribution."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    out = torch.empty((slices, tokens, d), dtype=torch.bfloat16, device=device)
+    for s in range(slices):
+        x = torch.randn((tokens, d), generator=g, device=device)
+        if n_outlier > 0:
+            ch = torch.randperm(d, generator=g, device=device)[:n_outlier]
+            x[:, ch] *= outlier_scale
+        if lognormal_sigma > 0:
+            x *= torch.exp(lognormal_sigma * torch.randn((tokens, 1), generator=g, device=device))
+        out[s] = x.to(torch.bfloat16)
+    return out.view(-1, d)
