@@ -67,10 +67,37 @@ def tensor_peak():
         return 1590.0, "fallback"
 
 
+_CLOCK_CHILD = r"""
+import select, sys
+import pynvml as nv
+nv.nvmlInit()
+key, period = sys.argv[1], float(sys.argv[2])
+try:
+    h = nv.nvmlDeviceGetHandleByUUID(key)
+except Exception:
+    h = nv.nvmlDeviceGetHandleByIndex(int(sys.argv[3]))
+mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+        nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+out = []
+print("ready", flush=True)
+while True:
+    try:
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+        out.append("%d,%d,%s" % (sm, mx, ",".join("1" if r & b else "0" for b in bits)))
+    except Exception:
+        pass
+    if select.select([sys.stdin], [], [], period)[0]:
+        break                                   # the parent closed our stdin: the region is over
+print("\n".join(out), flush=True)
+"""
+
+
 class ClockSampler:
-    """SM clock and throttle-reason samples while the timed region runs: NVML polled every 2 ms from
-    a thread (so a timed region of tens of milliseconds still gets many samples), else nvidia-smi
-    every 20 ms. Reads settings only."""
+    """SM clock and throttle-reason samples while the timed region runs. A child process polls NVML
+    every 2 ms (a thread of this process would compete for the interpreter lock with the launch
+    loop), else nvidia-smi reports every 20 ms. Reads settings only."""
 
     SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                   "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -81,75 +108,69 @@ class ClockSampler:
         self.period = period_s
         self.proc = None
         self.thread = None
-        self.stop = threading.Event()
         self.samples = []          # (sm_mhz, max_mhz, set of reason names)
         self.source = None
 
-    def _nvml_handle(self):
-        import pynvml
-        import torch
-        pynvml.nvmlInit()
+    def _parse(self, line):
+        parts = [x.strip() for x in line.strip().split(",")]
+        if len(parts) < 6:
+            return
         try:
-            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
-            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-        except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            sm, mx = float(parts[0]), float(parts[1])
+        except ValueError:
+            return
+        act = [v.lower().startswith("active") or v == "1" for v in parts[2:6]]
+        self.samples.append((sm, mx, {nm for nm, a in zip(self.NAMES, act) if a}))
 
-    def _poll_nvml(self, nv, h):
-        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
-                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
-                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
-                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
-        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
-        while not self.stop.is_set():
-            try:
-                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
-                self.samples.append((sm, mx, {k for k, v in bits.items() if r & v}))
-            except Exception:
-                pass
-            time.sleep(self.period)
-
-    def _read_smi(self):
-        for line in self.proc.stdout:
-            parts = [x.strip() for x in line.strip().split(",")]
-            if len(parts) < 6:
-                continue
-            try:
-                sm, mx = float(parts[0]), float(parts[1])
-            except ValueError:
-                continue
-            self.samples.append((sm, mx, {nm for nm, v in zip(self.NAMES, parts[2:6]) if v.lower().startswith("active")}))
+    def _start_nvml_child(self):
+        import torch
+        uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        proc = subprocess.Popen([sys.executable, "-c", _CLOCK_CHILD, uuid, str(self.period), str(self.index)],
+                                stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        if proc.stdout.readline().strip() != "ready":
+            proc.kill()
+            proc.wait()
+            raise RuntimeError("NVML sampler did not start")
+        return proc
 
     def __enter__(self):
         try:
-            nv, h = self._nvml_handle()
-            self.thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
-            self.source = "nvml, every 2 ms"
+            self.proc = self._start_nvml_child()
+            self.source = "nvml in a child process, every 2 ms"
         except Exception:
             try:
                 self.proc = subprocess.Popen(
                     ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.SMI_FIELDS}",
                      "--format=csv,noheader,nounits", "-lms", "20"],
                     stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-                self.thread = threading.Thread(target=self._read_smi, daemon=True)
+                self.thread = threading.Thread(target=lambda: [self._parse(ln) for ln in self.proc.stdout],
+                                               daemon=True)
+                self.thread.start()
                 self.source = "nvidia-smi, every 20 ms"
             except Exception:
-                self.thread = None
-        if self.thread is not None:
-            self.thread.start()
+                self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.stop.set()
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.proc is None:
+            return
+        if self.thread is None:
+            # the NVML child: closing its stdin ends the loop, then it prints its samples
             try:
-                self.proc.wait(timeout=5)
+                out, _ = self.proc.communicate(input="", timeout=30)
+                for ln in out.splitlines():
+                    self._parse(ln)
             except Exception:
                 self.proc.kill()
-        if self.thread is not None:
-            self.thread.join(timeout=5)
+                self.proc.wait()
+            return
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
 
     def summary(self):
         if not self.samples:
@@ -528,11 +549,18 @@ def run_ours(args):
     peak, peak_kind = peaks()
     att_bytes = B_ATT_TOKEN_HEAD * ATT_B * ATT_HKV * ATT_T + ATT_B * ATT_HQ * D * (2 + 4)
     att_gbs = att_bytes / (parts["attend"] * 1e-3) / 1e9
+    # DRAM bytes of one launch from the committed ncu capture, only while the kernel source is the
+    # one that was captured (its sha256 is recorded beside the figure)
     traffic = None
     prof = os.path.join(ROOT, "profiles", "attend_main_decode_attention_traffic.json")
     if os.path.exists(prof):
         try:
-            traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+            rec = json.load(open(prof))
+            import hashlib
+            with open(os.path.join(ROOT, "kv_cache_vector_encode_b200", "csrc", "attend.cu"), "rb") as f:
+                cur = hashlib.sha256(f.read()).hexdigest()
+            if rec.get("source_sha256") == cur:
+                traffic = rec.get("dram_bytes_per_launch")
         except Exception:
             traffic = None
     comp_bytes = {
@@ -859,6 +887,28 @@ def run_only_attend(args):
     return 0
 
 
+def run_only_tiled(args):
+    """Times tq_encode_prod on `--tiled-n` unit-norm fp32 rows of d = 1536 at 4 bits (the vector-search
+    encode, the tiled kernel and its gamma fix-up; a profiling entry point, not a bench line)."""
+    import torch
+    import kv_cache_vector_encode_b200 as tq
+    import workloads as W
+    dev = torch.device("cuda")
+    d, n = 1536, args.tiled_n
+    Pi, S = W.rotation(d), W.jl_matrix(d)
+    rot = tq.tq_rotation_prepare(torch.from_numpy(Pi).to(dev), torch.from_numpy(S).to(dev))
+    g = torch.Generator(device=dev).manual_seed(41)
+    X = torch.randn((n, d), generator=g, device=dev)
+    X = X / X.norm(dim=1, keepdim=True)
+    cb = tq.tq_codebook_init(d, 3)
+    c, sg, nn, gm = tq.empty_prod(n, d, 4, dev)
+    ws = torch.empty(max(16, tq.tq_encode_workspace_bytes(n, d, 2)), dtype=torch.uint8, device=dev)
+    ms = _timed(lambda: tq.tq_encode_prod(cb, X, rot, c, sg, nn, gm, ws=ws), args.steps, warmup=args.warmup)
+    tq.tq_sync_check()
+    print(json.dumps({"only": "tiled", "n": n, "d": d, "ms_per_call": ms, "vectors_per_s": n / (ms * 1e-3)}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -867,9 +917,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' measurements")
-    ap.add_argument("--only", choices=["attend", "block"], default=None,
+    ap.add_argument("--only", choices=["attend", "block", "tiled"], default=None,
                     help="profiling entry point: time one path alone (not a bench line)")
     ap.add_argument("--att-tokens", type=int, default=ATT_T)
+    ap.add_argument("--tiled-n", type=int, default=16384)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -879,6 +930,8 @@ def main():
         return run_only_attend(args)
     if args.only == "block":
         return run_only_block(args)
+    if args.only == "tiled":
+        return run_only_tiled(args)
     return run_ours(args)
 
 

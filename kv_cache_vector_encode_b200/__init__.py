@@ -198,17 +198,23 @@ def tq_decode(cb: Codebook, rot, codes, norms, out, signs=None, gammas=None, str
                            _ptr(out, "out", [torch.float32, torch.bfloat16]), _xdtype(out), _stream(stream)))
 
 
+_mixed_cache = {}
+
+
 def _mixed_args(d: int, group_bits):
-    """Host arrays of the mixed-width calls: the 4 codebooks of d (1..4 bits) and the group widths."""
-    G = d // 32
-    if len(group_bits) != G:
-        raise ValueError(f"group_bits needs {G} entries for d = {d}")
-    cbs = (Codebook * 4)()
-    for b in sorted(set(int(x) for x in group_bits)):
-        if 1 <= b <= 4:
-            cbs[b - 1] = tq_codebook_init(d, b)
-    gb = (ctypes.c_int32 * G)(*[int(x) for x in group_bits])
-    return cbs, gb
+    """Host arrays of the mixed-width calls: the 4 codebooks of d (1..4 bits) and the group widths
+    (made once per (d, widths); the codebooks come from the library's host solver)."""
+    key = (int(d), tuple(int(x) for x in group_bits))
+    if key not in _mixed_cache:
+        G = d // 32
+        if len(key[1]) != G:
+            raise ValueError(f"group_bits needs {G} entries for d = {d}")
+        cbs = (Codebook * 4)()
+        for b in sorted(set(key[1])):
+            if 1 <= b <= 4:
+                cbs[b - 1] = tq_codebook_init(d, b)
+        _mixed_cache[key] = (cbs, (ctypes.c_int32 * G)(*key[1]))
+    return _mixed_cache[key]
 
 
 def tq_encode_mse_mixed(group_bits, x, rot, codes, norms, stream=None):

@@ -19,10 +19,11 @@
 //   * values are accumulated in the rotated / sign domain. For each value plane P (the Walsh
 //     planes of the value codes, then the sign plane) the value MMA gives Y_P[i] = sum_t w_t b_P,t,i
 //     with the softmax weights w_t (times the value norm, times gamma for the sign plane) in 32-bit
-//     unsigned fixed point (24 bits) as 8-bit limbs. The chunk sums W = sum_t w_t (and of the other
-//     weight kinds) are exact integer warp reductions, and the per-chunk folds
+//     unsigned fixed point (24 bits) as 8-bit limbs. Over a run of chunks with unchanged maxima and
+//     scales, the value MMAs accumulate Y_P in TMEM, and the value MMA warp adds up the run's weights
+//     W = sum_t w_t (and W' of the sign plane) exactly from the same weight tiles; the folds
 //       O_P = sum_t w_t (1 - 2 b_P,t) = W - 2 Y_P,   O_z = sum_t w'_t (2 z_t - 1) = 2 Y_z - W'
-//     are formed per chunk before the running (rescaled) accumulation;
+//     are formed once per run before the running (rescaled) accumulation;
 //   * once per query head: out = (Pi^T sum_P beta_P O_P + alpha S^T O_z) / sum_t p_t.
 //
 // Bit expansion: a 32-bit plane word w covers 32 coordinates; register s (s = 0..7) of
@@ -76,10 +77,13 @@ struct AttParams {
   // token j of the pass and head h are virtual head j * Hgr + h. Decode has nqry = 1 (Hg = Hgr).
   int Hg, Hgr, nqry;
   int64_t q_bs, q_js;            // element strides of q and out: batch, query token (head stride d)
-  int64_t tlim0;                 // query token j of the pass attends the tokens t < tlim0 + j
+  int64_t tlim0;                 // query token j attends the tokens t < tlim0 + j
+  // A launch may hold several passes: work slice s is pass s / cslices over cache slice s % cslices
+  // (b * Hkv + hk); pass ps serves query tokens ps * nqry .. ps * nqry + nqry - 1 of nqtot.
+  int cslices, nqtot;
   int64_t T;                     // tokens attended per slice
   int64_t tstride;               // token slots per slice in the cache arrays (>= T)
-  int slices, nchunk, per_cta, maxseg;
+  int slices, nchunk, per_cta, maxseg;   // work slices (passes x cache slices), chunks per slice
   int nst;                       // depth of the packed-chunk ring
   int norm_bulk;                 // 1: the norm arrays are bulk-copied into the stage with the codes
                                  // (slot stride a multiple of 8 tokens, 16-byte aligned arrays)
@@ -186,8 +190,9 @@ __device__ void append_encode(const AttParams& p, int slice, const void* xsrc, b
 // prep: q' = Pi q per query head, fixed-point limbs of beta_S q' (scaled by 2^-s), constants
 // ------------------------------------------------------------------------------------------------
 __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
-  const int slice = blockIdx.x;                  // = b * Hkv + hk
-  const int b = slice / p.Hkv, hk = slice % p.Hkv;
+  const int slice = blockIdx.x;                  // work slice: pass * cslices + b * Hkv + hk
+  const int cs = slice % p.cslices, ps = slice / p.cslices;
+  const int b = cs / p.Hkv, hk = cs % p.Hkv;
   const int d = p.d, i = threadIdx.x;            // coordinate (128 threads)
   const int warp = i >> 5, lane = i & 31;
   __shared__ __align__(16) float sq[8][128];
@@ -204,9 +209,11 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
   uint8_t* img = p.bq_img + (size_t)slice * p.nq * kbytes;
   for (int o = i; o < p.nq * kbytes / 16; o += blockDim.x) ((uint4*)img)[o] = make_uint4(0, 0, 0, 0);
   for (int h = 0; h < p.Hg; ++h) {
-    const size_t qoff = (size_t)b * p.q_bs + (size_t)(h / p.Hgr) * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * d;
-    sq[h][i] = p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
-                        : ((const float*)p.q)[qoff + i];
+    const int j = ps * p.nqry + h / p.Hgr;       // query token of virtual head h (none past nqtot)
+    const size_t qoff = (size_t)b * p.q_bs + (size_t)j * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * d;
+    sq[h][i] = j >= p.nqtot ? 0.0f
+                            : (p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
+                                        : ((const float*)p.q)[qoff + i]);
   }
   __syncthreads();
   // q'_h[i] = sum_j Pi[i][j] q_h[j] for every head: one thread per output coordinate, its row of Pi
@@ -313,8 +320,9 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
 // (exact int32 limb sums) and the accumulator warps fold it once. Runs stop at 256 chunks, which
 // keeps every limb sum below 2^30. Run record (kRunRec bytes): [0, 32) running maxima of the 8
 // heads, [32] 1/sw, [36] 1/sw', [40] flags (1 = last run of its segment, 2 = last run of the CTA),
-// [44] segment ordinal, [48] slice, [64, 256) exact run sums (uint64) of the weight kinds
-// w, w gamma, p (2^22 fixed point) for the 8 heads.
+// [44] segment ordinal, [48] slice, [64, 192) exact run sums (uint64) of the weight kinds w and
+// w gamma for the 8 heads, [192, 224) the segment's sums of p for the 8 heads (last run of a
+// segment only).
 constexpr int kRunRec = 256;
 constexpr int kMaxRun = 256;
 
@@ -346,7 +354,7 @@ __host__ __device__ inline AttLayout att_layout(const AttParams& p, int nst) {
   L.off_bq = off; off += 2 * L.bq_bytes;
   L.off_sc = off; off += 4 * 64 * 4;               // chunk scalars, 4-deep ring of 64 floats
   L.off_red = off; off += 2 * 4 * 16 * 4;          // max exchange of the softmax warps: [group][warp][16]
-  L.off_sum = off; off += 4 * 4 * 24 * 4;          // chunk sums of the weights: [ring][warp][kind][head]
+  L.off_sum = off; off += 4 * 4 * 8 * 4;           // segment sums of p: [4 slots][warp][head]
   L.off_run = aru(off, 16); off = L.off_run + 2 * kRunRec;   // records of the two runs in flight
   L.off_bar = aru(off, 8); off = L.off_bar + 64 * 8;
   L.total = off + 1024;
@@ -368,7 +376,8 @@ enum ABars {
   RUN_DONE = V_DONE + 6,               // [2]  value MMA warp -> accumulators: a run's MMAs complete (commit)
                                        //      and its record written (arrive): 2 arrivals
   RUN_FREE = RUN_DONE + 2,             // [2]  accumulators -> value MMA warp: run buffer drained (4 warps)
-  ANBARS = RUN_FREE + 2
+  SC_FREE = RUN_FREE + 2,              // [2]  softmax -> key MMA warp: scores buffer read (8 warps)
+  ANBARS = SC_FREE + 2
 };
 
 // TMEM columns: A_K [2][32 (mk + ksign)] at 0, scores [2][nq (1 + ksign)] after them, value
@@ -378,18 +387,21 @@ enum ABars {
 // Walks this CTA's chunks in order (slice, chunk inside the slice, segment ordinal) without
 // integer division.
 struct ChunkIter {
-  int slice, cis, seg, nchunk;
+  int slice, cis, seg, nchunk, cs, ncs;   // work slice, chunk in it, segment ordinal; cache slice
   __device__ __forceinline__ void init(const AttParams& p, int gchunk) {
     nchunk = p.nchunk;
     slice = gchunk / nchunk;
     cis = gchunk - slice * nchunk;
     seg = 0;
+    ncs = p.cslices;
+    cs = slice % ncs;
   }
   __device__ __forceinline__ void next() {
     if (++cis == nchunk) {
       cis = 0;
       ++slice;
       ++seg;
+      if (++cs == ncs) cs = 0;
     }
   }
 };
@@ -413,10 +425,14 @@ __host__ __device__ constexpr int walsh_mask(int bits, int S) {
   return bits == 3 ? (S == 0 ? 1 : (S == 1 ? 2 : (S == 2 ? 4 : 7))) : (S == 0 ? 1 : 2);
 }
 
-// Exact int -> float for |x| < 2^22 with two full-rate operations (exponent-field trick).
-__device__ __forceinline__ float small_i2f(int x) {
-  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+// l0 + 2^8 l1 + 2^16 l2 + 2^24 l3 for signed limb sums |l| < 2^21: the pairs are exact in 32 bits
+// (|l0 + 2^8 l1| < 2^30), then two conversions and one FMA.
+__device__ __forceinline__ float limbs_to_float(uint32_t l0, uint32_t l1, uint32_t l2, uint32_t l3) {
+  const int lo = (int)l0 + (int)(l1 << 8);
+  const int hi = (int)l2 + (int)(l3 << 8);
+  return fmaf((float)hi, 65536.0f, (float)lo);
 }
+
 // Round-to-nearest of 0 <= v <= 2^23 to an integer with one FMA (v = a * b).
 __device__ __forceinline__ uint32_t fixed24(float a, float b) {
   return __float_as_uint(fmaf(a, b, 8388608.0f)) - 0x4B000000u;
@@ -439,6 +455,11 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
   uint32_t r;
   asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
   return r;
+}
+// exact warp sum of values below 2^43: the low 16 bits and the rest are reduced separately
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+  const uint32_t lo = warp_sum_u32((uint32_t)v & 0xFFFFu), hi = warp_sum_u32((uint32_t)(v >> 16));
+  return ((unsigned long long)hi << 16) + lo;
 }
 
 // Value planes of one token (thread = token t of the chunk): plane words (and sign words) ->
@@ -478,6 +499,8 @@ __device__ __forceinline__ void expand_v_rows(const AttParams& p, const AttLayou
 
 // HG: query heads per KV head (4 or 8, Hg <= HG); BK: key codebook bits; BV: value codebook bits;
 // VS: value sign plane (Algorithm 2 values); KS: key sign plane (Algorithm 2 keys, BK <= 2)
+// Register cap: the most that fits the warps an SM sub-partition holds (16384 registers each; 6 of
+// the 23 warps, or 5 of the 19, in units of 8 registers a thread).
 template <int HG, int BK, int BV, int VS, int KS>
 __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const __grid_constant__ AttParams p) {
   constexpr bool SPLITV = att_split_v(HG);
@@ -500,7 +523,6 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + ANBARS) + 1;
   float* scal = (float*)(smem + Lo.off_sc);
   float* red = (float*)(smem + Lo.off_red);
-  uint32_t* sums = (uint32_t*)(smem + Lo.off_sum);   // [4 ring][4 warps][3 kinds][8 heads]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = p.slices * p.nchunk;
   const int c_begin = blockIdx.x * p.per_cta;
@@ -526,6 +548,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       mbar_init(&bar[BW_FULL + s], 8);
       mbar_init(&bar[RUN_DONE + s], 2);
       mbar_init(&bar[RUN_FREE + s], 4);
+      mbar_init(&bar[SC_FREE + s], 8);
     }
     for (int s = 0; s < 3; ++s) mbar_init(&bar[AV_FULL + s], 4);
     for (int s = 0; s < 6; ++s) mbar_init(&bar[V_DONE + s], 1);
@@ -563,7 +586,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       const int st = rs.slot;
       if (!mbar_wait_warp(&bar[ST_EMPTY + st], rs.par ^ 1u, p.err, kDevTimeoutSync, abort_flag)) break;
       const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
-      const int64_t vec0 = (int64_t)it.slice * TS + (int64_t)it.cis * kChunk;  // record of the first token
+      const int64_t vec0 = (int64_t)it.cs * TS + (int64_t)it.cis * kChunk;  // record of the first token
       const uint32_t kb = (uint32_t)tc * G * BK * 4;
       const uint32_t vb = (uint32_t)tc * G * BV * 4;
       const uint32_t sb = VS ? (uint32_t)tc * G * 4 : 0u;
@@ -603,7 +626,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (!mbar_wait_warp(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
       }
       if (!mbar_wait_warp(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      // the scores buffer b is free once the softmax warps finished chunk c-2
+      // the scores buffer b is free once the softmax warps have read the scores of chunk c-2
       if (c >= 2 && !mbar_wait_warp(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag))
         break;
       tc_fence_after();
@@ -641,6 +664,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     int hlim[HH];                                   // each head sees the slice's tokens t < hlim (causal)
     float vmax_run = 0.0f, gmax_run = 0.0f, sw = 1.0f, sw2 = 1.0f, isw = 1.0f, isw2 = 1.0f;
     bool ok = true;
+    // this thread's token's share of the segment's sum of p (rescaled with the running maximum),
+    // reduced over the group once, at the segment's end, into one of 4 slots (a slot is written again
+    // four segments later, after the value MMA warp has read it)
+    float lt[HH];
+    float* segl = (float*)(smem + Lo.off_sum);      // [slot][warp][head]
     // fp16 norms of the chunk's tokens: from the stage (bulk-copied with the codes) where possible,
     // else from global memory (dead tokens read as zero)
     RingPos rs{0, nst, 0u};
@@ -657,7 +685,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (VS) gm_n = sn[2 * kChunk + t];
         if (KS) gk_n = sn[3 * kChunk + t];
       } else if (live) {
-        const int64_t rec = (int64_t)it.slice * TS + (int64_t)it.cis * kChunk + t;
+        const int64_t rec = (int64_t)it.cs * TS + (int64_t)it.cis * kChunk + t;
         nk_n = __ldg(p.k_norms + rec);
         nv_n = __ldg(p.v_norms + rec);
         if (VS) gm_n = __ldg(p.v_gammas + rec);
@@ -674,14 +702,16 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           mrun[i] = -INFINITY;
+          lt[i] = 0.0f;
           const float4 x = h0 + i < Hg ? __ldg(hc + h0 + i) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
           ha[i] = -2.0f * x.x * p.scale_log2e;
           hb[i] = x.y * p.scale_log2e;
           // key sign term alpha gamma <q'', 2z - 1> = alpha gamma (2 2^-F'' D_z - Q'')
           hs[i] = 2.0f * p.alpha * x.z * p.scale_log2e;
           hq[i] = -p.alpha * x.w * p.scale_log2e;
-          // virtual head h0 + i is query token (h0 + i) / Hgr of the pass
-          hlim[i] = (int)(p.tlim0 + (h0 + i) / p.Hgr);
+          // virtual head h0 + i is query token j = pass * nqry + (h0 + i) / Hgr; tokens t < tlim0 + j
+          const int j = (it.slice / p.cslices) * p.nqry + (h0 + i) / p.Hgr;
+          hlim[i] = (h0 + i < Hg && j < p.nqtot) ? (int)(p.tlim0 + j) : 0;   // heads past Hg see nothing
         }
       }
       const int tg = it.cis * kChunk + t;           // this thread's token, counted in the slice
@@ -701,18 +731,15 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       bool up = nv > vmax_run || nv * gm > gmax_run;
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        // the four limb products are exact integers below 2^21 in magnitude
-        const float dot = fmaf(fmaf(fmaf(small_i2f((int)dsr[4 * i + 3]), 256.0f, small_i2f((int)dsr[4 * i + 2])), 256.0f,
-                                    small_i2f((int)dsr[4 * i + 1])),
-                               256.0f, small_i2f((int)dsr[4 * i]));
+        // the four limb products are exact integers below 2^21 in magnitude: pairs of limbs combine
+        // exactly in 32 bits, then one fp32 rounding each
+        const float dot = limbs_to_float(dsr[4 * i], dsr[4 * i + 1], dsr[4 * i + 2], dsr[4 * i + 3]);
         float sc = fmaf(ha[i], dot, hb[i]);
         if (KS) {
-          const float dz = fmaf(fmaf(fmaf(small_i2f((int)dzr[4 * i + 3]), 256.0f, small_i2f((int)dzr[4 * i + 2])),
-                                     256.0f, small_i2f((int)dzr[4 * i + 1])),
-                                256.0f, small_i2f((int)dzr[4 * i]));
+          const float dz = limbs_to_float(dzr[4 * i], dzr[4 * i + 1], dzr[4 * i + 2], dzr[4 * i + 3]);
           sc = fmaf(gk, fmaf(hs[i], dz, hq[i]), sc);
         }
-        lg[i] = (h0 + i < Hg && live && tg < hlim[i]) ? nk * sc : -INFINITY;
+        lg[i] = (live && tg < hlim[i]) ? nk * sc : -INFINITY;
         up = up || lg[i] > mrun[i];
       }
       float corr[HH];
@@ -756,30 +783,28 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         isw2 = nisw2;
       }
       // weights: p = 2^(lg - m) <= 1, w = p |v|, w' = w gamma, as 24-bit unsigned fixed point
-      uint32_t wv[HH], wz[HH], pv[HH];
+      uint32_t wv[HH], wz[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         const float pr = (lg[i] == -INFINITY) ? 0.0f : fast_exp2(lg[i] - mrun[i]);
         const float w = pr * nv;
         wv[i] = fixed24(w, sw);
         wz[i] = VS ? fixed24(w * gm, sw2) : 0u;
-        pv[i] = fixed24(pr, 4194304.0f);            // p * 2^22
-      }
-      // chunk sums of each weight kind per head (exact: 32 values below 2^24 per warp)
-      uint32_t* su = sums + ((c & 3) * 4 + q) * 24 + h0;
-#pragma unroll
-      for (int i = 0; i < HH; ++i) {
-        const uint32_t s0 = warp_sum_u32(wv[i]);
-        const uint32_t s1 = VS ? warp_sum_u32(wz[i]) : 0u;
-        const uint32_t s2 = warp_sum_u32(pv[i]);
-        if (lane == 0) {
-          su[i] = s0;
-          su[8 + i] = s1;
-          su[16 + i] = s2;
-        }
+        lt[i] = fmaf(lt[i], corr[i], pr);
       }
       // the weight tiles of chunk c-2 (same buffer) must have been consumed by its value MMA
       if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + (c - 2) % 6], ((c - 2) / 6) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
+      if (c == nmy - 1 || it.cis == p.nchunk - 1) {
+        // the segment ends with this chunk: the group's sums of p of its heads
+        float* lp = segl + ((it.seg & 3) * 4 + q) * 8;
+#pragma unroll
+        for (int i = 0; i < HH; ++i) {
+          float sl = lt[i];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
+          if (lane == 0) lp[h0 + i] = sl;
+        }
+      }
       // this group's heads fill 4 HH bytes of the token's row (block h0 / 4, byte 4 (h0 % 4))
       uint8_t* bwb = smem + Lo.off_bw + b * Lo.bw_buf + (h0 >> 2) * kChunk * 16 + t * 16 + (h0 & 3) * 4;
       if (HH == 2) {
@@ -930,7 +955,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         const float mr = rm[h];
         corr[h] = macc[h] == -INFINITY ? 0.0f : fast_exp2(macc[h] - mr);
         macc[h] = mr;
-        if (m == 0) Lr[h] = fmaf(Lr[h], corr[h], (float)rs[16 + h] * (1.0f / 4194304.0f));
+        // sum of p of the segment (at the segment's final maxima), with its last run
+        if ((flags & 1) && m == 0) Lr[h] = ((const float*)(rr + 192))[h];
       }
       // one plane at a time (keeps the TMEM columns of a single plane in registers)
 #pragma unroll
@@ -977,17 +1003,33 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     // ------------------------------------ value MMA issuer (warp 18) ------------------------------
     // Runs beside the key MMA warp so that neither warp's barrier waits and commits sit behind the
     // other's tensor-core work. Warp-uniform schedule, one elected lane issues. It also keeps the
-    // runs: a chunk whose softmax scalars moved starts a new run in the other TMEM buffer; lanes
-    // 0..23 add up the chunk weight sums of the run (kind lane / 8, head lane % 8) in 64 bits.
+    // runs: a chunk whose softmax scalars moved starts a new run in the other TMEM buffer. The warp
+    // also adds up each run's weights exactly (lane = four tokens of each chunk) from the weight tiles.
     const uint32_t id_v = idesc_i8_s32(128, NQ, false, false, true, true);
     const uint64_t da0 = desc_smem(smem_u32(smem + Lo.off_av), 1024, 1024, 2);
     const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
     int R = -1, runlen = 0;
     bool open = false;
-    unsigned long long rsum = 0;
+    // this lane's share of the run's weight sums (tokens lane + 32 j of every chunk; below 2^33)
+    unsigned long long aw[HG], az[VS ? HG : 1];
+    const float* segl = (const float*)(smem + Lo.off_sum);
     auto close_run = [&](int flags, int seg) {
       uint8_t* rr = smem + Lo.off_run + (R & 1) * kRunRec;
-      if (lane < 24) ((unsigned long long*)(rr + 64))[lane] = rsum;
+      unsigned long long* rs = (unsigned long long*)(rr + 64);
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const unsigned long long tw = warp_sum_u64(aw[h]);
+        const unsigned long long tz = VS ? warp_sum_u64(az[VS ? h : 0]) : 0ull;
+        if (lane == 0) {
+          rs[h] = tw;
+          rs[8 + h] = tz;
+        }
+      }
+      if ((flags & 1) && lane < 8) {
+        // the segment's sums of p (four warp partials per head)
+        const float* lp = segl + (it.seg & 3) * 32 + lane;
+        ((float*)(rr + 192))[lane] = (lp[0] + lp[8]) + (lp[16] + lp[24]);
+      }
       if (lane == 0) {
         *(int*)(rr + 40) = flags;
         *(int*)(rr + 44) = seg;
@@ -1010,7 +1052,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (open) close_run(0, 0);
         ++R;
         runlen = 0;
-        rsum = 0;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          aw[h] = 0;
+          if (VS) az[VS ? h : 0] = 0;
+        }
         // the other buffer's previous run must have been drained by the accumulators
         if (R >= 2 && !mbar_wait_warp(&bar[RUN_FREE + (R & 1)], ((R >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
           break;
@@ -1018,10 +1064,6 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (lane < 10) ((float*)rr)[lane] = lane < 8 ? sc[16 + lane] : sc[32 + lane - 8];
         if (lane == 10) *(int*)(rr + 48) = it.slice;
         open = true;
-      }
-      if (lane < 24) {
-        const uint32_t* su = sums + (c & 3) * 96 + lane;
-        rsum += (unsigned long long)((su[0] + su[24]) + (su[48] + su[72]));   // four warp partials, < 2^31
       }
       tc_fence_after();
       const uint32_t dcol = tbase + dv0 + (R & 1) * dv_cols;
@@ -1036,8 +1078,31 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
             mma_i8_ss(dcol + P * NQ, da + ((P * Lo.av_bytes + ks * 32 * 128) >> 4),
                       db + (((sgn ? Lo.bw_kind : 0u) + ks * 32 * 16) >> 4), id_v, (ks > 0 || !newrun) ? 1u : 0u);
         }
-        mma_commit(&bar[V_DONE + c % 6]);
       }
+      __syncwarp();
+      {
+        // the chunk's weights into the run sums, read before the commit below releases the tiles to
+        // the softmax warps (the adds consume the loads first)
+        const uint8_t* bwt = smem + Lo.off_bw + b * Lo.bw_buf + lane * 16;
+#pragma unroll
+        for (int blk = 0; blk < HG / 4; ++blk) {
+#pragma unroll
+          for (int kind = 0; kind < 1 + VS; ++kind) {
+            const uint8_t* x = bwt + blk * kChunk * 16 + kind * Lo.bw_kind;
+            const uint4 a0 = *(const uint4*)x, a1 = *(const uint4*)(x + 32 * 16);
+            const uint4 a2 = *(const uint4*)(x + 64 * 16), a3 = *(const uint4*)(x + 96 * 16);
+            const uint32_t s4[4] = {(a0.x + a1.x) + (a2.x + a3.x), (a0.y + a1.y) + (a2.y + a3.y),
+                                    (a0.z + a1.z) + (a2.z + a3.z), (a0.w + a1.w) + (a2.w + a3.w)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (kind == 0) aw[4 * blk + j] += s4[j];
+              else az[VS ? 4 * blk + j : 0] += s4[j];
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (elect_one_sync()) mma_commit(&bar[V_DONE + c % 6]);
       __syncwarp();
       ++runlen;
       if (c == nmy - 1 || it.cis == p.nchunk - 1) {
@@ -1085,10 +1150,13 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
 // combine: merge the partial states of a slice, apply Pi^T and alpha S^T once per query head
 // ------------------------------------------------------------------------------------------------
 __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
-  const int slice = blockIdx.x / p.Hg;       // one block per (slice, virtual head)
+  const int slice = blockIdx.x / p.Hg;       // one block per (work slice, virtual head)
   const int h = blockIdx.x % p.Hg;
-  const int b = slice / p.Hkv, hk = slice % p.Hkv;
-  const size_t ooff = (size_t)b * p.q_bs + (size_t)(h / p.Hgr) * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * p.d;
+  const int cs = slice % p.cslices, ps = slice / p.cslices;
+  const int b = cs / p.Hkv, hk = cs % p.Hkv;
+  const int jq = ps * p.nqry + h / p.Hgr;
+  if (jq >= p.nqtot) return;                 // a virtual head past the last query token
+  const size_t ooff = (size_t)b * p.q_bs + (size_t)jq * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * p.d;
   const int d = p.d, i = threadIdx.x;
   __shared__ float orot[128], osgn[128];
   __shared__ float mmax, linv;
@@ -1172,7 +1240,7 @@ struct AttPlan {
 
 // Plan of one pass over T tokens of every slice with nqry query tokens per slice (Hg = nqry x Hq/Hkv
 // virtual heads, at most 8).
-bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl, int nqry = 1) {
+bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl, int nqry = 1, int npass = 1) {
   AttParams& p = pl.p;
   p = AttParams{};
   p.B = B;
@@ -1188,7 +1256,9 @@ bool att_plan(int B, int Hq, int Hkv, int64_t T, int d, int nsm, AttPlan& pl, in
   p.G = d / 32;
   p.T = T;
   p.tstride = T;
-  p.slices = B * Hkv;
+  p.cslices = B * Hkv;
+  p.slices = npass * p.cslices;
+  p.nqtot = nqry;
   p.nchunk = (int)((T + kChunk - 1) / kChunk);
   const long long totalc = (long long)p.slices * p.nchunk;
   const int ncta = (int)std::min<long long>(nsm, totalc);
@@ -1226,10 +1296,11 @@ namespace tq {
 namespace {
 // Geometry of one attention pass: nqry query tokens per slice, q / out strides, causal limit.
 struct PassGeom {
-  int nqry;                      // query tokens per slice in this pass (1 for decode)
+  int nqry;                      // query tokens per cache slice and pass (1 for decode)
+  int npass;                     // passes in the launch (query tokens nqry * npass >= nqtot)
+  int nqtot;                     // query tokens in all
   int64_t q_bs, q_js;            // element strides of q / out: batch, query token
-  int64_t q_off;                 // element offset of the pass's first query token
-  int64_t tlim0;                 // query token j of the pass attends t < tlim0 + j
+  int64_t tlim0;                 // query token j attends t < tlim0 + j
 };
 
 // The new token of every slice for tq_attend_append (written into slot t_new by the prep kernel).
@@ -1297,16 +1368,14 @@ tq_status attend_pass(const char* f, const tq_codebook* cb_k, const tq_codebook*
   const bool ksign = k_signs != nullptr;
   const bool vsign = v_signs != nullptr;
   AttPlan pl;
-  att_plan(B, Hq, Hkv, T, d, sm_count(), pl, g.nqry);
+  att_plan(B, Hq, Hkv, T, d, sm_count(), pl, g.nqry, g.npass);
   if (ws_bytes < pl.total) return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
   AttParams& p = pl.p;
   p.tstride = tstride;
   p.q_bs = g.q_bs;
   p.q_js = g.q_js;
   p.tlim0 = g.tlim0;
-  const size_t esz = q_dtype == TQ_BF16 ? 2 : 4;
-  q = (const uint8_t*)q + (size_t)g.q_off * esz;
-  out += g.q_off;
+  p.nqtot = g.nqtot;
   int kmask[8], vmask[8];
   float kbeta[8], vbeta[8];
   p.bk = cb_k->bits;
@@ -1385,16 +1454,17 @@ tq_status attend_pass(const char* f, const tq_codebook* cb_k, const tq_codebook*
 // Query tokens per pass of a prefill: as many as keep the virtual heads at 8 or fewer.
 int prefill_qpass(int Hg) { return std::max(1, 8 / Hg); }
 
+// One launch: the passes over the cache are work slices of their own.
+PassGeom prefill_geom(int32_t Hq, int32_t Qn, int64_t T, int32_t d, int Hg) {
+  const int qp = std::min(prefill_qpass(Hg), (int)Qn);
+  return PassGeom{qp, (Qn + qp - 1) / qp, Qn, (int64_t)Qn * Hq * d, (int64_t)Hq * d, T - Qn + 1};
+}
+
 size_t prefill_ws(int32_t B, int32_t Hq, int32_t Hkv, int32_t Qn, int64_t T, int32_t d, int nsm) {
-  const int qp = prefill_qpass(Hq / Hkv);
-  size_t need = 0;
-  for (int j0 = 0; j0 < Qn; j0 += qp) {
-    const int nq = std::min(qp, Qn - j0);
-    AttPlan pl;
-    att_plan(B, Hq, Hkv, T - Qn + j0 + nq, d, nsm, pl, nq);
-    need = std::max(need, pl.total);
-  }
-  return need;
+  const PassGeom g = prefill_geom(Hq, Qn, T, d, Hq / Hkv);
+  AttPlan pl;
+  att_plan(B, Hq, Hkv, T, d, nsm, pl, g.nqry, g.npass);
+  return pl.total;
 }
 }  // namespace
 
@@ -1410,7 +1480,7 @@ tq_status attend_impl(const char* f, const tq_codebook* cb_k, const tq_codebook*
   if (st != TQ_OK) return st;
   if (ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
     return fail(TQ_ERR_WORKSPACE, std::string(f) + ": workspace too small");
-  PassGeom g{1, (int64_t)Hq * d, 0, 0, T};
+  PassGeom g{1, 1, 1, (int64_t)Hq * d, 0, T};
   return attend_pass(f, cb_k, cb_v, B, Hq, Hkv, T, tstride, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas,
                      v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g);
 }
@@ -1456,18 +1526,11 @@ extern "C" TQ_API tq_status tq_attend_prefill(const tq_codebook* cb_k, const tq_
   if (st != TQ_OK) return st;
   if (ws_bytes < tq_attend_prefill_workspace_bytes(B, Hq, Hkv, Qn, T, d))
     return fail(TQ_ERR_WORKSPACE, "tq_attend_prefill: workspace too small");
-  const int qp = prefill_qpass(Hq / Hkv);
-  for (int j0 = 0; j0 < Qn; j0 += qp) {
-    const int nq = std::min(qp, Qn - j0);
-    // query token j (0-based among the Qn new tokens) sits at cache position T - Qn + j and sees
-    // the tokens t <= T - Qn + j; the pass covers exactly the tokens its last query sees
-    const int64_t Tp = T - Qn + j0 + nq;
-    PassGeom g{nq, (int64_t)Qn * Hq * d, (int64_t)Hq * d, (int64_t)j0 * Hq * d, T - Qn + j0 + 1};
-    st = attend_pass(f, cb_k, cb_v, B, Hq, Hkv, Tp, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas, v_codes,
+  // query token j (0-based among the Qn new tokens) sits at cache position T - Qn + j and sees the
+  // tokens t <= T - Qn + j; every pass reads all T slots (a pass's last few chunks are masked)
+  const PassGeom g = prefill_geom(Hq, Qn, T, d, Hq / Hkv);
+  return attend_pass(f, cb_k, cb_v, B, Hq, Hkv, T, T, d, q, q_dtype, rot, k_codes, k_norms, k_signs, k_gammas, v_codes,
                      v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g);
-    if (st != TQ_OK) return st;
-  }
-  return TQ_OK;
 }
 
 extern "C" TQ_API size_t tq_attend_append_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t T_cur, int32_t d,
@@ -1502,7 +1565,7 @@ extern "C" TQ_API tq_status tq_attend_append(const tq_codebook* cb_k, const tq_c
   if (ws_bytes < tq_attend_workspace_bytes(B, Hq, Hkv, T, d))
     return fail(TQ_ERR_WORKSPACE, "tq_attend_append: workspace too small");
   const AppendArgs app{k_new, v_new, x_dtype, T_cur, k_codes, k_norms, v_codes, v_signs, v_norms, v_gammas};
-  PassGeom g{1, (int64_t)Hq * d, 0, 0, T};
+  PassGeom g{1, 1, 1, (int64_t)Hq * d, 0, T};
   return attend_pass(f, cb_k, cb_v, B, Hq, Hkv, T, T_max, d, q, q_dtype, rot, k_codes, k_norms, nullptr, nullptr,
                      v_codes, v_signs, v_norms, v_gammas, scale, out, ws, ws_bytes, stream, g, &app);
 }
