@@ -39,12 +39,12 @@
 // Kernels: prep (q' limbs, per-head constants), main (persistent; one CTA per SM walks a
 // contiguous range of 128-token chunks, possibly spanning several (batch, KV head) slices), combine
 // (merges the per-CTA partial states of a slice and applies Pi^T, S^T).
-// Main-kernel roles (19 warps; 23 with at most four query heads per KV head): 0 bulk-copies packed
-// chunks; 1 owns TMEM and issues the key MMAs; 2-9 softmax (thread = token; two groups of four
-// warps, each group owning half of the query heads); 10-13 expand the key planes into TMEM (thread
-// = token), and with 19 warps also the value planes into shared memory; 14-17 accumulate the value
-// products (thread = coordinate); 18 issues the value MMAs; 19-22 (23 warps) expand the value
-// planes, so that key and value expansion run side by side.
+// Main-kernel roles (19 warps): 0 bulk-copies packed chunks; 1 owns TMEM and issues the key MMAs;
+// then the softmax warps (thread = token; one group of four warps per four query heads: 2-5, or
+// 2-9 with eight heads); then four warps that expand the key planes into TMEM (thread = token), and
+// with eight heads also the value planes into shared memory; four warps that accumulate the value
+// products (thread = coordinate); one that issues the value MMAs; and with four heads, four more
+// that expand the value planes, so that key and value expansion run side by side.
 // All mbarrier waits are bounded (sm100.cuh); the softmax warps' named barriers are reached the
 // same number of times by the four warps of a group (their loop never exits early).
 #include <cuda_fp16.h>
@@ -62,7 +62,11 @@ namespace {
 // warps of the main kernel: 23 when the value planes have their own expander warps (at most four
 // query heads per KV head; 80 registers a thread), else 19 (96 registers)
 __host__ __device__ constexpr bool att_split_v(int hg) { return hg <= 4; }
-__host__ __device__ constexpr int att_warps(int hg) { return att_split_v(hg) ? 23 : 19; }
+// softmax groups of four warps: one per four query heads
+__host__ __device__ constexpr int att_groups(int hg) { return hg / 4; }
+// producer, key MMA, softmax groups, key (and value) expanders, accumulators, value MMA, and with at
+// most four query heads separate value expanders: 19 warps either way
+__host__ __device__ constexpr int att_warps(int hg) { return 2 + 4 * att_groups(hg) + 8 + 1 + (att_split_v(hg) ? 4 : 0); }
 constexpr int kChunk = 128;                 // tokens per chunk
 constexpr int kMaxStages = 8;               // packed-chunk ring (depth chosen from shared memory)
 constexpr int kMaxSmem = 232448;            // 227 KB of dynamic shared memory per block
@@ -499,11 +503,16 @@ __device__ __forceinline__ void expand_v_rows(const AttParams& p, const AttLayou
 
 // HG: query heads per KV head (4 or 8, Hg <= HG); BK: key codebook bits; BV: value codebook bits;
 // VS: value sign plane (Algorithm 2 values); KS: key sign plane (Algorithm 2 keys, BK <= 2)
-// Register cap: the most that fits the warps an SM sub-partition holds (16384 registers each; 6 of
-// the 23 warps, or 5 of the 19, in units of 8 registers a thread).
+// Register cap: the most that fits the warps an SM sub-partition holds (16384 registers each, 5 of
+// the 19 warps, in units of 8 registers a thread).
 template <int HG, int BK, int BV, int VS, int KS>
-__global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const __grid_constant__ AttParams p) {
+__global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttParams p) {
+  static_assert(att_warps(HG) == 19, "the register cap assumes 19 warps");
   constexpr bool SPLITV = att_split_v(HG);
+  constexpr int NG = att_groups(HG);             // softmax groups
+  constexpr int W_EXP = 2 + 4 * NG;              // first key expander warp
+  constexpr int W_ACC = W_EXP + 4;               // first accumulator warp
+  constexpr int W_VMMA = W_ACC + 4;              // value MMA warp (then the value expanders)
   constexpr int MK = walsh_count(BK);
   constexpr int MKT = MK + KS;                   // key operand planes (Walsh planes, sign plane)
   constexpr int MV = walsh_count(BV);
@@ -514,6 +523,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   constexpr int NQ = HG <= 4 ? 16 : 32;
   constexpr int NQS = NQ * (1 + KS);            // score columns: Walsh part, then (KS) sign part
   constexpr int KSTEPS = MK * 128 / 32;          // K steps of the Walsh planes (the sign plane adds 4)
+  // The chunk's fp16 norms ride with the key planes through TMEM (the key expanders store them, the
+  // softmax warps load them with the scores): 4 buffers of 2 columns after the value products,
+  // where they fit; else the softmax warps read them from the stage.
+  constexpr uint32_t kNR0 = 2 * 32 * MKT + 2 * NQS + 2 * (MV + VS) * NQ;
+  constexpr bool NT = kNR0 + 8 <= 512;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nst = p.nst;
@@ -538,21 +552,22 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&bar[ST_FULL + s], 1);
-      mbar_init(&bar[ST_EMPTY + s], (SPLITV ? 8 : 4) + 8);   // key (and value) expanders, softmax
+      mbar_init(&bar[ST_EMPTY + s], (SPLITV ? 8 : 4) + (NT ? 0 : 4 * NG));   // key (and value) expanders, softmax
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[BQ_FULL + s], 1);
       mbar_init(&bar[BQ_EMPTY + s], 1);
       mbar_init(&bar[AK_FULL + s], 4);
       mbar_init(&bar[SC_DONE + s], 1);
-      mbar_init(&bar[BW_FULL + s], 8);
+      mbar_init(&bar[BW_FULL + s], 4 * NG);
       mbar_init(&bar[RUN_DONE + s], 2);
       mbar_init(&bar[RUN_FREE + s], 4);
-      mbar_init(&bar[SC_FREE + s], 8);
+      mbar_init(&bar[SC_FREE + s], 4 * NG);
     }
     for (int s = 0; s < 3; ++s) mbar_init(&bar[AV_FULL + s], 4);
     for (int s = 0; s < 6; ++s) mbar_init(&bar[V_DONE + s], 1);
     *abort_flag = 0;
+    for (int s = 0; s < 4; ++s) ((int*)(scal + s * 64))[40] = ((int*)(scal + s * 64))[41] = -1;   // no chunk yet
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -626,7 +641,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (!mbar_wait_warp(&bar[BQ_FULL + (sg & 1)], (sg >> 1) & 1, p.err, kDevTimeoutLoad, abort_flag)) break;
       }
       if (!mbar_wait_warp(&bar[AK_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
-      // the scores buffer b is free once the softmax warps have read the scores of chunk c-2
+      // the scores buffer b is free once the softmax warps finished chunk c-2 (the whole chunk: the
+      // key expanders of chunk c+2, which follow these MMAs, reuse the norm columns of chunk c-2)
       if (c >= 2 && !mbar_wait_warp(&bar[BW_FULL + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutSync, abort_flag))
         break;
       tc_fence_after();
@@ -648,11 +664,11 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       }
       __syncwarp();
     }
-  } else if (warp < 10) {
+  } else if (warp < W_EXP) {
     // ------------------------------------ softmax warps (thread = token) ---------------------------
-    // group gq of four warps owns query heads [h0, h0 + HH); both groups track the same value-norm
-    // maxima (same tokens, same rule), so the fixed-point scales agree
-    constexpr int HH = HG / 2;
+    // group gq of four warps owns query heads [h0, h0 + HH); with two groups both track the same
+    // value-norm maxima (same tokens, same rule), so the fixed-point scales agree
+    constexpr int HH = HG / NG;
     const int q = warp & 3;
     const int gq = (warp - 2) >> 2;
     const int h0 = gq * HH;
@@ -669,16 +685,17 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     // four segments later, after the value MMA warp has read it)
     float lt[HH];
     float* segl = (float*)(smem + Lo.off_sum);      // [slot][warp][head]
-    // fp16 norms of the chunk's tokens: from the stage (bulk-copied with the codes) where possible,
-    // else from global memory (dead tokens read as zero)
     RingPos rs{0, nst, 0u};
     for (int c = 0; c < nmy; ++c, it.next(), rs.next()) {     // no early exit: the named barriers must match
       const int b = c & 1;
       const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
       const bool live = t < tc;
       uint16_t nk_n = 0, nv_n = 0, gm_n = 0, gk_n = 0;
-      ok = mbar_wait_warp(&bar[ST_FULL + rs.slot], rs.par, p.err, kDevTimeoutLoad, abort_flag) && ok;
-      if (p.norm_bulk && t < (tc & ~7)) {
+      // fp16 norms of the chunk's tokens: with the scores (TMEM), else from the stage (bulk-copied
+      // with the codes) where possible, else from global memory (dead tokens read as zero)
+      if (!NT) ok = mbar_wait_warp(&bar[ST_FULL + rs.slot], rs.par, p.err, kDevTimeoutLoad, abort_flag) && ok;
+      if (NT) {
+      } else if (p.norm_bulk && t < (tc & ~7)) {
         const uint16_t* sn = (const uint16_t*)(smem + Lo.off_stage + rs.slot * Lo.stage_bytes + Lo.nrm_off);
         nk_n = sn[t];
         nv_n = sn[kChunk + t];
@@ -691,11 +708,10 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (VS) gm_n = __ldg(p.v_gammas + rec);
         if (KS) gk_n = __ldg(p.k_gammas + rec);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[ST_EMPTY + rs.slot]);   // done with the stage
-      const float nk = __half2float(__ushort_as_half(nk_n)), nv = __half2float(__ushort_as_half(nv_n));
-      const float gm = VS ? __half2float(__ushort_as_half(gm_n)) : 0.0f;
-      const float gk = KS ? __half2float(__ushort_as_half(gk_n)) : 0.0f;
+      if (!NT) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[ST_EMPTY + rs.slot]);   // done with the stage
+      }
       if (c == 0 || it.cis == 0) {
         vmax_run = gmax_run = 0.0f;
         const float4* hc = (const float4*)(p.head_c + it.slice * 32);
@@ -725,7 +741,18 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (HH == 2) tmem_ld8(scol + NQ, *(uint32_t(*)[8]) & dzr[0]);
         else tmem_ld16(scol + NQ, *(uint32_t(*)[16]) & dzr[0]);
       }
+      uint32_t nrw[2];
+      if (NT) tmem_ld2(tbase + lane_base + kNR0 + (c & 3) * 2, nrw);
       tmem_ld_wait();
+      if (NT) {
+        nk_n = (uint16_t)(nrw[0] & 0xFFFFu);
+        nv_n = (uint16_t)(nrw[0] >> 16);
+        gm_n = (uint16_t)(nrw[1] & 0xFFFFu);
+        gk_n = (uint16_t)(nrw[1] >> 16);
+      }
+      const float nk = __half2float(__ushort_as_half(nk_n)), nv = __half2float(__ushort_as_half(nv_n));
+      const float gm = VS ? __half2float(__ushort_as_half(gm_n)) : 0.0f;
+      const float gk = KS ? __half2float(__ushort_as_half(gk_n)) : 0.0f;
       tc_fence_before();
       float lg[HH];
       bool up = nv > vmax_run || nv * gm > gmax_run;
@@ -792,8 +819,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         wz[i] = VS ? fixed24(w * gm, sw2) : 0u;
         lt[i] = fmaf(lt[i], corr[i], pr);
       }
-      // the weight tiles of chunk c-2 (same buffer) must have been consumed by its value MMA
-      if (c >= 2) ok = mbar_wait_warp(&bar[V_DONE + (c - 2) % 6], ((c - 2) / 6) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
+      if (c >= 2)
+        ok = mbar_wait_warp(&bar[V_DONE + (c - 2) % 6], ((c - 2) / 6) & 1, p.err, kDevTimeoutMma, abort_flag) && ok;
       if (c == nmy - 1 || it.cis == p.nchunk - 1) {
         // the segment ends with this chunk: the group's sums of p of its heads
         float* lp = segl + ((it.seg & 3) * 4 + q) * 8;
@@ -816,23 +843,21 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
           *(uint4*)(bwb + Lo.bw_kind) = make_uint4(wz[0], wz[HH > 1 ? 1 : 0], wz[HH > 2 ? 2 : 0], wz[HH > 3 ? 3 : 0]);
       }
       fence_proxy_async_smem();
-      if (q == 0 && lane == 0) {
-        // chunk scalars for the value MMA warp (4-deep ring): running maxima, scales, and whether this
-        // group's maxima or scales moved (the chunk then starts a new run)
+      if (q == 0 && lane == 0 && (changed || c == 0 || it.cis == 0)) {
+        // where this group's maxima or scales moved (or a segment starts), the chunk starts a new run:
+        // its scalars for the value MMA warp (4-deep ring), stamped with the chunk
         float* sc = scal + (c & 3) * 64;
 #pragma unroll
         for (int i = 0; i < HH; ++i) sc[16 + h0 + i] = mrun[i];
-        if (gq == 0) {
-          sc[32] = isw;
-          sc[33] = isw2;
-        }
-        sc[34 + gq] = changed ? 1.0f : 0.0f;
+        sc[32 + 2 * gq] = isw;
+        sc[33 + 2 * gq] = isw2;
+        ((int*)sc)[40 + gq] = c;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[BW_FULL + b]);
     }
     (void)ok;
-  } else if (warp < 14) {
+  } else if (warp < W_ACC) {
     // ------------------------------------ expanders (thread = token) -------------------------------
     const int q = warp & 3;
     const int t = q * 32 + lane;
@@ -844,7 +869,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       voff[2 * g + 1] = sw128_offset(t, g * 32 + 16, 128);
     }
     RingPos rs{0, nst, 0u};
-    for (int c = 0; c < nmy; ++c, rs.next()) {
+    for (int c = 0; c < nmy; ++c, rs.next(), it.next()) {
       const int st = rs.slot, b = c & 1;
       if (!mbar_wait_warp(&bar[ST_FULL + st], rs.par, p.err, kDevTimeoutLoad, abort_flag)) break;
       if (c >= 2 && !mbar_wait_warp(&bar[SC_DONE + b], ((c - 2) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag))
@@ -889,7 +914,24 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
           tmem_st8(ak + MK * 32 + g * 8, r);
         }
       }
-      // the key planes are complete once this warp's TMEM stores are
+      if (NT) {
+        // the token's fp16 norms for the softmax warps: (key norm | value norm << 16), (value gamma |
+        // key gamma << 16), in buffer c % 4 (free: the key MMAs of chunk c-2, which this warp waited
+        // for, followed the softmax of chunk c-4)
+        const int tc = it.cis == p.nchunk - 1 ? tail : kChunk;
+        uint32_t nr[2] = {0u, 0u};
+        if (p.norm_bulk && t < (tc & ~7)) {
+          const uint16_t* sn = (const uint16_t*)(stg + Lo.nrm_off);
+          nr[0] = (uint32_t)sn[t] | ((uint32_t)sn[kChunk + t] << 16);
+          nr[1] = (VS ? (uint32_t)sn[2 * kChunk + t] : 0u) | (KS ? (uint32_t)sn[3 * kChunk + t] << 16 : 0u);
+        } else if (t < tc) {
+          const int64_t rec = (int64_t)it.cs * TS + (int64_t)it.cis * kChunk + t;
+          nr[0] = (uint32_t)__ldg(p.k_norms + rec) | ((uint32_t)__ldg(p.v_norms + rec) << 16);
+          nr[1] = (VS ? (uint32_t)__ldg(p.v_gammas + rec) : 0u) | (KS ? (uint32_t)__ldg(p.k_gammas + rec) << 16 : 0u);
+        }
+        tmem_st2(tbase + lane_base + kNR0 + (c & 3) * 2, nr);
+      }
+      // the key planes (and norms) are complete once this warp's TMEM stores are
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -912,7 +954,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         mbar_arrive(&bar[ST_EMPTY + st]);
       }
     }
-  } else if (warp < 18) {
+  } else if (warp < W_VMMA) {
     // ------------------------------------ accumulators (thread = coordinate row) -------------------
     // One pass per run: the run's limb sums from TMEM and its exact weight sums are folded in int64,
     //   O_P = 2^s W - 2 Y_P (Walsh planes),  O_z = 2 Y_z - 2^s W' (sign plane),
@@ -999,8 +1041,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       }
       if (flags & 2) break;
     }
-  } else if (warp == 18) {
-    // ------------------------------------ value MMA issuer (warp 18) ------------------------------
+  } else if (warp == W_VMMA) {
+    // ------------------------------------ value MMA issuer ------------------------------------------
     // Runs beside the key MMA warp so that neither warp's barrier waits and commits sit behind the
     // other's tensor-core work. Warp-uniform schedule, one elected lane issues. It also keeps the
     // runs: a chunk whose softmax scalars moved starts a new run in the other TMEM buffer. The warp
@@ -1010,6 +1052,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
     const uint64_t db0 = desc_smem(smem_u32(smem + Lo.off_bw), 128, kChunk * 16, 0);
     int R = -1, runlen = 0;
     bool open = false;
+    float cur_sc = 0.0f;                         // lane < 10: scalar `lane` of the current run
     // this lane's share of the run's weight sums (tokens lane + 32 j of every chunk; below 2^33)
     unsigned long long aw[HG], az[VS ? HG : 1];
     const float* segl = (const float*)(smem + Lo.off_sum);
@@ -1047,7 +1090,8 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       if (!mbar_wait_warp(&bar[BW_FULL + b], (c >> 1) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
       if (!mbar_wait_warp(&bar[AV_FULL + c3], (c / 3) & 1, p.err, kDevTimeoutSync, abort_flag)) break;
       const float* sc = scal + (c & 3) * 64;
-      const bool newrun = !open || sc[34] != 0.0f || sc[35] != 0.0f || runlen == kMaxRun;
+      const bool st0 = ((const int*)sc)[40] == c, st1 = NG > 1 && ((const int*)sc)[41] == c;
+      const bool newrun = !open || st0 || st1 || runlen == kMaxRun;
       if (newrun) {
         if (open) close_run(0, 0);
         ++R;
@@ -1061,7 +1105,13 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
         if (R >= 2 && !mbar_wait_warp(&bar[RUN_FREE + (R & 1)], ((R >> 1) - 1) & 1, p.err, kDevTimeoutSync, abort_flag))
           break;
         uint8_t* rr = smem + Lo.off_run + (R & 1) * kRunRec;
-        if (lane < 10) ((float*)rr)[lane] = lane < 8 ? sc[16 + lane] : sc[32 + lane - 8];
+        // lanes 0..9 keep the run's scalars (8 maxima, 1/sw, 1/sw'), from the stamped groups
+        if (lane < 8) {
+          if ((lane / (HG / NG) == 0 ? st0 : st1)) cur_sc = sc[16 + lane];
+        } else if (lane < 10) {
+          if (st0 || st1) cur_sc = sc[32 + (st0 ? 0 : 2) + lane - 8];
+        }
+        if (lane < 10) ((float*)rr)[lane] = cur_sc;
         if (lane == 10) *(int*)(rr + 48) = it.slice;
         open = true;
       }
@@ -1111,7 +1161,7 @@ __global__ void __maxnreg__(att_split_v(HG) ? 80 : 96) attend_main_kernel(const 
       }
     }
   } else if (SPLITV) {
-    // ------------------------------------ value expanders (warps 19-22, thread = token) -----------
+    // ------------------------------------ value expanders (last four warps, thread = token) -------
     const int q = warp & 3;
     const int t = q * 32 + lane;
     uint32_t voff[8];                               // this token's 16-byte slots in a value plane
