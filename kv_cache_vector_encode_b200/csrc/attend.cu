@@ -193,7 +193,12 @@ __device__ void append_encode(const AttParams& p, int slice, const void* xsrc, b
 // ------------------------------------------------------------------------------------------------
 // prep: q' = Pi q per query head, fixed-point limbs of beta_S q' (scaled by 2^-s), constants
 // ------------------------------------------------------------------------------------------------
+constexpr int kPrepRow = 129;                   // staged matrix row (floats): row reads hit distinct banks
+size_t prep_smem_bytes(int ksign) { return (size_t)(ksign ? 2 : 1) * 128 * kPrepRow * sizeof(float); }
+
 __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
+  extern __shared__ float prep_mat[];           // Pi, then S (Algorithm 2 keys): [128][kPrepRow]
+  grid_dep_launch();                            // the main kernel may be scheduled (it waits for this grid)
   const int slice = blockIdx.x;                  // work slice: pass * cslices + b * Hkv + hk
   const int cs = slice % p.cslices, ps = slice / p.cslices;
   const int b = cs / p.Hkv, hk = cs % p.Hkv;
@@ -219,32 +224,40 @@ __global__ void attend_prep_kernel(const __grid_constant__ AttParams p) {
                             : (p.q_bf16 ? __uint_as_float((uint32_t)((const uint16_t*)p.q)[qoff + i] << 16)
                                         : ((const float*)p.q)[qoff + i]);
   }
+  // Pi (and S) into shared memory: coalesced 16-byte loads, all in flight at once, stored into
+  // padded rows
+  for (int mtx = 0; mtx < (p.ksign ? 2 : 1); ++mtx) {
+    const float4* src = (const float4*)(mtx ? p.S : p.Pi);
+    float* dst = prep_mat + mtx * 128 * kPrepRow;
+#pragma unroll 8
+    for (int o = i; o < 128 * 32; o += 128) {
+      const float4 v = __ldg(src + o);
+      float* q = dst + (o >> 5) * kPrepRow + (o & 31) * 4;
+      q[0] = v.x;
+      q[1] = v.y;
+      q[2] = v.z;
+      q[3] = v.w;
+    }
+  }
   __syncthreads();
   // q'_h[i] = sum_j Pi[i][j] q_h[j] for every head: one thread per output coordinate, its row of Pi
-  // read as float4, fp64 accumulation (one independent chain per head)
+  // from shared memory, fp64 accumulation (one independent chain per head)
   // (q''_h = S q_h the same way, for Algorithm 2 keys)
   double acc[8], acc2[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) acc[h] = acc2[h] = 0.0;
-  const float4* row = (const float4*)(p.Pi + (size_t)i * d);
-  const float4* srow = (const float4*)(p.S + (size_t)i * d);
-  for (int j4 = 0; j4 < d / 4; ++j4) {
-    const float4 pv = __ldg(row + j4);
-    const float4 sv = p.ksign ? __ldg(srow + j4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const float* row = prep_mat + i * kPrepRow;
+  const float* srow = prep_mat + 128 * kPrepRow + i * kPrepRow;
+#pragma unroll 4
+  for (int j = 0; j < 128; ++j) {
+    const double pv = (double)row[j];
+    const double sv = p.ksign ? (double)srow[j] : 0.0;
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       if (h < p.Hg) {
-        const float4 qv = *(const float4*)&sq[h][4 * j4];
-        acc[h] = fma((double)pv.x, (double)qv.x, acc[h]);
-        acc[h] = fma((double)pv.y, (double)qv.y, acc[h]);
-        acc[h] = fma((double)pv.z, (double)qv.z, acc[h]);
-        acc[h] = fma((double)pv.w, (double)qv.w, acc[h]);
-        if (p.ksign) {
-          acc2[h] = fma((double)sv.x, (double)qv.x, acc2[h]);
-          acc2[h] = fma((double)sv.y, (double)qv.y, acc2[h]);
-          acc2[h] = fma((double)sv.z, (double)qv.z, acc2[h]);
-          acc2[h] = fma((double)sv.w, (double)qv.w, acc2[h]);
-        }
+        const double qv = (double)sq[h][j];
+        acc[h] = fma(pv, qv, acc[h]);
+        if (p.ksign) acc2[h] = fma(sv, qv, acc2[h]);
       }
     }
   }
@@ -577,6 +590,10 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched as a dependent of the prep kernel: its query images, constants (and appended records)
+  // are read only after this; the combine kernel may in turn be scheduled from here on
+  grid_dep_wait();
+  grid_dep_launch();
   const uint32_t tbase = *tmem_slot;
 
   ChunkIter it;
@@ -1199,24 +1216,33 @@ __global__ void __maxnreg__(96) attend_main_kernel(const __grid_constant__ AttPa
 // ------------------------------------------------------------------------------------------------
 // combine: merge the partial states of a slice, apply Pi^T and alpha S^T once per query head
 // ------------------------------------------------------------------------------------------------
+size_t combine_smem_bytes(int vsign) { return (size_t)(vsign ? 2 : 1) * 128 * 128 * sizeof(float); }
+
 __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
-  const int slice = blockIdx.x / p.Hg;       // one block per (work slice, virtual head)
-  const int h = blockIdx.x % p.Hg;
+  const int slice = blockIdx.x;              // one block per work slice, all its virtual heads
   const int cs = slice % p.cslices, ps = slice / p.cslices;
   const int b = cs / p.Hkv, hk = cs % p.Hkv;
-  const int jq = ps * p.nqry + h / p.Hgr;
-  if (jq >= p.nqtot) return;                 // a virtual head past the last query token
-  const size_t ooff = (size_t)b * p.q_bs + (size_t)jq * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * p.d;
-  const int d = p.d, i = threadIdx.x;
-  __shared__ float orot[128], osgn[128];
-  __shared__ float mmax, linv;
+  const int d = p.d, i = threadIdx.x, Hg = p.Hg;
+  extern __shared__ float cmb_mat[];         // Pi, then S (Algorithm 2 values): [128][128]
+  __shared__ float orot[8][128], osgn[8][128];
+  __shared__ float mmax[8], linv[8];
+  // Pi (and S) into shared memory (coalesced 16-byte copies, all in flight at once); column j of
+  // Pi^T is row j of Pi, read across the threads without bank conflicts
+  for (int mtx = 0; mtx < (p.vsign ? 2 : 1); ++mtx) {
+    const float4* src = (const float4*)(mtx ? p.S : p.Pi);
+    float4* dst = (float4*)(cmb_mat + mtx * 128 * 128);
+#pragma unroll 8
+    for (int o = i; o < 128 * 32; o += 128) dst[o] = __ldg(src + o);
+  }
+  grid_dep_wait();                           // the main kernel's partial states
   // CTAs that touched this slice
   const int first = (slice * p.nchunk) / p.per_cta;
   const int last = (slice * p.nchunk + p.nchunk - 1) / p.per_cta;
   const int nseg = last - first + 1;
-  const float* base = p.partial + (size_t)slice * p.maxseg * p.Hg * att_rec(d) + (size_t)h * att_rec(d);
-  const size_t stride = (size_t)p.Hg * att_rec(d);
-  if (i == 0) {
+  const float* base0 = p.partial + (size_t)slice * p.maxseg * Hg * att_rec(d);
+  const size_t stride = (size_t)Hg * att_rec(d);
+  if (i < Hg) {
+    const float* base = base0 + (size_t)i * att_rec(d);
     float M = -INFINITY;
     for (int sgi = 0; sgi < nseg; ++sgi) M = fmaxf(M, base[sgi * stride]);
     float L = 0.0f;
@@ -1224,44 +1250,49 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttParams p) {
       const float ms = base[sgi * stride];
       if (ms > -INFINITY) L += base[sgi * stride + 1] * exp2f(ms - M);
     }
-    mmax = M;
-    linv = L > 0.0f ? 1.0f / L : 0.0f;
+    mmax[i] = M;
+    linv[i] = L > 0.0f ? 1.0f / L : 0.0f;
   }
   __syncthreads();
-  if (i < d) {
+  for (int h = 0; h < Hg; ++h) {
+    const float* base = base0 + (size_t)h * att_rec(d);
     float y[3] = {0.0f, 0.0f, 0.0f};
     for (int sgi = 0; sgi < nseg; ++sgi) {
       const float ms = base[sgi * stride];
       if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - mmax);
+      const float f = exp2f(ms - mmax[h]);
       for (int P = 0; P < p.np; ++P) y[P] = fmaf(base[sgi * stride + 4 + P * d + i], f, y[P]);
     }
     float a = 0.0f;
     for (int P = 0; P < p.mv; ++P) a = fmaf(p.beta_v[P], y[P], a);
-    orot[i] = a * linv;
-    osgn[i] = p.vsign ? y[p.np - 1] * linv : 0.0f;
+    orot[h][i] = a * linv[h];
+    osgn[h][i] = p.vsign ? y[p.np - 1] * linv[h] : 0.0f;
   }
   __syncthreads();
-  if (i < d) {
-    // four independent partial sums per product (the loads of a column of Pi / S are coalesced
-    // across the threads)
-    float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
-    for (int j = 0; j < d; j += 4) {
+  // out_h[i] = sum_j Pi[j][i] orot_h[j] + alpha sum_j S[j][i] osgn_h[j]
+  float acc[8], z[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) a[u] = fmaf(__ldg(p.Pi + (size_t)(j + u) * d + i), orot[j + u], a[u]);
-    }
-    float acc = (a[0] + a[1]) + (a[2] + a[3]);
-    if (p.vsign) {
-      float z[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int h = 0; h < 8; ++h) acc[h] = z[h] = 0.0f;
+  const float* scol = cmb_mat + 128 * 128;
 #pragma unroll 4
-      for (int j = 0; j < d; j += 4) {
+  for (int j = 0; j < 128; ++j) {
+    const float pj = cmb_mat[j * 128 + i];
+    const float sj = p.vsign ? scol[j * 128 + i] : 0.0f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) z[u] = fmaf(__ldg(p.S + (size_t)(j + u) * d + i), osgn[j + u], z[u]);
+    for (int h = 0; h < 8; ++h) {
+      if (h < Hg) {
+        acc[h] = fmaf(pj, orot[h][j], acc[h]);
+        if (p.vsign) z[h] = fmaf(sj, osgn[h][j], z[h]);
       }
-      acc = fmaf(p.alpha, (z[0] + z[1]) + (z[2] + z[3]), acc);
     }
-    p.out[ooff + i] = acc;
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    if (h >= Hg) break;
+    const int jq = ps * p.nqry + h / p.Hgr;
+    if (jq >= p.nqtot) continue;               // a virtual head past the last query token
+    const size_t ooff = (size_t)b * p.q_bs + (size_t)jq * p.q_js + (size_t)(hk * p.Hgr + h % p.Hgr) * d;
+    p.out[ooff + i] = p.vsign ? fmaf(p.alpha, z[h], acc[h]) : acc[h];
   }
 }
 
@@ -1488,16 +1519,37 @@ tq_status attend_pass(const char* f, const tq_codebook* cb_k, const tq_codebook*
   p.nst = nst;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  attend_prep_kernel<<<p.slices, 128, 0, st>>>(p);
+  const size_t prep_sm = prep_smem_bytes(p.ksign), cmb_sm = combine_smem_bytes(p.vsign);
+  e = cudaFuncSetAttribute(attend_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_sm);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cmb_sm);
+  if (e != cudaSuccess) return cuda_fail(e, (std::string(f) + ": shared memory attribute").c_str());
+  attend_prep_kernel<<<p.slices, 128, prep_sm, st>>>(p);
   const AttLayout Lo = att_layout(p, nst);
   const MainKernel kern = pick_main(p.Hg, p.bk, p.bv, p.vsign, p.ksign);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, (std::string(f) + ": shared memory attribute").c_str());
   const long long totalc = (long long)p.slices * p.nchunk;
   const int grid = (int)((totalc + p.per_cta - 1) / p.per_cta);
-  kern<<<grid, 32 * att_warps(p.Hg <= 4 ? 4 : 8), Lo.total, st>>>(p);
-  attend_combine_kernel<<<p.slices * p.Hg, 128, 0, st>>>(p);
+  // main and combine are launched as programmatic dependents of the kernel before them: their
+  // launch and set-up overlap its tail, and each waits (griddepcontrol) before reading its results
+  cudaLaunchAttribute dep[1];
+  dep[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  dep[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(32 * att_warps(p.Hg <= 4 ? 4 : 8));
+  cfg.dynamicSmemBytes = Lo.total;
+  cfg.stream = st;
+  cfg.attrs = dep;
+  cfg.numAttrs = 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, (std::string(f) + ": launch").c_str());
+  if ((e = cudaLaunchKernelEx(&cfg, kern, p)) != cudaSuccess) return cuda_fail(e, (std::string(f) + ": launch").c_str());
+  cfg.gridDim = dim3(p.slices);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = cmb_sm;
+  if ((e = cudaLaunchKernelEx(&cfg, attend_combine_kernel, p)) != cudaSuccess)
+    return cuda_fail(e, (std::string(f) + ": launch").c_str());
   return TQ_OK;
 }
 

@@ -288,6 +288,12 @@ __device__ __forceinline__ void tmem_st2(uint32_t taddr, const uint32_t (&r)[2])
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- programmatic dependent launch -------------------------------------------------------------
+// wait: every read of the previous kernel's results follows it (a no-op when the kernel was not
+// launched as a dependent); launch: lets the next kernel, launched as a dependent, start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- named barriers ---------------------------------------------------------------------------
 // Only for groups of warps that all execute the same sequence of these barriers (no early exit).
 
