@@ -550,15 +550,18 @@ def run_ours(args):
     att_bytes = B_ATT_TOKEN_HEAD * ATT_B * ATT_HKV * ATT_T + ATT_B * ATT_HQ * D * (2 + 4)
     att_gbs = att_bytes / (parts["attend"] * 1e-3) / 1e9
     # DRAM bytes of one launch from the committed ncu capture, only while the kernel source is the
-    # one that was captured (its sha256 is recorded beside the figure)
+    # one that was captured (the sha256 of attend.cu + sm100.cuh is recorded beside the figure)
     traffic = None
     prof = os.path.join(ROOT, "profiles", "attend_main_decode_attention_traffic.json")
     if os.path.exists(prof):
         try:
             rec = json.load(open(prof))
             import hashlib
-            with open(os.path.join(ROOT, "kv_cache_vector_encode_b200", "csrc", "attend.cu"), "rb") as f:
-                cur = hashlib.sha256(f.read()).hexdigest()
+            h = hashlib.sha256()
+            for src in ("attend.cu", "sm100.cuh"):
+                with open(os.path.join(ROOT, "kv_cache_vector_encode_b200", "csrc", src), "rb") as f:
+                    h.update(f.read())
+            cur = h.hexdigest()
             if rec.get("source_sha256") == cur:
                 traffic = rec.get("dram_bytes_per_launch")
         except Exception:
