@@ -278,19 +278,24 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
       uint8_t* raw = smem + raw_off(s);
       double ss = 0.0;
       if (!F32) {
+        // four independent fp64 partial sums (one per 32-bit word of a 16-byte chunk), so the
+        // sum of squares is not one long chain of dependent FMAs
         const int cpp = (KP / 8) / TPV;   // 16-byte chunks (8 values) per thread
+        double s4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
         for (int c = part * cpp; c < (part + 1) * cpp; ++c) {
           const uint4 w = *(const uint4*)(raw + sw128_offset(v, c * 16, NV));
-          auto acc = [&](uint32_t u) {
+          auto acc = [&](double& a, uint32_t u) {
             const double lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xFFFF0000u);
-            ss = fma(lo, lo, ss);
-            ss = fma(hi, hi, ss);
+            a = fma(lo, lo, a);
+            a = fma(hi, hi, a);
           };
-          acc(w.x);
-          acc(w.y);
-          acc(w.z);
-          acc(w.w);
+          acc(s4[0], w.x);
+          acc(s4[1], w.y);
+          acc(s4[2], w.z);
+          acc(s4[3], w.w);
         }
+        ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       } else {
         const int nch = (d + 3) / 4;            // 16-byte chunks of 4 floats actually holding data
         const int cpp = (nch + TPV - 1) / TPV;
@@ -388,135 +393,182 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
     };
     uint8_t* rho_hi = ALG2 ? smem + Lo.off_rho[0] : nullptr;
     uint8_t* rho_lo = ALG2 ? smem + Lo.off_rho[1] : nullptr;
-    for (int k = 0; k < my_tiles; ++k) {
+    // Algorithm 2 runs the epilogue one tile behind for the signs: tile k is quantised and its rho
+    // kept in registers while the T rho products of tile k-1 finish; then the signs of tile k-1 are
+    // read, and only then is rho of tile k stored (the rho buffer is free once those products are
+    // done) and handed to the T rho issuer. One extra pass finishes the last tile's signs.
+    constexpr int NB = NV / 32, NB_UNROLL = ALG2 ? NV / 32 : 1;
+    int64_t v0p = 0;
+    int rowsp = 0;
+    for (int k = 0; k < my_tiles + (ALG2 ? 1 : 0); ++k) {
+      const bool has_tile = k < my_tiles;
       const int a = k & 1;
       const int64_t v0 = (int64_t)(blockIdx.x + k * gridDim.x) * NV;
-      const int rows = (int)min((int64_t)NV, p.n - v0);
-      if (!mbar_wait_warp(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t dhi = tbase + lane_base + a * COLS, dlo = dhi + NV;
-      for (int c0 = cbeg; c0 < cend; c0 += 16) {
-        uint32_t hi[16], lo[16];
-        tmem_ld16(dhi + c0, hi);
-        tmem_ld16(dlo + c0, lo);
-        tmem_ld_wait();
-        uint32_t myw[BMAX];
+      const int rows = has_tile ? (int)min((int64_t)NV, p.n - v0) : 0;
+      uint32_t rhw[NV / 32][8], rlw[NV / 32][8];   // NV = 64: fp16 words of rho 2^14 per batch
+      __half rhs[16], rls[16];                                       // NV = 32: one half per vector
+      if (has_tile) {
+        if (!mbar_wait_warp(&bar[ACC_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dhi = tbase + lane_base + a * COLS, dlo = dhi + NV;
+        // batches of 16 vectors inside this warp's half (unrolled with Algorithm 2, whose rho of
+        // each batch stays in registers)
+#pragma unroll NB_UNROLL
+        for (int bt = 0; bt < NB; ++bt) {
+          const int c0 = cbeg + 16 * bt;
+          uint32_t hi[16], lo[16];
+          tmem_ld16(dhi + c0, hi);
+          tmem_ld16(dlo + c0, lo);
+          tmem_ld_wait();
+          uint32_t myw[BMAX];
 #pragma unroll
-        for (int pl = 0; pl < BMAX; ++pl) myw[pl] = 0u;
-        float r2[16];                       // rho * 2^14 of the 16 vectors (Algorithm 2)
+          for (int pl = 0; pl < BMAX; ++pl) myw[pl] = 0u;
+          float r2[16];                       // rho * 2^14 of the 16 vectors (Algorithm 2)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int v = c0 + j;
-          const float inv = info[a * NV + v];
-          const float y = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j])) * inv;
-          const bool neg = !(y > 0.0f);
-          const int m = MIX ? sym_m_rt(fabsf(y), P, gbw) : sym_m<BMAX>(fabsf(y), P);
+          for (int j = 0; j < 16; ++j) {
+            const int v = c0 + j;
+            const float inv = info[a * NV + v];
+            const float y = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j])) * inv;
+            const bool neg = !(y > 0.0f);
+            const int m = MIX ? sym_m_rt(fabsf(y), P, gbw) : sym_m<BMAX>(fabsf(y), P);
 #pragma unroll
-          for (int pl = 0; pl < BMAX; ++pl) {
-            if (MIX && pl >= gbw) break;            // warp-uniform
-            const bool bit = pl == gbw - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
-            const uint32_t w = __ballot_sync(0xffffffffu, active && bit);
-            if (lane == j) myw[pl] = w;
-          }
-          if (ALG2) {
-            const float cm = sym_c<BMAX>(m, C);
-            float rho = neg ? y + cm : y - cm;
-            if (!active || inv == 0.0f) rho = 0.0f;
-            if (NV == 64) {
-              r2[j] = rho * kRhoScale;            // stored below, two vectors per word
-            } else {
-              // K-major rho (32-vector tiles): one fp16 per (vector row, coordinate)
-              r2[j] = rho * rho;
-              const float rs = rho * kRhoScale;
-              const __half rh = __float2half_rn(rs);
-              const __half rl = __float2half_rn((rs - __half2float(rh)) * kSplitScale);
-              if (i < KP) {
-                const uint32_t off = sw128_offset(v, 2 * i, NV);
-                *(__half*)(rho_hi + off) = rh;
-                *(__half*)(rho_lo + off) = rl;
+            for (int pl = 0; pl < BMAX; ++pl) {
+              if (MIX && pl >= gbw) break;            // warp-uniform
+              const bool bit = pl == gbw - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
+              const uint32_t w = __ballot_sync(0xffffffffu, active && bit);
+              if (lane == j) myw[pl] = w;
+            }
+            if (ALG2) {
+              const float cm = sym_c<BMAX>(m, C);
+              float rho = neg ? y + cm : y - cm;
+              if (!active || inv == 0.0f) rho = 0.0f;
+              if (NV == 64) {
+                r2[j] = rho * kRhoScale;            // packed below, two vectors per word
+              } else {
+                // K-major rho (32-vector tiles): one fp16 per (vector row, coordinate), kept
+                r2[j] = rho * rho;
+                const float rs = rho * kRhoScale;
+                rhs[j] = __float2half_rn(rs);
+                rls[j] = __float2half_rn((rs - __half2float(rhs[j])) * kSplitScale);
               }
             }
           }
-        }
-        if (ALG2) {
-          // fp16 hi / lo split of rho 2^14, two vectors per word, into this coordinate's row
-          if (NV == 64 && i < KP) {
-            uint32_t hw[8], lw[8];
+          if (ALG2) {
+            if (NV == 64) {
+              // fp16 hi / lo split of rho 2^14, two vectors per word, kept for this coordinate's row
 #pragma unroll
-            for (int jp = 0; jp < 8; ++jp) {
-              const __half2 h2 = __floats2half2_rn(r2[2 * jp], r2[2 * jp + 1]);
-              const float2 back = __half22float2(h2);
-              hw[jp] = h2_bits(h2);
-              lw[jp] = h2_bits(__floats2half2_rn((r2[2 * jp] - back.x) * kSplitScale,
-                                                 (r2[2 * jp + 1] - back.y) * kSplitScale));
+              for (int jp = 0; jp < 8; ++jp) {
+                const __half2 h2 = __floats2half2_rn(r2[2 * jp], r2[2 * jp + 1]);
+                const float2 back = __half22float2(h2);
+                rhw[bt][jp] = h2_bits(h2);
+                rlw[bt][jp] = h2_bits(__floats2half2_rn((r2[2 * jp] - back.x) * kSplitScale,
+                                                                       (r2[2 * jp + 1] - back.y) * kSplitScale));
+              }
+              // |rho|^2 terms: (rho 2^14)^2 2^-28 rounds exactly like rho^2 (power-of-two scaling)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) r2[j] = r2[j] * r2[j] * (1.0f / 268435456.0f);
             }
-            const uint32_t o0 = sw128_offset(i, 2 * c0, 128), o1 = sw128_offset(i, 2 * c0 + 16, 128);
-            *(uint4*)(rho_hi + o0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *(uint4*)(rho_hi + o1) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-            *(uint4*)(rho_lo + o0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            *(uint4*)(rho_lo + o1) = make_uint4(lw[4], lw[5], lw[6], lw[7]);
           }
-          // |rho|^2 terms: (rho 2^14)^2 2^-28 rounds exactly like rho^2 (power-of-two scaling)
-          if (NV == 64) {
+          if (q < G && lane < 16) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) r2[j] = r2[j] * r2[j] * (1.0f / 268435456.0f);
+            for (int pl = 0; pl < BMAX; ++pl)
+              if (!MIX || pl < gbw) codes_stage[(c0 + lane) * wrec + woff + pl] = myw[pl];
           }
-        }
-        if (q < G && lane < 16) {
-#pragma unroll
-          for (int pl = 0; pl < BMAX; ++pl)
-            if (!MIX || pl < gbw) codes_stage[(c0 + lane) * wrec + woff + pl] = myw[pl];
+          if (ALG2) {
+            const float tot = transpose_reduce16(r2, lane);
+            if (lane < 16) gpart[q * NV + c0 + lane] = tot;
+          }
         }
         if (ALG2) {
-          const float tot = transpose_reduce16(r2, lane);
-          if (lane < 16) gpart[q * NV + c0 + lane] = tot;
+          // the tile's products of x and its scales are consumed: the next-but-one tile may use them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[ACC_EMPTY + a]);
+            mbar_arrive(&bar[INFO_EMPTY + a]);
+          }
         }
       }
       if (ALG2) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[RHO_FULL]);
+        if (k >= 1) {
+          // signs of tile k-1: sign(S r) = sign(T rho) from its T rho products
+          const int ap = (k - 1) & 1;
+          if (!mbar_wait_warp(&bar[T_FULL + ap], ((k - 1) >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t dT1 = tbase + lane_base + ap * COLS + 2 * NV, dT2 = dT1 + NV;
+          // eight vectors per TMEM load: this pass runs while rho of tile k is held in registers
+          for (int c0 = cbeg; c0 < cend; c0 += 16) {
+            uint32_t mys = 0;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t s1[8], s2[8];
+              tmem_ld8(dT1 + c0 + 8 * hh, s1);
+              tmem_ld8(dT2 + c0 + 8 * hh, s2);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float sv = fmaf(__uint_as_float(s2[j]), kSplitScaleInv, __uint_as_float(s1[j]));
+                const uint32_t w = __ballot_sync(0xffffffffu, active && sv >= 0.0f);
+                if (lane == 8 * hh + j) mys = w;
+              }
+            }
+            if (q < G && lane < 16) signs_stage[(c0 + lane) * G + q] = mys;
+          }
+          tc_fence_before();
+        }
+        if (has_tile) {
+          // the rho buffer is free (the T rho products of tile k-1 are complete): store rho of tile k
+          if (NV == 64) {
+            if (i < KP) {
+#pragma unroll
+              for (int bt = 0; bt < (NV == 64 ? 2 : 1); ++bt) {
+                const int c0 = cbeg + 16 * bt;
+                const uint32_t o0 = sw128_offset(i, 2 * c0, 128), o1 = sw128_offset(i, 2 * c0 + 16, 128);
+                *(uint4*)(rho_hi + o0) = make_uint4(rhw[bt][0], rhw[bt][1], rhw[bt][2], rhw[bt][3]);
+                *(uint4*)(rho_hi + o1) = make_uint4(rhw[bt][4], rhw[bt][5], rhw[bt][6], rhw[bt][7]);
+                *(uint4*)(rho_lo + o0) = make_uint4(rlw[bt][0], rlw[bt][1], rlw[bt][2], rlw[bt][3]);
+                *(uint4*)(rho_lo + o1) = make_uint4(rlw[bt][4], rlw[bt][5], rlw[bt][6], rlw[bt][7]);
+              }
+            }
+          } else if (i < KP) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t off = sw128_offset(cbeg + j, 2 * i, NV);
+              *(__half*)(rho_hi + off) = rhs[j];
+              *(__half*)(rho_lo + off) = rls[j];
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[RHO_FULL]);
+        }
       }
       if (!epi_sync()) break;
-      {
+      if (has_tile) {
         uint32_t* dst = p.codes + v0 * wrec;
         const int nw = rows * wrec;
         for (int w = te; w < nw; w += 256) dst[w] = codes_stage[w];
-      }
-      if (ALG2) {
-        if (te < rows) {
+        if (ALG2 && te < rows) {
           float g2 = 0.0f;
           for (int qq = 0; qq < G; ++qq) g2 += gpart[qq * NV + te];
           p.gammas[v0 + te] = __half_as_ushort(__float2half_rn(sqrtf(g2)));
         }
-        if (!mbar_wait_warp(&bar[T_FULL + a], (k >> 1) & 1, p.err, kDevTimeoutMma, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t dT1 = tbase + lane_base + a * COLS + 2 * NV, dT2 = dT1 + NV;
-        for (int c0 = cbeg; c0 < cend; c0 += 16) {
-          uint32_t s1[16], s2[16];
-          tmem_ld16(dT1 + c0, s1);
-          tmem_ld16(dT2 + c0, s2);
-          tmem_ld_wait();
-          uint32_t mys = 0;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float sv = fmaf(__uint_as_float(s2[j]), kSplitScaleInv, __uint_as_float(s1[j]));
-            const uint32_t w = __ballot_sync(0xffffffffu, active && sv >= 0.0f);
-            if (lane == j) mys = w;
-          }
-          if (q < G && lane < 16) signs_stage[(c0 + lane) * G + q] = mys;
-        }
-        if (!epi_sync()) break;
-        uint32_t* dst = p.signs + v0 * G;
-        const int nw = rows * G;
+      }
+      if (ALG2 && k >= 1) {
+        uint32_t* dst = p.signs + v0p * G;
+        const int nw = rowsp * G;
         for (int w = te; w < nw; w += 256) dst[w] = signs_stage[w];
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[ACC_EMPTY + a]);
-        mbar_arrive(&bar[INFO_EMPTY + a]);
+      if (!ALG2) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[ACC_EMPTY + a]);
+          mbar_arrive(&bar[INFO_EMPTY + a]);
+        }
       }
+      v0p = v0;
+      rowsp = rows;
       if (!epi_sync()) break;   // stage buffers are reused by the next tile
     }
   }
