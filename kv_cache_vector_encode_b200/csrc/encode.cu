@@ -95,10 +95,12 @@ __host__ __device__ inline EncLayout enc_layout(int d, int KP, int G) {
       for (int h = 0; h < 2; ++h) { L.off_bx[s][h] = off; off += L.bx_bytes; }
   if (ALG2)
     for (int h = 0; h < 2; ++h) { L.off_rho[h] = off; off += L.bx_bytes; }
-  L.off_codes = off; off += round_up((uint32_t)NV * G * BITS * 4, 128);
-  L.off_signs = off; off += round_up((uint32_t)NV * G * 4, 128);
+  // code, sign and gamma staging of the epilogue: two of each (tile parity), so that one
+  // synchronisation of the epilogue warps per tile suffices
+  L.off_codes = off; off += 2 * round_up((uint32_t)NV * G * BITS * 4, 128);
+  L.off_signs = off; off += 2 * round_up((uint32_t)NV * G * 4, 128);
   L.off_info = off; off += 2u * NV * 4;
-  L.off_gpart = off; off += 4u * NV * 4;
+  L.off_gpart = off; off += 2 * 4u * NV * 4;
   L.off_bar = round_up(off, 8); off = L.off_bar + 32 * 8;
   L.total = off + 1024;  // slack for 1024-byte alignment of the dynamic buffer
   return L;
@@ -143,9 +145,10 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
   uint32_t* tmem_slot = (uint32_t*)(bar + NBARS);
   volatile uint32_t* abort_flag = (volatile uint32_t*)(bar + NBARS) + 1;
   float* info = (float*)(smem + Lo.off_info);
-  float* gpart = (float*)(smem + Lo.off_gpart);
-  uint32_t* codes_stage = (uint32_t*)(smem + Lo.off_codes);
-  uint32_t* signs_stage = (uint32_t*)(smem + Lo.off_signs);
+  float* gpart0 = (float*)(smem + Lo.off_gpart);
+  uint32_t* codes_stage0 = (uint32_t*)(smem + Lo.off_codes);
+  uint32_t* signs_stage0 = (uint32_t*)(smem + Lo.off_signs);
+  const uint32_t codes_words = (Lo.off_signs - Lo.off_codes) / 8, signs_words = (Lo.off_info - Lo.off_signs) / 8;
   // stage-indexed buffers by arithmetic (keeps the layout struct out of local memory)
   const uint32_t raw0 = Lo.off_raw[0], raw_stride = Lo.off_raw[1] - Lo.off_raw[0];
   const uint32_t bx0 = F32 ? Lo.off_bx[0][0] : 0u, bx_stride = F32 ? Lo.off_bx[1][0] - Lo.off_bx[0][0] : 0u;
@@ -403,6 +406,10 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
     for (int k = 0; k < my_tiles + (ALG2 ? 1 : 0); ++k) {
       const bool has_tile = k < my_tiles;
       const int a = k & 1;
+      // this iteration's staging buffers (the other pair may still be read by slower warps)
+      uint32_t* codes_stage = codes_stage0 + a * codes_words;
+      uint32_t* signs_stage = signs_stage0 + a * signs_words;
+      float* gpart = gpart0 + a * 4 * NV;
       const int64_t v0 = (int64_t)(blockIdx.x + k * gridDim.x) * NV;
       const int rows = has_tile ? (int)min((int64_t)NV, p.n - v0) : 0;
       uint32_t rhw[NV / 32][8], rlw[NV / 32][8];   // NV = 64: fp16 words of rho 2^14 per batch
@@ -569,7 +576,6 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
       }
       v0p = v0;
       rowsp = rows;
-      if (!epi_sync()) break;   // stage buffers are reused by the next tile
     }
   }
 
