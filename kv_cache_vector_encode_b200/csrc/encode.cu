@@ -29,11 +29,11 @@
 // i.e. already in the tensor-core operand layout, with out-of-range rows / columns zero-filled.
 // bf16 tiles are converted to fp16 in place.
 //
-// Roles (14 warps, 15 for Algorithm 2): warp 0 issues the bulk / TMA copies; warp 1 owns TMEM and
-// issues the products of x; warp 14 (Algorithm 2) issues the T rho products; warps 2-5 convert (one
-// thread per vector: norm, power-of-two scale, fp16); warps 6-13 are the epilogue (two warps per
-// TMEM lane quarter, splitting the vectors of a tile). Buffers: input stage x2, TMEM accumulators
-// x2. All waits are bounded (sm100.cuh).
+// Roles: warp 0 issues the bulk / TMA copies; warp 1 owns TMEM and issues the products of x; then
+// the converters (norm, power-of-two scale, fp16; 4 warps, or 8 with two threads per vector for
+// Algorithm 1 on 128-vector tiles); then 8 epilogue warps (two per TMEM lane quarter, splitting the
+// vectors of a tile); and for Algorithm 2 a last warp that issues the T rho products (14 to 18 warps
+// in all). Buffers: input stage x2, TMEM accumulators x2. All waits are bounded (sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -46,8 +46,13 @@
 namespace tq {
 namespace {
 
-// threads: 14 warps, plus (Algorithm 2) a 15th that issues the T rho products
-__host__ __device__ constexpr int enc_threads(bool alg2) { return alg2 ? 480 : 448; }
+// converter warps: 8 for Algorithm 1 on 128-vector tiles (two threads per vector), else 4
+__host__ __device__ constexpr int enc_conv_warps(bool alg2, int nv) { return !alg2 && nv == 128 ? 8 : 4; }
+// threads: producer, MMA, converters, 8 epilogue warps, and (Algorithm 2) one that issues the T rho
+// products
+__host__ __device__ constexpr int enc_threads(bool alg2, int nv) {
+  return 32 * (2 + enc_conv_warps(alg2, nv) + 8 + (alg2 ? 1 : 0));
+}
 constexpr float kRhoScale = 16384.0f;   // 2^14: |rho| < 2 keeps rho * 2^14 below the fp16 maximum
 
 struct EncodeParams {
@@ -128,7 +133,7 @@ __device__ __forceinline__ float transpose_reduce16(float (&r)[16], int lane) {
 }
 
 template <int XT, bool ALG2, int NV, int BITS>
-__global__ void __launch_bounds__(enc_threads(ALG2), 1)
+__global__ void __launch_bounds__(enc_threads(ALG2, NV), 1)
     encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmap) {
   constexpr bool F32 = XT == TQ_F32;
   constexpr bool MIX = BITS == 0;                          // widths per channel group (Algorithm 1)
@@ -136,7 +141,10 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
   static_assert(!(MIX && ALG2), "mixed widths are an Algorithm 1 format");
   constexpr uint32_t COLS = ALG2 ? 4 * NV : 2 * NV;       // TMEM columns per accumulator buffer
   constexpr uint32_t NCOLS = 2 * COLS;
-  constexpr int TPV = 128 / NV;                            // converter threads per vector
+  constexpr int NCV = enc_conv_warps(ALG2, NV);            // converter warps (2 .. 1 + NCV)
+  constexpr int TPV = 32 * NCV / NV;                       // converter threads per vector
+  constexpr int W_EPI = 2 + NCV;                           // first of the 8 epilogue warps
+  constexpr int W_T = W_EPI + 8;                           // T rho issuer (Algorithm 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int d = p.d, KP = p.KP, G = p.G;
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[RAW_FULL + s], 1);
       mbar_init(&bar[STAGE_EMPTY + s], 1);
-      mbar_init(&bar[STAGE_READY + s], 4);     // one arrival per converter warp
+      mbar_init(&bar[STAGE_READY + s], NCV);   // one arrival per converter warp
       mbar_init(&bar[ACC_FULL + s], 1);
       mbar_init(&bar[ACC_EMPTY + s], 8);       // one arrival per epilogue warp
       mbar_init(&bar[INFO_EMPTY + s], 8);
@@ -205,9 +213,9 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
       }
       __syncwarp();
     }
-  } else if (warp == 1 || (ALG2 && warp == 14)) {
+  } else if (warp == 1 || (ALG2 && warp == W_T)) {
     // ---------------- MMA issuers ---------------------------------------------------------------
-    // warp 1 issues the products of x, warp 14 (Algorithm 2) those of rho, so that the T rho
+    // warp 1 issues the products of x, warp W_T (Algorithm 2) those of rho, so that the T rho
     // products of a tile start as soon as its rho is written, not after the next tile's x products.
     // Warp-uniform schedules (descriptors stay in uniform registers); one elected lane issues.
     if (mbar_wait_warp(&bar[A_FULL], 0, p.err, kDevTimeoutLoad, abort_flag)) {
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
         return true;
       };
       bool ok = true;
-      if (ALG2 && warp == 14) {
+      if (ALG2 && warp == W_T) {
         for (int j = 0; j < my_tiles && ok; ++j) ok = issue_T(j);
         ok = false;                                  // the x products are warp 1's
       }
@@ -269,7 +277,7 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
         __syncwarp();
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < W_EPI) {
     // ---------------- converters: one thread per vector (TPV threads when NV < 128) -------------
     const int ct = tid - 64;
     const int v = ct / TPV, part = ct % TPV;
@@ -367,13 +375,13 @@ __global__ void __launch_bounds__(enc_threads(ALG2), 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[STAGE_READY + s]);
     }
-  } else if (warp < 14) {
+  } else if (warp < W_EPI + 8) {
     // ---------------- epilogue: quantise, ballot-pack, residual, signs -------------------------
-    const int e = warp - 6;                 // 0..7
+    const int e = warp - W_EPI;             // 0..7
     const int q = warp & 3;                 // TMEM lane quarter = packing group
     const int i = q * 32 + lane;            // coordinate
     const bool active = i < d;
-    const int te = tid - 6 * 32;            // 0..255
+    const int te = tid - W_EPI * 32;        // 0..255
     const int cbeg = (e >> 2) * (NV / 2), cend = cbeg + NV / 2;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     float P[8], C[8];
@@ -599,7 +607,7 @@ tq_status launch_encode(EncodeParams& p, const void* x, cudaStream_t st) {
   if (e != cudaSuccess) return cuda_fail(e, "encode: shared memory attribute");
   p.ntiles = (int)((p.n + NV - 1) / NV);
   const int grid = std::min(p.ntiles, sm_count());
-  kern<<<grid, enc_threads(ALG2), Lo.total, st>>>(p, tmap);
+  kern<<<grid, enc_threads(ALG2, NV), Lo.total, st>>>(p, tmap);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "encode: launch");
   return TQ_OK;
 }
