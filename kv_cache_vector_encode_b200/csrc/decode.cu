@@ -299,23 +299,37 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           tmem_ld16(d2a + c0, rc);
           tmem_ld16(d2b + c0, rd);
         }
+        // Algorithm 1: the 16 vectors' norms as four 16-byte loads (Algorithm 2 reads its scales one
+        // by one, which keeps its four TMEM blocks in registers)
+        float nvs[16];
+        if (!ALG2) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 f = *(const float4*)&info[(a * 2 + 0) * NV + c0 + 4 * u];
+            nvs[4 * u] = f.x;
+            nvs[4 * u + 1] = f.y;
+            nvs[4 * u + 2] = f.z;
+            nvs[4 * u + 3] = f.w;
+          }
+        }
         tmem_ld_wait();
+        // row pointers advance by d elements per vector; a full batch needs no row check
+        const bool full = c0 + 16 <= rows;
+        const size_t row0 = (size_t)(v0 + c0) * d + j;
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          const int v = c0 + jj;
-          const float nv = info[(a * 2 + 0) * NV + v];
           float val = fmaf(__uint_as_float(rb[jj]), kSplitScaleInv, __uint_as_float(ra[jj]));
           if (ALG2) {
-            const float ag = info[(a * 2 + 1) * NV + v];
             const float sv = fmaf(__uint_as_float(rd[jj]), kSplitScaleInv, __uint_as_float(rc[jj]));
-            val = fmaf(ag, sv, val);
+            val = fmaf(info[(a * 2 + 1) * NV + c0 + jj], sv, val);
           }
-          val *= nv;
-          if (active && v < rows) {
+          val *= ALG2 ? info[(a * 2 + 0) * NV + c0 + jj] : nvs[jj];
+          if (active && (full || c0 + jj < rows)) {
+            const size_t o = row0 + (size_t)jj * d;
             if (OUT_BF16)
-              ((__nv_bfloat16*)p.out)[(v0 + v) * d + j] = __float2bfloat16_rn(val);
+              ((__nv_bfloat16*)p.out)[o] = __float2bfloat16_rn(val);
             else
-              ((float*)p.out)[(v0 + v) * d + j] = val;
+              ((float*)p.out)[o] = val;
           }
         }
       }
