@@ -48,6 +48,36 @@ B_DEC_V = (V_BITS_BLOCK - 1) * D // 8 + D // 8 + 4 + 4 * D
 B_ATT_TOKEN_HEAD = (K_BITS * D // 8 + 2) + ((V_BITS_CACHE - 1) * D // 8 + D // 8 + 4)   # 86 bytes
 
 
+TRAFFIC_SOURCES = ("attend.cu", "sm100.cuh")
+
+
+def traffic_from_record(rec, sources):
+    """DRAM bytes per launch from an ncu capture record, or None unless the sha256 recorded in it
+    equals the sha256 of `sources` (the kernel's source files' bytes, in order): a figure taken on
+    an earlier version of the kernel is not reported."""
+    import hashlib
+    h = hashlib.sha256()
+    for b in sources:
+        h.update(b)
+    if not isinstance(rec, dict) or rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def captured_traffic():
+    """DRAM bytes of one attention launch from the committed capture (profiles/), or None."""
+    prof = os.path.join(ROOT, "profiles", "attend_main_decode_attention_traffic.json")
+    try:
+        rec = json.load(open(prof))
+        srcs = []
+        for src in TRAFFIC_SOURCES:
+            with open(os.path.join(ROOT, "kv_cache_vector_encode_b200", "csrc", src), "rb") as f:
+                srcs.append(f.read())
+        return traffic_from_record(rec, srcs)
+    except Exception:
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -549,23 +579,7 @@ def run_ours(args):
     peak, peak_kind = peaks()
     att_bytes = B_ATT_TOKEN_HEAD * ATT_B * ATT_HKV * ATT_T + ATT_B * ATT_HQ * D * (2 + 4)
     att_gbs = att_bytes / (parts["attend"] * 1e-3) / 1e9
-    # DRAM bytes of one launch from the committed ncu capture, only while the kernel source is the
-    # one that was captured (the sha256 of attend.cu + sm100.cuh is recorded beside the figure)
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "attend_main_decode_attention_traffic.json")
-    if os.path.exists(prof):
-        try:
-            rec = json.load(open(prof))
-            import hashlib
-            h = hashlib.sha256()
-            for src in ("attend.cu", "sm100.cuh"):
-                with open(os.path.join(ROOT, "kv_cache_vector_encode_b200", "csrc", src), "rb") as f:
-                    h.update(f.read())
-            cur = h.hexdigest()
-            if rec.get("source_sha256") == cur:
-                traffic = rec.get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = captured_traffic()
     comp_bytes = {
         "encode_k": B_ENC_K * nblk, "encode_v": B_ENC_V * nblk,
         "decode_k": B_DEC_K * nblk, "decode_v": B_DEC_V * nblk, "attend": att_bytes,
