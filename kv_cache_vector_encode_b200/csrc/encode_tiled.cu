@@ -103,42 +103,54 @@ __device__ __forceinline__ void sym_bounds(int m, const float (&P)[8], float& lo
   }
 }
 
-// Exact (fp64) recomputation of one decision whose fp32 tensor-core value lies next to a boundary.
-// Rare: only values within 20x the parity band of a boundary take this path.
+// Exact (fp64) recomputation of a decision whose fp32 tensor-core value lies next to a boundary:
+// y_i = (Pi x)_i / |x| for a code, and for a sign (S r)_j for r = x / |x| - Pi^T c[idx], evaluated
+// as (S x)_j / |x| - (T c[idx])_j from the fp32 S and T and the vector's own codes (already
+// written). Rare: only values within 20x the parity band of a boundary take this path.
+// Both are computed by a whole warp for one lane's vector: each lane sums a strided slice of the d
+// terms in fp64, then a butterfly sum leaves the same total in every lane, so a decision next to a
+// boundary costs the warp d / 32 terms per lane instead of d serial terms.
 template <bool F32>
-__device__ __noinline__ double exact_row_dot_x(const float* prow, const void* x, int64_t v, int d) {
-  double acc = 0.0;
-  if (F32) {
-    const float* xr = (const float*)x + v * d;
-    for (int k = 0; k < d; ++k) acc = fma((double)prow[k], (double)xr[k], acc);
-  } else {
-    const uint16_t* xr = (const uint16_t*)x + v * d;
-    for (int k = 0; k < d; ++k) acc = fma((double)prow[k], (double)__uint_as_float((uint32_t)xr[k] << 16), acc);
+__device__ __noinline__ double warp_row_dot_x(const float* prow, const void* x, int64_t v, int d, int lane) {
+  double a0 = 0.0, a1 = 0.0;
+  for (int k = lane; k < d; k += 64) {
+    const int k1 = k + 32;
+    if (F32) {
+      const float* xr = (const float*)x + v * d;
+      a0 = fma((double)__ldg(prow + k), (double)__ldg(xr + k), a0);
+      if (k1 < d) a1 = fma((double)__ldg(prow + k1), (double)__ldg(xr + k1), a1);
+    } else {
+      const unsigned short* xr = (const unsigned short*)x + v * d;
+      a0 = fma((double)__ldg(prow + k), (double)__uint_as_float((uint32_t)__ldg(xr + k) << 16), a0);
+      if (k1 < d) a1 = fma((double)__ldg(prow + k1), (double)__uint_as_float((uint32_t)__ldg(xr + k1) << 16), a1);
+    }
   }
-  return acc;
+  double s = a0 + a1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
 }
 
-// (S r)_j for r = x / |x| - Pi^T c[idx], evaluated as (S x)_j / |x| - (T c[idx])_j in fp64 from
-// the fp32 S and T and this vector's codes (already written by this thread).
 template <bool F32, int BITS>
-__device__ __noinline__ double exact_sign_value(const float* srow, const float* trow, const void* x, int64_t v, int d,
-                                                double nrm, const uint32_t* vcodes, const float (&C)[8]) {
-  const double sx = exact_row_dot_x<F32>(srow, x, v, d) / nrm;
+__device__ __noinline__ double warp_sign_value(const float* srow, const float* trow, const void* x, int64_t v, int d,
+                                               double nrm, const uint32_t* vcodes, const float (&C)[8], int lane) {
+  const double sx = warp_row_dot_x<F32>(srow, x, v, d, lane) / nrm;
   constexpr int H = 1 << (BITS - 1);
   double tc = 0.0;
-  for (int k = 0; k < d; ++k) {
+  for (int k = lane; k < d; k += 32) {              // coordinate k = 32 (k >> 5) + lane of the code words
     const uint32_t* wk = vcodes + (k >> 5) * BITS;
-    const int l = k & 31;
-    const bool neg = ((wk[BITS - 1] >> l) & 1u) == 0u;
+    const bool neg = ((wk[BITS - 1] >> lane) & 1u) == 0u;
     int m = 0;
-    for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> l) & 1u) << pl;
+    for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> lane) & 1u) << pl;
     if (neg) m ^= H - 1;
     float cm = C[0];
 #pragma unroll
     for (int q = 1; q < H; ++q)
       if (q == m) cm = C[q];
-    tc = fma((double)trow[k], neg ? -(double)cm : (double)cm, tc);
+    tc = fma((double)__ldg(trow + k), neg ? -(double)cm : (double)cm, tc);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tc += __shfl_xor_sync(0xffffffffu, tc, o);
   return sx - tc;
 }
 
@@ -547,17 +559,27 @@ __global__ void __launch_bounds__(kTThreads, 1)
               float blo, bhi;
               sym_bounds<BITS>(m, P, blo, bhi);
               const float a = fabsf(y);
-              if (live && inv != 0.0f && fminf(a - blo, bhi - a) < tau_y) {
-                // next to a boundary: decide on the fp64 value
+              // next to a boundary: decide on the fp64 value, computed by the whole warp for each
+              // lane that needs one (coordinate i is the same for every lane)
+              uint32_t nm = __ballot_sync(0xffffffffu, live && inv != 0.0f && fminf(a - blo, bhi - a) < tau_y);
+              if (nm) {
                 const int i = nb * 128 + g * 32 + j;
-                const double yd = exact_row_dot_x<F32>(p.pi32 + (size_t)i * p.d, p.x, v, p.d) / nrm;
-                neg = !(yd > 0.0);
-                const double ad = fabs(yd);
-                int mm = 0;
+                const float* prow = p.pi32 + (size_t)i * p.d;
+                while (nm) {
+                  const int L = __ffs(nm) - 1;
+                  nm &= nm - 1;
+                  const double dot = warp_row_dot_x<F32>(prow, p.x, __shfl_sync(0xffffffffu, v, L), p.d, lane);
+                  if (lane == L) {
+                    const double yd = dot / nrm;
+                    neg = !(yd > 0.0);
+                    const double ad = fabs(yd);
+                    int mm = 0;
 #pragma unroll
-                for (int k = 0; k < (1 << (BITS - 1)) - 1; ++k) mm += (double)P[k] < ad ? 1 : 0;
-                m = mm;
-                y = (float)yd;
+                    for (int k = 0; k < (1 << (BITS - 1)) - 1; ++k) mm += (double)P[k] < ad ? 1 : 0;
+                    m = mm;
+                    y = (float)yd;
+                  }
+                }
               }
             }
 #pragma unroll
@@ -642,11 +664,20 @@ __global__ void __launch_bounds__(kTThreads, 1)
             for (int j = 0; j < 32; ++j) {
               const float sv = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j]));
               bool bit = sv >= 0.0f;
-              if (live && fabsf(sv) < tau_s) {
-                // next to zero: decide on the exact fp64 value (the residual's own rounding included)
+              // next to zero: decide on the exact fp64 value (the residual's own rounding included),
+              // computed by the whole warp for each lane that needs one
+              uint32_t nm = __ballot_sync(0xffffffffu, live && fabsf(sv) < tau_s);
+              if (nm) {
                 const int jg = nb * 128 + g * 32 + j;
-                bit = exact_sign_value<F32, BITS>(p.s32 + (size_t)jg * p.d, p.t32 + (size_t)jg * p.d, p.x, v, p.d, nrm,
-                                                  p.codes + (size_t)v * G * BITS, C) >= 0.0;
+                while (nm) {
+                  const int L = __ffs(nm) - 1;
+                  nm &= nm - 1;
+                  const int64_t vl = __shfl_sync(0xffffffffu, v, L);
+                  const double val = warp_sign_value<F32, BITS>(
+                      p.s32 + (size_t)jg * p.d, p.t32 + (size_t)jg * p.d, p.x, vl, p.d, __shfl_sync(0xffffffffu, nrm, L),
+                      p.codes + (size_t)vl * G * BITS, C, lane);
+                  if (lane == L) bit = val >= 0.0;
+                }
               }
               w |= (bit ? 1u : 0u) << j;
             }
