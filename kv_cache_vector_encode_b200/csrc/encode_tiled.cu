@@ -23,7 +23,8 @@
 // for the fp16 rounding of gamma = |r|: a gamma within 2^-15 (relative) of an fp16 rounding
 // midpoint, far wider than the fp32 accumulation error, is flagged, and a fix-up kernel recomputes
 // r = x / |x| - Pi^T c[idx] for that vector in fp64 from x, the fp32 Pi and the vector's own codes,
-// and rewrites gamma (a few percent of the vectors; about d^2 fp64 operations each).
+// and rewrites gamma (about 9 % of the vectors; d^2 fp64 operations each, one pass over Pi serving
+// a batch of eight).
 //
 // Roles (10 warps): 0 TMA / bulk copies; 1 TMEM owner and MMA issuer; 2-5 converters (thread =
 // vector: fp64 norm, fp16 split of x, copies of the rho images); 6-9 epilogue (thread = vector).
@@ -168,69 +169,164 @@ __device__ __forceinline__ bool near_f16_midpoint(double x, double tol) {
   return fabs(x - mid) <= tol * x;
 }
 
+constexpr int kFixThreads = 256;
+constexpr size_t kFixCounterBytes = 16;          // the fix-up's claim counter, after the flag words
+constexpr int kFixChunkWords = 4;                // flag words (128 vectors) a block claims at a time
+
 // Exact gamma for the flagged vectors: r = x / |x| - Pi^T c[idx] in fp64 (original domain, the
-// vector's own codes), gamma = |r| rounded to fp16. One block of 256 threads per flagged vector.
-template <bool F32, int BITS>
-__global__ void __launch_bounds__(256) gamma_fixup_kernel(const __grid_constant__ TEParams p, int nwords) {
-  extern __shared__ double fx[];                      // [d] x (fp64), [d] c[idx] (fp64)
-  __shared__ double red[8];
+// vector's own codes), gamma = |r| rounded to fp16. Blocks claim chunks of flag words from a
+// counter that follows the flag words, and take the flagged vectors VB at a time: one pass over the
+// fp32 Pi serves the whole batch (Pi is read once per VB vectors) and every thread keeps 2 x VB
+// independent fp64 sums in flight. For each vector the sums are formed in the order of a plain
+// one-vector loop: (Pi^T c)_j = sum over i ascending, |x|^2 and |r|^2 over this thread's columns
+// j = tid + 256 t ascending, then a warp butterfly and the warps' totals in warp order.
+template <bool F32, int BITS, int VB>
+__global__ void __launch_bounds__(kFixThreads) gamma_fixup_kernel(const __grid_constant__ TEParams p, int nwords) {
+  extern __shared__ __align__(16) double cs[];        // [d][VB]: c_i of the batch's vectors (fp64)
+  __shared__ double red[kFixThreads / 32][VB];
+  __shared__ double nrm_s[VB];
+  __shared__ int64_t vsel[VB];
+  __shared__ int nsel;
+  constexpr int NW = kFixThreads / 32, H = 1 << (BITS - 1);
   const int d = p.d, G = p.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  double* xs = fx;
-  double* cs = fx + d;
-  constexpr int H = 1 << (BITS - 1);
-  auto block_sum = [&](double v) -> double {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    double t = 0.0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) t += red[w];
-    return t;
+  unsigned int* counter = (unsigned int*)(p.gflag + nwords);
+  auto xval = [&](int64_t v, int j) -> double {
+    return F32 ? (double)((const float*)p.x)[v * d + j]
+               : (double)__uint_as_float((uint32_t)((const uint16_t*)p.x)[v * d + j] << 16);
   };
-  for (int wi = blockIdx.x; wi < nwords; wi += gridDim.x) {
-    uint32_t bits = p.gflag[wi];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      const int64_t v = (int64_t)wi * 32 + b;
-      double ss = 0.0;
-      for (int j = tid; j < d; j += 256) {
-        const double xj = F32 ? (double)((const float*)p.x)[v * d + j]
-                              : (double)__uint_as_float((uint32_t)((const uint16_t*)p.x)[v * d + j] << 16);
-        xs[j] = xj;
-        ss = fma(xj, xj, ss);
-      }
-      const double nrm = sqrt(block_sum(ss));
-      const uint32_t* vc = p.codes + (size_t)v * G * BITS;
-      for (int i = tid; i < d; i += 256) {
-        const uint32_t* wk = vc + (i >> 5) * BITS;
-        const int l = i & 31;
-        const bool neg = ((wk[BITS - 1] >> l) & 1u) == 0u;
-        int m = 0;
-        for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> l) & 1u) << pl;
-        if (neg) m ^= H - 1;
-        float cm = p.C[0];
+  // totals of VB per-thread values over the block (every thread gets them; red is free afterwards)
+  auto block_sums = [&](double (&v)[VB], double (&out)[VB]) {
 #pragma unroll
-        for (int q = 1; q < H; ++q)
-          if (q == m) cm = p.C[q];
-        cs[i] = neg ? -(double)cm : (double)cm;
-      }
-      __syncthreads();
-      double g2 = 0.0;
-      for (int j = tid; j < d; j += 256) {
-        double a = 0.0;                                  // (Pi^T c)_j = sum_i Pi[i][j] c_i
-        for (int i = 0; i < d; ++i) a = fma((double)__ldg(p.pi32 + (size_t)i * d + j), cs[i], a);
-        const double r = xs[j] / nrm - a;
-        g2 = fma(r, r, g2);
-      }
-      g2 = block_sum(g2);
-      if (tid == 0) p.gammas[v] = __half_as_ushort(__double2half(sqrt(g2)));
-      __syncthreads();
+    for (int k = 0; k < VB; ++k) {
+      double t = v[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) red[warp][k] = t;
     }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < VB; ++k) {
+      double t = 0.0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) t += red[w][k];
+      out[k] = t;
+    }
+    __syncthreads();
+  };
+  // thread 0's cursor over the claimed flag words
+  int cur = 0, cend = 0, wbase = 0;
+  uint32_t bits = 0u;
+  bool drained = false;
+  for (;;) {
+    __syncthreads();                                  // the previous batch's vsel / nsel are read
+    if (tid == 0) {
+      int n = 0;
+      while (n < VB && !drained) {
+        if (bits) {
+          vsel[n++] = (int64_t)wbase * 32 + (__ffs(bits) - 1);
+          bits &= bits - 1u;
+        } else if (cur < cend) {
+          wbase = cur;
+          bits = p.gflag[cur++];
+        } else {
+          const int c = (int)atomicAdd(counter, 1u) * kFixChunkWords;
+          if (c >= nwords) {
+            drained = true;
+          } else {
+            cur = c;
+            cend = min(nwords, c + kFixChunkWords);
+          }
+        }
+      }
+      nsel = n;
+    }
+    __syncthreads();
+    const int n = nsel;
+    if (n == 0) break;
+    // |x| of the batch
+    double acc[VB], tot[VB];
+#pragma unroll
+    for (int k = 0; k < VB; ++k) acc[k] = 0.0;
+    for (int j = tid; j < d; j += kFixThreads) {
+#pragma unroll
+      for (int k = 0; k < VB; ++k)
+        if (k < n) {
+          const double xj = xval(vsel[k], j);
+          acc[k] = fma(xj, xj, acc[k]);
+        }
+    }
+    block_sums(acc, tot);
+#pragma unroll
+    for (int k = 0; k < VB; ++k)
+      if (tid == k) nrm_s[k] = sqrt(tot[k]);
+    // c[idx] of the batch from its code words
+    for (int i = tid; i < d; i += kFixThreads) {
+      const int l = i & 31;
+#pragma unroll
+      for (int k = 0; k < VB; ++k) {
+        double c = 0.0;
+        if (k < n) {
+          const uint32_t* wk = p.codes + (size_t)vsel[k] * G * BITS + (i >> 5) * BITS;
+          const bool neg = ((wk[BITS - 1] >> l) & 1u) == 0u;
+          int m = 0;
+          for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> l) & 1u) << pl;
+          if (neg) m ^= H - 1;
+          float cm = p.C[0];
+#pragma unroll
+          for (int q = 1; q < H; ++q)
+            if (q == m) cm = p.C[q];
+          c = neg ? -(double)cm : (double)cm;
+        }
+        cs[(size_t)i * VB + k] = c;
+      }
+    }
+    __syncthreads();
+    // r_j = x_j / |x| - (Pi^T c)_j for this thread's columns, two at a time
+#pragma unroll
+    for (int k = 0; k < VB; ++k) acc[k] = 0.0;         // |r|^2
+    for (int j0 = tid; j0 < d; j0 += 2 * kFixThreads) {
+      const int j1 = j0 + kFixThreads;
+      const bool h1 = j1 < d;
+      double a0[VB], a1[VB];
+#pragma unroll
+      for (int k = 0; k < VB; ++k) a0[k] = a1[k] = 0.0;
+      const float* p0 = p.pi32 + j0;
+      const float* p1 = p.pi32 + (h1 ? j1 : j0);
+#pragma unroll 4
+      for (int i = 0; i < d; ++i) {
+        const double pi0 = (double)__ldg(p0 + (size_t)i * d);
+        const double pi1 = (double)__ldg(p1 + (size_t)i * d);
+        const double2* cv = (const double2*)(cs + (size_t)i * VB);
+#pragma unroll
+        for (int kk = 0; kk < VB / 2; ++kk) {
+          const double2 c2 = cv[kk];
+          a0[2 * kk] = fma(pi0, c2.x, a0[2 * kk]);
+          a0[2 * kk + 1] = fma(pi0, c2.y, a0[2 * kk + 1]);
+          a1[2 * kk] = fma(pi1, c2.x, a1[2 * kk]);
+          a1[2 * kk + 1] = fma(pi1, c2.y, a1[2 * kk + 1]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < VB; ++k)
+        if (k < n) {
+          const double nk = nrm_s[k];
+          const double r0 = xval(vsel[k], j0) / nk - a0[k];
+          acc[k] = fma(r0, r0, acc[k]);
+          if (h1) {
+            const double r1 = xval(vsel[k], j1) / nk - a1[k];
+            acc[k] = fma(r1, r1, acc[k]);
+          }
+        }
+    }
+    block_sums(acc, tot);
+#pragma unroll
+    for (int k = 0; k < VB; ++k)
+      if (tid == k && k < n) p.gammas[vsel[k]] = __half_as_ushort(__double2half(sqrt(tot[k])));
   }
 }
+
+// Fix-up batch size: the batch's fp64 codebook values (d x VB) must fit in shared memory.
+inline int fixup_batch(int d) { return d <= 3072 ? 8 : 4; }
 
 template <bool F32, bool ALG2, int BITS>
 __global__ void __launch_bounds__(kTThreads, 1)
@@ -718,15 +814,17 @@ tq_status launch_tiled(TEParams& p, const void* x, int grid, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo.total);
   if (e != cudaSuccess) return cuda_fail(e, "encode: shared memory attribute");
   const int nwords = (int)((p.n + 31) / 32);
-  if (ALG2 && (e = cudaMemsetAsync(p.gflag, 0, (size_t)nwords * 4, st)) != cudaSuccess)
+  if (ALG2 && (e = cudaMemsetAsync(p.gflag, 0, (size_t)nwords * 4 + kFixCounterBytes, st)) != cudaSuccess)
     return cuda_fail(e, "encode: clear the gamma flags");
   kern<<<grid, kTThreads, Lo.total, st>>>(p, tmap);
   if (ALG2) {
-    auto fix = gamma_fixup_kernel<F32, BITS>;
-    const int fsm = 2 * p.d * (int)sizeof(double);
+    const int vb = fixup_batch(p.d);
+    auto fix = vb == 8 ? gamma_fixup_kernel<F32, BITS, 8> : gamma_fixup_kernel<F32, BITS, 4>;
+    const int fsm = p.d * vb * (int)sizeof(double);
     if (fsm > 48 * 1024 && (e = cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm)) != cudaSuccess)
       return cuda_fail(e, "encode: gamma fix-up shared memory attribute");
-    fix<<<std::max(1, std::min(nwords, 4 * grid)), 256, fsm, st>>>(p, nwords);
+    const int nchunks = (nwords + kFixChunkWords - 1) / kFixChunkWords;
+    fix<<<std::max(1, std::min(nchunks, 2 * sm_count())), kFixThreads, fsm, st>>>(p, nwords);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "encode: launch");
   return TQ_OK;
@@ -745,7 +843,7 @@ tq_status launch_tiled_bits(TEParams& p, int bits, const void* x, int grid, cuda
 }  // namespace
 
 // Algorithm 2 workspace: the residual slots of the tiles in flight (one per CTA), then one flag bit
-// per vector (gamma next to an fp16 rounding midpoint).
+// per vector (gamma next to an fp16 rounding midpoint), then the fix-up's claim counter.
 size_t tiled_rho_bytes(int64_t n, int d, int nsm) {
   const int64_t ntiles = (n + 127) / 128;
   const int64_t grid = std::min<int64_t>(ntiles, nsm);
@@ -754,7 +852,7 @@ size_t tiled_rho_bytes(int64_t n, int d, int nsm) {
 
 size_t encode_tiled_ws_bytes(int64_t n, int d, bool alg2, int nsm) {
   if (!alg2 || d <= 128 || n <= 0) return 0;
-  return tiled_rho_bytes(n, d, nsm) + (size_t)((n + 31) / 32) * 4;
+  return tiled_rho_bytes(n, d, nsm) + (size_t)((n + 31) / 32) * 4 + kFixCounterBytes;
 }
 
 tq_status encode_tiled(const tq_codebook* cb, int64_t n, int d, const void* x, int xt, const void* rot,

@@ -49,6 +49,23 @@ def test_tiled_vector_search_shape(dev):
     print("tiled prod d1536", st)
 
 
+@pytest.mark.parametrize("d", [3072, 4096])
+def test_tiled_prod_largest_d(dev, d):
+    # the largest dimensions (the exact-gamma fix-up holds a batch's codebook values of all d
+    # coordinates in shared memory: eight vectors at a time up to d = 3072, four above)
+    x = W.gaussian(700, d, seed=d, tag=W.TAG_X)
+    st = check_prod(x, d, 3, torch.float32, dev, decode=False)
+    print("tiled prod", d, st)
+
+
+def test_tiled_prod_many_fixup_batches(dev):
+    # enough rows that every fix-up block claims several chunks of flag words and fills batches
+    # across chunk boundaries (about 4 % of the gammas lie near an fp16 rounding midpoint)
+    x = W.gaussian(120_000, 256, seed=77, tag=W.TAG_X)
+    st = check_prod(x, 256, 3, torch.float32, dev, decode=False)
+    print("tiled prod d256 n120000", st)
+
+
 def test_tiled_mse_d1536_bf16(dev):
     x = W.round_to_bf16(W.gaussian(300, 1536, seed=3, tag=W.TAG_X))
     st = check_mse(x, 1536, 3, torch.bfloat16, dev, decode=False)
