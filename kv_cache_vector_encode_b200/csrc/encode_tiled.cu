@@ -90,18 +90,25 @@ enum TBars {
   NORM_READY = 16, INFO_EMPTY = 18, RHO_READY = 20, TNBARS = 21
 };
 
+// P[k] for 0 <= k < H - 1, as a tree of selects on the bits of k: with no indexed access to P the
+// compiler keeps the boundaries in registers (an indexed form placed them in local memory, whose
+// loads missed the small L1 left beside this kernel's shared memory).
+template <int BITS>
+__device__ __forceinline__ float sym_p(int k, const float (&P)[8]) {
+  if (BITS <= 2) return P[0];
+  if (BITS == 3) return (k & 2) ? P[2] : ((k & 1) ? P[1] : P[0]);
+  const float lo = (k & 2) ? ((k & 1) ? P[3] : P[2]) : ((k & 1) ? P[1] : P[0]);
+  const float hi = (k & 2) ? P[6] : ((k & 1) ? P[5] : P[4]);
+  return (k & 4) ? hi : lo;
+}
+
 // Cell of |y| the symmetric quantiser chose: (lo, hi] with lo = P[m-1] (0 for m = 0), hi = P[m]
 // (infinity for the top cell).
 template <int BITS>
 __device__ __forceinline__ void sym_bounds(int m, const float (&P)[8], float& lo, float& hi) {
   constexpr int H = 1 << (BITS - 1);
-  lo = 0.0f;
-  hi = INFINITY;
-#pragma unroll
-  for (int k = 0; k < H - 1; ++k) {
-    if (k == m - 1) lo = P[k];
-    if (k == m) hi = P[k];
-  }
+  lo = m == 0 ? 0.0f : sym_p<BITS>(m - 1, P);
+  hi = m == H - 1 ? INFINITY : sym_p<BITS>(m, P);
 }
 
 // Exact (fp64) recomputation of a decision whose fp32 tensor-core value lies next to a boundary:
@@ -134,7 +141,7 @@ __device__ __noinline__ double warp_row_dot_x(const float* prow, const void* x, 
 
 template <bool F32, int BITS>
 __device__ __noinline__ double warp_sign_value(const float* srow, const float* trow, const void* x, int64_t v, int d,
-                                               double nrm, const uint32_t* vcodes, const float (&C)[8], int lane) {
+                                               double nrm, const uint32_t* vcodes, const float* C, int lane) {
   const double sx = warp_row_dot_x<F32>(srow, x, v, d, lane) / nrm;
   constexpr int H = 1 << (BITS - 1);
   double tc = 0.0;
@@ -144,10 +151,7 @@ __device__ __noinline__ double warp_sign_value(const float* srow, const float* t
     int m = 0;
     for (int pl = 0; pl < BITS - 1; ++pl) m |= (int)((wk[pl] >> lane) & 1u) << pl;
     if (neg) m ^= H - 1;
-    float cm = C[0];
-#pragma unroll
-    for (int q = 1; q < H; ++q)
-      if (q == m) cm = C[q];
+    const float cm = C[m];
     tc = fma((double)__ldg(trow + k), neg ? -(double)cm : (double)cm, tc);
   }
 #pragma unroll
@@ -342,6 +346,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = p.KB, NB = p.NB, G = p.G;
   const int nsweeps = 1 + NB + (ALG2 ? NB : 0);
+  __shared__ float c_tab[8];                 // the positive centroids, for the exact sign fallback
+  if (tid < 8) c_tab[tid] = p.C[tid];
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -581,17 +587,26 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int nb = 0; nb < NB && ok; ++nb) {
           for (int kb = 0; kb < KB; ++kb) {
             const int as = ja & 1;
+            // all sixteen loads of this thread's row go out before the stage wait and the stores
+            // (interleaved, each store waited for its load: one L2 round trip per 32 bytes)
+            const uint8_t* src = slot + (size_t)kb * 2 * kBlk;
+            uint4 vh[8], vl[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t off = sw128_offset(r, c * 16, 128);
+              vh[c] = __ldcg((const uint4*)(src + off));
+              vl[c] = __ldcg((const uint4*)(src + kBlk + off));
+            }
             if (ja >= 2 && !mbar_wait_warp(&bar[A_EMPTY + as], ((ja >> 1) - 1) & 1, p.err, kDevTimeoutMma, abort_flag)) {
               ok = false;
               break;
             }
-            const uint8_t* src = slot + (size_t)kb * 2 * kBlk;
             uint8_t* ah = smem + Lo.a + as * 2 * kBlk;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               const uint32_t off = sw128_offset(r, c * 16, 128);
-              *(uint4*)(ah + off) = __ldcg((const uint4*)(src + off));
-              *(uint4*)(ah + kBlk + off) = __ldcg((const uint4*)(src + kBlk + off));
+              *(uint4*)(ah + off) = vh[c];
+              *(uint4*)(ah + kBlk + off) = vl[c];
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -633,8 +648,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t words[4][BITS];
-#pragma unroll
+        // the 4 x BITS words of this band are contiguous in the vector's record: group g's BITS
+        // plane words at g BITS. The group loop stays rolled: unrolled four times, with the
+        // unrolled coordinate loop inside, the epilogue's code outgrew the instruction cache.
+        uint32_t* dst = p.codes + (live ? ((size_t)v * G + 4 * nb) * BITS : 0);
+#pragma unroll 1
         for (int g = 0; g < 4; ++g) {
           uint32_t hi[32], lo[32];
           const uint32_t col = tbase + lane_base + acc * 256 + g * 32;
@@ -643,8 +661,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
           tmem_ld16(col + 128, *(uint32_t(*)[16]) & lo[0]);
           tmem_ld16(col + 144, *(uint32_t(*)[16]) & lo[16]);
           tmem_ld_wait();
+          uint32_t words[BITS];
 #pragma unroll
-          for (int pl = 0; pl < BITS; ++pl) words[g][pl] = 0u;
+          for (int pl = 0; pl < BITS; ++pl) words[pl] = 0u;
           float rho[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -681,7 +700,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
             for (int pl = 0; pl < BITS; ++pl) {
               const bool bit = pl == BITS - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
-              words[g][pl] |= (bit ? 1u : 0u) << j;
+              words[pl] |= (bit ? 1u : 0u) << j;
             }
             if (ALG2) {
               const float cm = sym_c<BITS>(m, C);
@@ -712,25 +731,15 @@ __global__ void __launch_bounds__(kTThreads, 1)
               *(uint4*)(blk + kBlk + off) = make_uint4(l[0], l[1], l[2], l[3]);
             }
           }
+          if (live) {
+#pragma unroll
+            for (int pl = 0; pl < BITS; ++pl) dst[g * BITS + pl] = words[pl];
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[ACC_EMPTY + acc]);
         ++jacc;
-        if (live) {
-          // the 4 x BITS words of this band are contiguous in the vector's record
-          uint32_t* dst = p.codes + ((size_t)v * G + 4 * nb) * BITS;
-#pragma unroll
-          for (int w = 0; w < BITS; ++w) {
-            uint32_t o[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int flat = 4 * w + u;
-              o[u] = words[flat / BITS][flat % BITS];
-            }
-            *(uint4*)(dst + 4 * w) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
       }
       if (!ok) break;
       if (ALG2) {
@@ -745,8 +754,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
             break;
           }
           tc_fence_after();
-          uint32_t sw[4];
-#pragma unroll
+#pragma unroll 1
           for (int g = 0; g < 4; ++g) {
             uint32_t hi[32], lo[32];
             const uint32_t col = tbase + lane_base + acc * 256 + g * 32;
@@ -771,19 +779,18 @@ __global__ void __launch_bounds__(kTThreads, 1)
                   const int64_t vl = __shfl_sync(0xffffffffu, v, L);
                   const double val = warp_sign_value<F32, BITS>(
                       p.s32 + (size_t)jg * p.d, p.t32 + (size_t)jg * p.d, p.x, vl, p.d, __shfl_sync(0xffffffffu, nrm, L),
-                      p.codes + (size_t)vl * G * BITS, C, lane);
+                      p.codes + (size_t)vl * G * BITS, c_tab, lane);
                   if (lane == L) bit = val >= 0.0;
                 }
               }
               w |= (bit ? 1u : 0u) << j;
             }
-            sw[g] = w;
+            if (live) p.signs[(size_t)v * G + 4 * nb + g] = w;
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar[ACC_EMPTY + acc]);
           ++jacc;
-          if (live) *(uint4*)(p.signs + (size_t)v * G + 4 * nb) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
         }
         if (!ok) break;
         if (live) {
