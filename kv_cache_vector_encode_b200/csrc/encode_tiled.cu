@@ -649,84 +649,83 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         tc_fence_after();
         // the 4 x BITS words of this band are contiguous in the vector's record: group g's BITS
-        // plane words at g BITS. The group loop stays rolled: unrolled four times, with the
-        // unrolled coordinate loop inside, the epilogue's code outgrew the instruction cache.
+        // plane words at g BITS. The loops over groups and over 8-coordinate chunks stay rolled:
+        // fully unrolled, the epilogue's code outgrew the instruction cache.
         uint32_t* dst = p.codes + (live ? ((size_t)v * G + 4 * nb) * BITS : 0);
 #pragma unroll 1
         for (int g = 0; g < 4; ++g) {
-          uint32_t hi[32], lo[32];
-          const uint32_t col = tbase + lane_base + acc * 256 + g * 32;
-          tmem_ld16(col, *(uint32_t(*)[16]) & hi[0]);
-          tmem_ld16(col + 16, *(uint32_t(*)[16]) & hi[16]);
-          tmem_ld16(col + 128, *(uint32_t(*)[16]) & lo[0]);
-          tmem_ld16(col + 144, *(uint32_t(*)[16]) & lo[16]);
-          tmem_ld_wait();
           uint32_t words[BITS];
 #pragma unroll
           for (int pl = 0; pl < BITS; ++pl) words[pl] = 0u;
-          float rho[32];
+          const int i0 = nb * 128 + g * 32;
+#pragma unroll 1
+          for (int kq = 0; kq < 4; ++kq) {              // coordinates i0 + 8 kq .. + 7
+            uint32_t hi[8], lo[8];
+            const uint32_t col = tbase + lane_base + acc * 256 + g * 32 + 8 * kq;
+            tmem_ld8(col, hi);
+            tmem_ld8(col + 128, lo);
+            tmem_ld_wait();
+            float rho[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float y = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j])) * inv;
-            bool neg = !(y > 0.0f);
-            int m = sym_m<BITS>(fabsf(y), P);
-            {
-              float blo, bhi;
-              sym_bounds<BITS>(m, P, blo, bhi);
-              const float a = fabsf(y);
-              // next to a boundary: decide on the fp64 value, computed by the whole warp for each
-              // lane that needs one (coordinate i is the same for every lane)
-              uint32_t nm = __ballot_sync(0xffffffffu, live && inv != 0.0f && fminf(a - blo, bhi - a) < tau_y);
-              if (nm) {
-                const int i = nb * 128 + g * 32 + j;
-                const float* prow = p.pi32 + (size_t)i * p.d;
-                while (nm) {
-                  const int L = __ffs(nm) - 1;
-                  nm &= nm - 1;
-                  const double dot = warp_row_dot_x<F32>(prow, p.x, __shfl_sync(0xffffffffu, v, L), p.d, lane);
-                  if (lane == L) {
-                    const double yd = dot / nrm;
-                    neg = !(yd > 0.0);
-                    const double ad = fabs(yd);
-                    int mm = 0;
+            for (int jj = 0; jj < 8; ++jj) {
+              const int j = 8 * kq + jj;
+              float y = fmaf(__uint_as_float(lo[jj]), kSplitScaleInv, __uint_as_float(hi[jj])) * inv;
+              bool neg = !(y > 0.0f);
+              int m = sym_m<BITS>(fabsf(y), P);
+              {
+                float blo, bhi;
+                sym_bounds<BITS>(m, P, blo, bhi);
+                const float a = fabsf(y);
+                // next to a boundary: decide on the fp64 value, computed by the whole warp for each
+                // lane that needs one (coordinate i is the same for every lane)
+                uint32_t nm = __ballot_sync(0xffffffffu, live && inv != 0.0f && fminf(a - blo, bhi - a) < tau_y);
+                if (nm) {
+                  const int i = i0 + j;
+                  const float* prow = p.pi32 + (size_t)i * p.d;
+                  while (nm) {
+                    const int L = __ffs(nm) - 1;
+                    nm &= nm - 1;
+                    const double dot = warp_row_dot_x<F32>(prow, p.x, __shfl_sync(0xffffffffu, v, L), p.d, lane);
+                    if (lane == L) {
+                      const double yd = dot / nrm;
+                      neg = !(yd > 0.0);
+                      const double ad = fabs(yd);
+                      int mm = 0;
 #pragma unroll
-                    for (int k = 0; k < (1 << (BITS - 1)) - 1; ++k) mm += (double)P[k] < ad ? 1 : 0;
-                    m = mm;
-                    y = (float)yd;
+                      for (int k = 0; k < (1 << (BITS - 1)) - 1; ++k) mm += (double)P[k] < ad ? 1 : 0;
+                      m = mm;
+                      y = (float)yd;
+                    }
                   }
                 }
               }
-            }
 #pragma unroll
-            for (int pl = 0; pl < BITS; ++pl) {
-              const bool bit = pl == BITS - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
-              words[pl] |= (bit ? 1u : 0u) << j;
+              for (int pl = 0; pl < BITS; ++pl) {
+                const bool bit = pl == BITS - 1 ? !neg : ((((m >> pl) & 1) != 0) != neg);
+                words[pl] |= (bit ? 1u : 0u) << j;
+              }
+              if (ALG2) {
+                const float cm = sym_c<BITS>(m, C);
+                float rr = neg ? y + cm : y - cm;
+                if (inv == 0.0f) rr = 0.0f;
+                g2 = fma((double)rr, (double)rr, g2);
+                rho[jj] = rr;
+              }
             }
             if (ALG2) {
-              const float cm = sym_c<BITS>(m, C);
-              float rr = neg ? y + cm : y - cm;
-              if (inv == 0.0f) rr = 0.0f;
-              g2 = fma((double)rr, (double)rr, g2);
-              rho[j] = rr;
-            }
-          }
-          if (ALG2) {
-            // rho * 2^14 as hi + 2^-12 lo fp16 into the rho image (block kb, elements e0 .. e0+31)
-            const int i0 = nb * 128 + g * 32;
-            uint8_t* blk = slot + (size_t)(i0 >> 6) * 2 * kBlk;
-            const int e0 = i0 & 63;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
+              // rho * 2^14 as hi + 2^-12 lo fp16 into the rho image (block i0 / 64, 16 bytes at
+              // element (i0 mod 64) + 8 kq of this vector's row)
+              uint8_t* blk = slot + (size_t)(i0 >> 6) * 2 * kBlk;
               uint32_t h[4], l[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                const float a = rho[8 * k + 2 * u] * kRhoScaleT, b = rho[8 * k + 2 * u + 1] * kRhoScaleT;
+                const float a = rho[2 * u] * kRhoScaleT, b = rho[2 * u + 1] * kRhoScaleT;
                 const __half2 hh = __floats2half2_rn(a, b);
                 const float2 back = __half22float2(hh);
                 h[u] = h2_bits(hh);
                 l[u] = h2_bits(__floats2half2_rn((a - back.x) * kSplitScale, (b - back.y) * kSplitScale));
               }
-              const uint32_t off = sw128_offset(r, ((e0 >> 3) + k) * 16, 128);
+              const uint32_t off = sw128_offset(r, (((i0 & 63) >> 3) + kq) * 16, 128);
               *(uint4*)(blk + off) = make_uint4(h[0], h[1], h[2], h[3]);
               *(uint4*)(blk + kBlk + off) = make_uint4(l[0], l[1], l[2], l[3]);
             }
@@ -756,34 +755,36 @@ __global__ void __launch_bounds__(kTThreads, 1)
           tc_fence_after();
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {
-            uint32_t hi[32], lo[32];
-            const uint32_t col = tbase + lane_base + acc * 256 + g * 32;
-            tmem_ld16(col, *(uint32_t(*)[16]) & hi[0]);
-            tmem_ld16(col + 16, *(uint32_t(*)[16]) & hi[16]);
-            tmem_ld16(col + 128, *(uint32_t(*)[16]) & lo[0]);
-            tmem_ld16(col + 144, *(uint32_t(*)[16]) & lo[16]);
-            tmem_ld_wait();
             uint32_t w = 0;
+#pragma unroll 1
+            for (int kq = 0; kq < 4; ++kq) {            // coordinates g 32 + 8 kq .. + 7 of the band
+              uint32_t hi[8], lo[8];
+              const uint32_t col = tbase + lane_base + acc * 256 + g * 32 + 8 * kq;
+              tmem_ld8(col, hi);
+              tmem_ld8(col + 128, lo);
+              tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float sv = fmaf(__uint_as_float(lo[j]), kSplitScaleInv, __uint_as_float(hi[j]));
-              bool bit = sv >= 0.0f;
-              // next to zero: decide on the exact fp64 value (the residual's own rounding included),
-              // computed by the whole warp for each lane that needs one
-              uint32_t nm = __ballot_sync(0xffffffffu, live && fabsf(sv) < tau_s);
-              if (nm) {
-                const int jg = nb * 128 + g * 32 + j;
-                while (nm) {
-                  const int L = __ffs(nm) - 1;
-                  nm &= nm - 1;
-                  const int64_t vl = __shfl_sync(0xffffffffu, v, L);
-                  const double val = warp_sign_value<F32, BITS>(
-                      p.s32 + (size_t)jg * p.d, p.t32 + (size_t)jg * p.d, p.x, vl, p.d, __shfl_sync(0xffffffffu, nrm, L),
-                      p.codes + (size_t)vl * G * BITS, c_tab, lane);
-                  if (lane == L) bit = val >= 0.0;
+              for (int jj = 0; jj < 8; ++jj) {
+                const int j = 8 * kq + jj;
+                const float sv = fmaf(__uint_as_float(lo[jj]), kSplitScaleInv, __uint_as_float(hi[jj]));
+                bool bit = sv >= 0.0f;
+                // next to zero: decide on the exact fp64 value (the residual's own rounding
+                // included), computed by the whole warp for each lane that needs one
+                uint32_t nm = __ballot_sync(0xffffffffu, live && fabsf(sv) < tau_s);
+                if (nm) {
+                  const int jg = nb * 128 + g * 32 + j;
+                  while (nm) {
+                    const int L = __ffs(nm) - 1;
+                    nm &= nm - 1;
+                    const int64_t vl = __shfl_sync(0xffffffffu, v, L);
+                    const double val = warp_sign_value<F32, BITS>(
+                        p.s32 + (size_t)jg * p.d, p.t32 + (size_t)jg * p.d, p.x, vl, p.d,
+                        __shfl_sync(0xffffffffu, nrm, L), p.codes + (size_t)vl * G * BITS, c_tab, lane);
+                    if (lane == L) bit = val >= 0.0;
+                  }
                 }
+                w |= (bit ? 1u : 0u) << j;
               }
-              w |= (bit ? 1u : 0u) << j;
             }
             if (live) p.signs[(size_t)v * G + 4 * nb + g] = w;
           }
