@@ -627,7 +627,7 @@ def run_ours(args):
     return 0
 
 
-def _timed(fn, iters, warmup=2):
+def _timed(fn, iters, warmup=3):
     """Mean device time (ms) of fn() over `iters` calls on the current stream (CUDA events)."""
     import torch
     for _ in range(warmup):
@@ -787,12 +787,12 @@ def extra_workloads(dev, peak_hbm, peak_tensor):
     cb3 = tq.tq_codebook_init(d, 3)
     c, sg, nn, gm = tq.empty_prod(n, d, 4, dev)
     ws = torch.empty(max(16, tq.tq_encode_workspace_bytes(n, d, 2)), dtype=torch.uint8, device=dev)
-    ms_enc = _timed(lambda: tq.tq_encode_prod(cb3, X, rotv, c, sg, nn, gm, ws=ws), 2, warmup=1)
+    ms_enc = _timed(lambda: tq.tq_encode_prod(cb3, X, rotv, c, sg, nn, gm, ws=ws), 3)
     ids = torch.empty((nq, k), dtype=torch.int32, device=dev)
     sc = torch.empty((nq, k), dtype=torch.float32, device=dev)
     wss = torch.empty(max(16, tq.tq_scores_workspace_bytes(nq, n, d, k)), dtype=torch.uint8, device=dev)
     ms_sc = _timed(lambda: tq.tq_scores(cb3, qv, rotv, c, nn, signs=sg, gammas=gm, k=k, topk_ids=ids,
-                                        topk_scores=sc, ws=wss), 3, warmup=1)
+                                        topk_scores=sc, ws=wss), 3)
     tq.tq_sync_check()
     # algorithmic flops: encode 2 d^2 (Pi x) + 2 d^2 (T rho) per vector; scores 2 d (<q', c>) + 2 d
     # (<q'', z>) per (query, vector). Issued: the tiled encoder's split products (2 or 3 for Pi x with
