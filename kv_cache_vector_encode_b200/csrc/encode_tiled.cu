@@ -91,8 +91,7 @@ enum TBars {
 };
 
 // P[k] for 0 <= k < H - 1, as a tree of selects on the bits of k: with no indexed access to P the
-// compiler keeps the boundaries in registers (an indexed form placed them in local memory, whose
-// loads missed the small L1 left beside this kernel's shared memory).
+// compiler keeps the boundaries in registers (an indexed form placed them in local memory).
 template <int BITS>
 __device__ __forceinline__ float sym_p(int k, const float (&P)[8]) {
   if (BITS <= 2) return P[0];
