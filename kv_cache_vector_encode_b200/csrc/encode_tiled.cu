@@ -19,7 +19,7 @@
 // Precision: products exact in the tensor core, fp32 accumulation over K = d. For large d the
 // accumulated rounding approaches the parity band, so a decision whose value lies within 20x the
 // band of a boundary (a quantiser boundary, or zero for a sign) is recomputed exactly in fp64 from
-// the fp32 matrices -- rare (about 1e-4 of the coordinates) and off the fast path. The same holds
+// the fp32 matrices -- rare (below 1e-3 of the decisions at d = 1536) and off the fast path. The same holds
 // for the fp16 rounding of gamma = |r|: a gamma within 2^-15 (relative) of an fp16 rounding
 // midpoint, far wider than the fp32 accumulation error, is flagged, and a fix-up kernel recomputes
 // r = x / |x| - Pi^T c[idx] for that vector in fp64 from x, the fp32 Pi and the vector's own codes,
