@@ -19,12 +19,12 @@
 // Precision: products exact in the tensor core, fp32 accumulation over K = d. For large d the
 // accumulated rounding approaches the parity band, so a decision whose value lies within 20x the
 // band of a boundary (a quantiser boundary, or zero for a sign) is recomputed exactly in fp64 from
-// the fp32 matrices -- rare (below 1e-3 of the decisions at d = 1536) and off the fast path. The same holds
-// for the fp16 rounding of gamma = |r|: a gamma within 2^-15 (relative) of an fp16 rounding
-// midpoint, far wider than the fp32 accumulation error, is flagged, and a fix-up kernel recomputes
-// r = x / |x| - Pi^T c[idx] for that vector in fp64 from x, the fp32 Pi and the vector's own codes,
-// and rewrites gamma (about 9 % of the vectors; d^2 fp64 operations each, one pass over Pi serving
-// a batch of eight).
+// the fp32 matrices -- rare (below 1e-3 of the decisions at d = 1536) and off the fast path. The
+// same holds for the fp16 rounding of gamma = |r|: a gamma within 2^-15 (relative) of an fp16
+// rounding midpoint, far wider than the fp32 accumulation error, is flagged, and a fix-up kernel
+// recomputes r = x / |x| - Pi^T c[idx] for that vector in fp64 from x, the fp32 Pi and the vector's
+// own codes, and rewrites gamma (about 9 % of the vectors; d^2 fp64 operations each, one pass over
+// Pi serving a batch of eight).
 //
 // Roles (10 warps): 0 TMA / bulk copies; 1 TMEM owner and MMA issuer; 2-5 converters (thread =
 // vector: fp64 norm, fp16 split of x, copies of the rho images); 6-9 epilogue (thread = vector).
